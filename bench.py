@@ -1,0 +1,501 @@
+"""Benchmark of the ExpertsInt8 MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jmoe|reference]
+
+A step is one pass of the per-token hot path -- router (logits, softmax,
+top-2), grouping by expert, gate/up GEMM with in-kernel INT8->BF16
+dequantisation and SwiGLU, down GEMM, gate-weighted combine -- over one batch
+of synthetic tokens, with the weights (quantised once at load time, as the
+method prescribes) resident in HBM.  The headline workload is the
+Jamba-1.5-Mini-shaped decode batch (T = 8 tokens, d_model 4096, d_ff 14336,
+16 experts, top-2); the other workloads are reported under "also".
+
+With N > 1 (torchrun), every rank runs its own independent batch (the layer
+is per-token: no data-path collective) and rank 0 prints the aggregate.
+
+--impl reference times the CPU oracle on this machine's host cores on a
+bounded sample of the same workload (the pages ship no code to run).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DENSE,  # noqa: E402
+                             MINI_PREFILL, SIGMA_R, SIGMA_W, SIGMA_X, TINY, Workload)
+
+HEADLINE = MINI_DECODE
+METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 roofline"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.02):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            uuid = getattr(props, "uuid", None)
+            h = None
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device)
+            self.handle = h
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # NVML unavailable: report it
+            self.error = str(exc)
+
+    def run(self):
+        if self.handle is None:
+            return
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+                self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        self.join(timeout=2)
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"]}
+        reasons = [name for bit, name in self.NAMES.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- device layer
+
+
+class Layer:
+    """One MoE layer's device tensors: seeded inputs, weights quantised once."""
+
+    def __init__(self, wl: Workload, device):
+        import torch
+
+        import int8_weight_moe_b200 as jm
+
+        self.wl, self.device = wl, device
+        s, E, d, f = wl.seed, wl.E, wl.d_model, wl.d_ff
+        self.x = synth.normal_bf16_gpu(s, synth.X, SIGMA_X, (wl.T, d), device=device)
+        self.w_router = None if wl.dense else synth.normal_f32_gpu(s, synth.WR, SIGMA_R, (E, d),
+                                                                   device=device)
+        self.bias = (torch.tensor(wl.bias, dtype=torch.float32, device=device)
+                     if wl.bias is not None else None)
+        w = synth.normal_bf16_gpu(s, synth.WGU, SIGMA_W, (E, 2 * f, d), device=device)
+        self.w_gu, self.s_gu = jm.jmoe_quantize(w)
+        del w
+        w = synth.normal_bf16_gpu(s, synth.WD, SIGMA_W, (E, d, f), device=device)
+        self.w_d, self.s_d = jm.jmoe_quantize(w)
+        del w
+        torch.cuda.synchronize(device)
+        self.desc = jm.make_desc(self.w_gu, self.s_gu, self.w_d, self.s_d, top_k=wl.top_k)
+        self.out = torch.empty_like(self.x)
+        if wl.dense:
+            self.ws = torch.empty(jm.jmoe_mlp_workspace_size(wl.T, d, f), dtype=torch.uint8,
+                                  device=device)
+        else:
+            self.ids = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device=device)
+            self.gates = torch.empty((wl.T, wl.top_k), dtype=torch.float32, device=device)
+            self.ws = torch.empty(jm.jmoe_forward_workspace_size(self.desc, wl.T),
+                                  dtype=torch.uint8, device=device)
+
+    def step(self, x=None, out=None):
+        """One pass of the hot path on the current stream; returns #kernel launches."""
+        import int8_weight_moe_b200 as jm
+
+        x = self.x if x is None else x
+        out = self.out if out is None else out
+        if self.wl.dense:
+            jm.jmoe_mlp_forward(x, self.w_gu[0], self.s_gu[0], self.w_d[0], self.s_d[0], out=out,
+                                workspace=self.ws)
+            # fill (unit gates), grouping, gate/up, down, combine/finalize (+ gather on the
+            # tensor-core path)
+            return 6 if self.prefill_path() else 5
+        jm.jmoe_route(x, self.w_router, self.wl.top_k, self.bias, topk_ids=self.ids,
+                      topk_w=self.gates)
+        jm.jmoe_forward(self.desc, x, self.ids, self.gates, out=out, workspace=self.ws)
+        return 6 if self.prefill_path() else 5
+
+    def prefill_path(self):
+        """Whether the library's automatic choice is the tensor-core path here
+        (the two paths need different workspaces, which reveals the choice)."""
+        import int8_weight_moe_b200 as jm
+
+        return jm.uses_prefill_path(self.desc, self.wl.T)
+
+    def touched_experts(self):
+        if self.wl.dense:
+            return 1
+        return int(np.unique(self.ids.cpu().numpy()).size)
+
+    def weight_bytes(self):
+        return self.w_gu.numel() + self.w_d.numel()
+
+
+def kernel_work(layer: Layer):
+    """Algorithmic work of the dominant kernel (gate/up stage) per launch, and
+    of the whole step: bytes for the HBM-bound regime, FLOPs for prefill."""
+    wl = layer.wl
+    d, f, A, T = wl.d_model, wl.d_ff, wl.A, wl.T
+    touched = layer.touched_experts()
+    gu_bytes = touched * 2 * f * (d + 4) + A * d * 2 + A * f * 2
+    step_bytes = touched * 3 * d * f + touched * (2 * f + d) * 4 + T * d * 2 * 2
+    return {"touched": touched, "gate_up_bytes": gu_bytes, "step_bytes": step_bytes,
+            "gate_up_flops": 4 * A * d * f, "step_flops": 6 * A * d * f}
+
+
+def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: bool = True):
+    """Warm-up, then exactly `steps` timed steps between barriers; per-stage
+    CUDA events recorded live on the launching stream."""
+    import torch
+
+    import int8_weight_moe_b200 as jm
+
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    stage_events = []
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    start.record()
+    for _ in range(steps):
+        if profile:
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+            jm.jmoe_profile_events(evs)
+            stage_events.append(evs)
+        launches += layer.step()
+    stop.record()
+    jm.jmoe_profile_events(None)
+    torch.cuda.synchronize()
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    stages = {}
+    for i, name in enumerate(jm.STAGES):
+        times = []
+        for evs in stage_events:
+            try:
+                times.append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
+            except RuntimeError:
+                pass  # this stage did not run on this path
+        if times:
+            stages[name] = sum(times) / len(times)
+    return total_ms, stages, launches
+
+
+def roofline_entry(layer: Layer, stages: dict, peaks: dict, traffic=None):
+    work = kernel_work(layer)
+    ms = stages.get("gate_up")
+    if ms is None or ms <= 0:
+        return None
+    if layer.prefill_path():
+        achieved = work["gate_up_flops"] / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        return {"bound": "tensor", "kernel": "gate_up", "achieved": round(achieved, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": traffic, "ms": round(ms, 4),
+                "peak_source": peaks["source"] + " sustained bf16"}
+    achieved = work["gate_up_bytes"] / (ms * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "kernel": "gate_up", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+            "ms": round(ms, 4), "peak_source": peaks["source"] + " hbm copy"}
+
+
+def e2e_run(layer: Layer, steps: int, warmup: int):
+    """Same metric through the public API with host buffers: per step a
+    host->device copy of the tokens from pinned memory and a device->host read
+    of the layer output, inside the timed region."""
+    import torch
+
+    wl = layer.wl
+    xh = layer.x.cpu().pin_memory()
+    oh = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    xd = torch.empty_like(layer.x)
+    for _ in range(warmup):
+        xd.copy_(xh, non_blocking=True)
+        layer.step(x=xd)
+        oh.copy_(layer.out, non_blocking=True)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        xd.copy_(xh, non_blocking=True)
+        layer.step(x=xd)
+        oh.copy_(layer.out, non_blocking=True)
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / steps
+    nbytes = wl.T * wl.d_model * 2
+    return {"value": round(wl.T / (ms * 1e-3), 1), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_threads():
+    if os.environ.get("OMP_NUM_THREADS"):
+        return int(os.environ["OMP_NUM_THREADS"])
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+class OracleRun:
+    """The CPU oracle on a sample of a workload's tokens (weights generated
+    and quantised on the host for the experts the sample touches)."""
+
+    def __init__(self, wl: Workload, tokens):
+        import oracle
+
+        self.o = oracle
+        self.wl = wl
+        s, E, d, f = wl.seed, wl.E, wl.d_model, wl.d_ff
+        self.tokens = np.asarray(tokens)
+        self.x = synth.normal_bf16_bits(s, synth.X, SIGMA_X, (wl.T, d))[self.tokens]
+        self.wr = None if wl.dense else synth.normal_f32(s, synth.WR, SIGMA_R, (E, d))
+        self.bias = None if wl.bias is None else np.array(wl.bias, dtype=np.float32)
+        if wl.dense:
+            ids = np.zeros((len(self.tokens), 1), dtype=np.int32)
+        else:
+            _, ids, _ = oracle.route(self.x, self.wr, wl.top_k, self.bias)
+        self.tables = [[None] * E for _ in range(4)]
+        for e in sorted(set(int(v) for v in ids.reshape(-1))):
+            wgu = synth.normal_bf16_bits(s, synth.WGU, SIGMA_W, (2 * f, d), start=e * 2 * f * d)
+            qg, sg = oracle.quantize(wgu)
+            del wgu
+            wdn = synth.normal_bf16_bits(s, synth.WD, SIGMA_W, (d, f), start=e * d * f)
+            qd, sd = oracle.quantize(wdn)
+            del wdn
+            for i, a in enumerate((qg, sg, qd, sd)):
+                self.tables[i][e] = a
+
+    def step(self):
+        """Route, group and run the experts for the sample; returns #tokens."""
+        if self.wl.dense:
+            e = 0
+            self.o.mlp_forward(self.x, self.tables[0][e], self.tables[1][e], self.tables[2][e],
+                               self.tables[3][e])
+        else:
+            _, ids, g = self.o.route(self.x, self.wr, self.wl.top_k, self.bias)
+            self.o.permute(ids, self.wl.E)
+            self.o.moe_forward(self.x, ids, g, *self.tables)
+        return len(self.tokens)
+
+
+def cpu_baseline(wl: Workload, budget_s: float = 12.0):
+    run = OracleRun(wl, np.arange(min(wl.T, 8)))
+    t0 = time.perf_counter()
+    n = 0
+    reps = 0
+    while True:
+        n += run.step()
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 3), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{wl.name}: {len(run.tokens)} tokens x {reps} repetitions "
+                      f"(route + group + experts, fp64 C oracle), {dt:.1f} s"}
+
+
+def reference_arm(args):
+    """--impl reference: the oracle on the host cores, on the headline config."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = HEADLINE
+    run = OracleRun(wl, np.arange(1))  # one token (two expert assignments) per step
+    for _ in range(args.warmup):
+        run.step()
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(args.steps):
+        n += run.step()
+    dt = time.perf_counter() - t0
+    value = n / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**wl.describe(), "sample_tokens_per_step": 1},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle_threads(),
+                             "kind": "oracle",
+                             "sample": f"{wl.name}: 1 token per step (route + group + 2 experts)"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="jmoe", choices=["jmoe", "reference"])
+    ap.add_argument("--no-also", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--only", default=None, help="run only this workload (name) as headline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import int8_weight_moe_b200 as jm
+
+    peaks = load_peaks()
+    wl = HEADLINE
+    if args.only:
+        from synth.workloads import BY_NAME
+
+        wl = BY_NAME[args.only]
+    layer = Layer(wl, torch.device("cuda", local))
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, stages, launches = timed_run(layer, args.steps, args.warmup, dist_on)
+    clocks = sampler.stop()
+    if dist_on:
+        import torch.distributed as dist
+
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / args.steps
+    value = world * wl.T / (ms * 1e-3)
+    roof = roofline_entry(layer, stages, peaks)
+    e2e = e2e_run(layer, max(args.steps // 2, 10), 3)
+    e2e["value"] = round(e2e["value"] * world, 1)
+    work = kernel_work(layer)
+    step_gbs = work["step_bytes"] / (ms * 1e-3) / 1e9
+    del layer
+    torch.cuda.empty_cache()
+
+    also = []
+    if not args.no_also and not args.only:
+        for other in (TINY, MINI_PREFILL, MINI_DENSE, LARGE_DECODE, LARGE_PREFILL_SKEW):
+            lay = Layer(other, torch.device("cuda", local))
+            steps = 20 if other.regime == "prefill" else 100
+            tms, st, _ = timed_run(lay, steps, 3, dist_on)
+            oms = tms / steps
+            w2 = kernel_work(lay)
+            entry = {"workload": other.name, "tokens_per_s": round(other.T / (oms * 1e-3), 1),
+                     "ms_per_step": round(oms, 4), "path": "prefill" if lay.prefill_path() else "decode",
+                     "stages_ms": {k: round(v, 4) for k, v in st.items()},
+                     "roofline": roofline_entry(lay, st, peaks),
+                     "step_hbm_gbs": round(w2["step_bytes"] / (oms * 1e-3) / 1e9, 1),
+                     "step_tflops": round(w2["step_flops"] / (oms * 1e-3) / 1e12, 2)}
+            also.append(entry)
+            del lay
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {**wl.describe(),
+                           "weights": "int8 per-output-channel (quantised once on device)",
+                           "l2": "inputs larger than L2 (touched int8 weights "
+                                 f"{work['touched'] * 3 * wl.d_model * wl.d_ff / 1e9:.2f} GB "
+                                 "> 126 MB L2), no flush",
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clocks,
+                "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+                "step_hbm_gbs": round(step_gbs, 1),
+                "touched_experts": work["touched"], "also": also}
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

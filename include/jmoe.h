@@ -1,0 +1,181 @@
+/*
+ * jmoe -- the ExpertsInt8 mixture-of-experts layer on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libjmoe.so.  Plain pointers and sizes only; no CUDA or PyTorch
+ * types appear in the signatures.  A `stream` argument is a cudaStream_t
+ * passed as `void*` (NULL = the legacy default stream).
+ *
+ * The method (sources cited by page title and section):
+ *  - "Jamba-1.5: Hybrid Transformer-Mamba Models at Scale" (paper summary,
+ *    arXiv 2408.12570), section "ExpertsInt8 Quantization (Section 3.1)":
+ *    step 1, MoE and MLP weights are quantised BF16 -> INT8 once at load time
+ *    without calibration; step 2, they are stored as INT8; step 3, they are
+ *    dequantised back to BF16 inside the fused MoE kernel as they move from
+ *    HBM to on-chip memory; step 4, activations stay BF16.
+ *  - same page, section "The Jamba Hybrid Block Structure": the MoE layer
+ *    output MoE(x) = sum over the top-2 experts of g_i(x) * Expert_i(x),
+ *    16 experts.
+ *  - "Jamba: A Hybrid Transformer-Mamba Language Model" (paper summary,
+ *    arXiv 2403.19887), section "Mixture-of-Experts (MoE) in Jamba: Router,
+ *    Top-K, and Load Balancing": g = softmax(W_r h), top-K selection, and
+ *    y = sum over the selected set of g_i * Expert_i(h) with g renormalised
+ *    over the selected set; its layer list: experts are MLPs with SwiGLU.
+ *
+ * Conventions shared by every call:
+ *  - Ownership: the caller owns every buffer.  The library never allocates,
+ *    frees or synchronises on these calls (jmoe_last_error excepted); all
+ *    work is enqueued on `stream` in order and may be captured in a CUDA graph.
+ *  - Layouts are row-major.  A weight row is one output channel and its
+ *    elements run along the input dimension (the contraction dimension is
+ *    contiguous).  bf16 buffers hold IEEE bfloat16 bit patterns.
+ *  - Pointers named *device* must be device-accessible CUDA allocations and
+ *    16-byte aligned; d_model and d_ff must be multiples of 64.
+ *  - Argument and shape errors return a status before anything is launched.
+ *    A failed launch returns JMOE_ECUDA.  Conditions only the device can see
+ *    (an expert id out of range, a bounded wait that ran out) set a sticky
+ *    device error word that jmoe_last_error() reports; kernels never trap.
+ *  - Non-finite inputs are outside the contract and are not checked.
+ */
+#ifndef JMOE_H
+#define JMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JMOE_OK = 0,
+    JMOE_EINVAL = 1,       /* a null pointer, a negative size, an out-of-range count */
+    JMOE_EALIGN = 2,       /* a pointer is not 16-byte aligned */
+    JMOE_EUNSUPPORTED = 3, /* a shape or option this build does not implement */
+    JMOE_EWORKSPACE = 4,   /* workspace smaller than the size query returned */
+    JMOE_ECUDA = 5,        /* a CUDA runtime call or launch failed */
+    JMOE_ETIMEOUT = 6,     /* (device word) a bounded wait inside a kernel ran out */
+    JMOE_EDEVICE = 7       /* (device word) a kernel saw an invalid expert id */
+} jmoe_status;
+
+/* Which expert-GEMM kernels jmoe_forward / jmoe_mlp_forward use. */
+typedef enum {
+    JMOE_PATH_AUTO = 0,    /* decode kernels for few assignments, else tensor-core kernels */
+    JMOE_PATH_DECODE = 1,  /* bandwidth-bound GEMV-like kernels (any size; slow when large) */
+    JMOE_PATH_PREFILL = 2  /* tcgen05 / TMEM grouped GEMM kernels */
+} jmoe_path;
+
+/* The quantised expert weights of one MoE layer (all device pointers).
+ *   w_gu : int8  [E][2*d_ff][d_model]  rows 0..d_ff-1 of each expert are the
+ *          gate projection, rows d_ff..2*d_ff-1 the up projection
+ *   s_gu : fp32  [E][2*d_ff]           one scale per row of w_gu
+ *   w_d  : int8  [E][d_model][d_ff]    down projection
+ *   s_d  : fp32  [E][d_model]          one scale per row of w_d
+ * A row's dequantised weights are q * s (ExpertsInt8 step 3). */
+typedef struct {
+    int32_t E;       /* number of experts, 1..16 */
+    int32_t top_k;   /* experts per token, 1 or 2, <= E */
+    int64_t d_model; /* hidden size, multiple of 64 */
+    int64_t d_ff;    /* expert intermediate size, multiple of 64 */
+    const int8_t* w_gu;
+    const float* s_gu;
+    const int8_t* w_d;
+    const float* s_d;
+    int32_t path;    /* a jmoe_path value */
+} jmoe_moe_desc;
+
+/* ExpertsInt8 step 1 (load-time, calibration-free quantisation).
+ * w_bf16 : device, bf16 [rows][cols], row = output channel
+ * q      : device, int8 [rows][cols]   (written)
+ * scales : device, fp32 [rows]         (written)
+ * Per row: a = max |w|; s = a / 127 (one correctly rounded fp32 division);
+ * q = round-half-even(w / s) (one fp32 division per element) clamped to
+ * [-127, 127]; an all-zero row gets s = 0, q = 0.  cols must be a multiple
+ * of 8 (16-byte rows of bf16); rows >= 0 (0 is a no-op). */
+jmoe_status jmoe_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t* q,
+                          float* scales, void* stream);
+
+/* Router (Jamba summary, "Router mechanism" and "Top-K selection").
+ * x_bf16   : device, bf16 [T][d]
+ * w_router : device, fp32 [E][d]
+ * bias     : device, fp32 [E] added to the logits, or NULL (the pages' router
+ *            has no bias; it exists to build skewed-routing workloads)
+ * topk_ids : device, int32 [T][top_k] (written) largest logit first, ties to
+ *            the lower expert index
+ * topk_w   : device, fp32 [T][top_k]  (written) softmax probabilities of the
+ *            selected experts renormalised to sum to 1 (1.0 when top_k = 1)
+ * logits   : device, fp32 [T][E] (written) or NULL
+ * Logits are fp64 dot products summed in a fixed order (lane j of 32 sums
+ * the elements k = j mod 32 in ascending k, then a halving tree over the 32
+ * lanes), plus the bias, rounded once to fp32; selection uses these fp32
+ * logits, so ids are reproducible bit for bit.  E in 1..16, top_k in {1,2},
+ * d a multiple of 64, T >= 0. */
+jmoe_status jmoe_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
+                       const float* bias, int32_t E, int32_t top_k, int32_t* topk_ids,
+                       float* topk_w, float* logits, void* stream);
+
+/* Grouping of the T*top_k token->expert assignments by expert (the dispatch
+ * step the fused MoE kernel performs; Jamba-1.5 summary, "Innovation 2").
+ * Assignment a = t*top_k + j.  offsets: device int32 [E+1] (written),
+ * exclusive prefix of the per-expert counts (offsets[E] = T*top_k); perm:
+ * device int32 [T*top_k] (written), the assignments of expert 0 in
+ * ascending a, then expert 1, ...; inv: device int32 [T*top_k] (written),
+ * inv[perm[i]] = i.  Deterministic and bit-exact.  An id outside [0, E)
+ * sets JMOE_EDEVICE in the device error word and the assignment is dropped.
+ * A single thread block does the work (T*top_k up to 2^24). */
+jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int32_t E,
+                         int32_t* offsets, int32_t* perm, int32_t* inv, void* stream);
+
+/* Workspace bytes jmoe_forward needs for T tokens with this descriptor. */
+jmoe_status jmoe_forward_workspace_size(const jmoe_moe_desc* desc, int64_t T, size_t* bytes);
+
+/* The MoE layer forward (ExpertsInt8 steps 3-4 with the MoE equation).
+ * x_bf16   : device, bf16 [T][d_model]
+ * topk_ids : device, int32 [T][top_k] (from jmoe_route or the caller)
+ * topk_w   : device, fp32 [T][top_k]
+ * out_bf16 : device, bf16 [T][d_model] (written)
+ * workspace: device, >= jmoe_forward_workspace_size bytes, 256-byte aligned
+ * out_t = sum_j topk_w[t][j] * Expert_{topk_ids[t][j]}(x_t), where
+ * Expert_e(x) = W_d (silu(W_g x) * (W_u x)) with W = q * s.  The hidden
+ * activation between the two projections is stored as bf16 and every dot
+ * product accumulates in fp32.  T >= 0 (0 is a no-op). */
+jmoe_status jmoe_forward(const jmoe_moe_desc* desc, const void* x_bf16, int64_t T,
+                         const int32_t* topk_ids, const float* topk_w, void* out_bf16,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes jmoe_mlp_forward needs. */
+jmoe_status jmoe_mlp_workspace_size(int64_t T, int64_t d_model, int64_t d_ff, int32_t path,
+                                    size_t* bytes);
+
+/* The dense SwiGLU MLP with INT8 weights (ExpertsInt8 quantises "MoE and
+ * MLP weights"): out_t = Expert(x_t) with one expert (E = 1, gate 1).
+ * w_gu int8 [2*d_ff][d_model], s_gu fp32 [2*d_ff], w_d int8 [d_model][d_ff],
+ * s_d fp32 [d_model]; other arguments as jmoe_forward. */
+jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int64_t d_ff,
+                             const int8_t* w_gu, const float* s_gu, const int8_t* w_d,
+                             const float* s_d, void* out_bf16, void* workspace,
+                             size_t ws_bytes, int32_t path, void* stream);
+
+/* Stage timing hook (diagnostics).  Registers `n` CUDA events (cudaEvent_t
+ * handles passed as void*) that the following jmoe_forward / jmoe_mlp_forward
+ * calls record on their stream around their kernels: events[2*i] before and
+ * events[2*i+1] after stage i, where the stages are 0 = grouping by expert,
+ * 1 = row gather (tensor-core path only), 2 = gate/up GEMM + SwiGLU,
+ * 3 = down GEMM, 4 = combine.  Stages that do not run record nothing.
+ * n = 0 or events = NULL switches recording off.  The registration is
+ * process-wide and not thread-safe; the caller keeps the events alive.
+ * n must be 0 or 10. */
+jmoe_status jmoe_profile_events(void* const* events, int32_t n);
+
+/* Reads and clears the device error word of the current device.  Unlike the
+ * other calls it synchronises the device.  Returns JMOE_OK when no kernel
+ * has flagged anything since the last call. */
+jmoe_status jmoe_last_error(void);
+
+/* A static, human-readable name for a status. */
+const char* jmoe_status_string(jmoe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JMOE_H */

@@ -1,0 +1,344 @@
+// C ABI of libjmoe.so (declared in include/jmoe.h): argument validation,
+// workspace layout and kernel dispatch.  Nothing here allocates, frees or
+// synchronises, except jmoe_last_error.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "../../include/jmoe.h"
+#include "kernels.h"
+#include "prefill.h"
+
+namespace {
+
+__device__ unsigned g_jmoe_err_word;
+
+constexpr int kMaxDevices = 64;
+constexpr int kStages = 5;
+cudaEvent_t g_stage_events[2 * kStages];
+std::atomic<bool> g_profile_on{false};
+std::atomic<unsigned*> g_err_ptr[kMaxDevices];
+std::atomic<int> g_num_sms[kMaxDevices];
+
+// Below this many token->expert assignments the decode (GEMV-like) kernels
+// run; at and above it the tcgen05 grouped GEMM.
+constexpr int64_t kDecodeMaxAssignments = 128;
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+unsigned* err_word() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    unsigned* p = g_err_ptr[dev].load();
+    if (!p) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_jmoe_err_word) != cudaSuccess) return nullptr;
+        p = static_cast<unsigned*>(addr);
+        g_err_ptr[dev].store(p);
+    }
+    return p;
+}
+
+int num_sms() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int n = g_num_sms[dev].load();
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_num_sms[dev].store(n);
+    }
+    return n;
+}
+
+void stage_mark(int stage, bool after, cudaStream_t s) {
+    if (g_profile_on.load(std::memory_order_relaxed))
+        cudaEventRecord(g_stage_events[2 * stage + (after ? 1 : 0)], s);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+jmoe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? JMOE_OK : JMOE_ECUDA; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Workspace carve-up shared by the size query and the forward calls.
+struct Workspace {
+    size_t offsets, padded_offsets, perm, inv;  // routing tables
+    size_t H, P;                                // decode path
+    size_t xperm, Hp, Yg;                       // tensor-core path
+    size_t total;
+    int nsplit;
+    int64_t rows_padded;  // upper bound of the padded expert-grouped rows
+};
+
+Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) {
+    Workspace w{};
+    size_t at = 0;
+    auto take = [&](size_t bytes) {
+        size_t off = at;
+        at = round_up(at + bytes, 256);
+        return off;
+    };
+    w.offsets = take(sizeof(int32_t) * (size_t)(E + 1));
+    w.padded_offsets = take(sizeof(int32_t) * (size_t)(E + 1));
+    w.perm = take(sizeof(int32_t) * (size_t)A);
+    w.inv = take(sizeof(int32_t) * (size_t)A);
+    (void)T;
+    if (!prefill) {
+        w.nsplit = jmoe::decode_split_for(f);
+        w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
+        w.P = take(sizeof(float) * (size_t)w.nsplit * (size_t)A * (size_t)d);
+    } else {
+        const int64_t tm = jmoe::kPrefillTileM;
+        w.rows_padded = (A + (int64_t)E * (tm - 1) + tm - 1) / tm * tm;
+        w.xperm = take(sizeof(uint16_t) * (size_t)w.rows_padded * (size_t)d);
+        w.Hp = take(sizeof(uint16_t) * (size_t)w.rows_padded * (size_t)f);
+        w.Yg = take(sizeof(float) * (size_t)A * (size_t)d);
+    }
+    w.total = at;
+    return w;
+}
+
+bool use_prefill(int32_t path, int64_t A) {
+    if (path == JMOE_PATH_DECODE) return false;
+    if (path == JMOE_PATH_PREFILL) return true;
+    return A >= kDecodeMaxAssignments && jmoe::prefill_available();
+}
+
+jmoe_status check_desc(const jmoe_moe_desc* desc) {
+    if (!desc) return JMOE_EINVAL;
+    if (desc->E < 1 || desc->E > 16) return JMOE_EUNSUPPORTED;
+    if (desc->top_k < 1 || desc->top_k > 2 || desc->top_k > desc->E) return JMOE_EUNSUPPORTED;
+    if (desc->d_model <= 0 || desc->d_ff <= 0) return JMOE_EINVAL;
+    if (desc->d_model % 64 || desc->d_ff % 64) return JMOE_EUNSUPPORTED;
+    if (desc->path < JMOE_PATH_AUTO || desc->path > JMOE_PATH_PREFILL) return JMOE_EINVAL;
+    if (!desc->w_gu || !desc->s_gu || !desc->w_d || !desc->s_d) return JMOE_EINVAL;
+    if (!aligned16(desc->w_gu) || !aligned16(desc->s_gu) || !aligned16(desc->w_d) ||
+        !aligned16(desc->s_d))
+        return JMOE_EALIGN;
+    return JMOE_OK;
+}
+
+// The expert MLPs over routed rows, shared by the MoE and dense entries.
+jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
+                        const int32_t* ids, const float* gates, void* out, void* ws,
+                        size_t ws_bytes, bool dense, cudaStream_t stream) {
+    const int E = desc->E, k = desc->top_k;
+    const int64_t A = T * k, d = desc->d_model, f = desc->d_ff;
+    const bool prefill = use_prefill(desc->path, A);
+    if (prefill && !jmoe::prefill_available()) return JMOE_EUNSUPPORTED;
+    const Workspace w = plan(T, A, E, d, f, prefill);
+    if (!ws || ws_bytes < w.total) return JMOE_EWORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return JMOE_EALIGN;
+    char* base = static_cast<char*>(ws);
+    auto at = [&](size_t off) { return static_cast<void*>(base + off); };
+    int32_t* offsets = static_cast<int32_t*>(at(w.offsets));
+    int32_t* poff = static_cast<int32_t*>(at(w.padded_offsets));
+    int32_t* perm = static_cast<int32_t*>(at(w.perm));
+    int32_t* inv = static_cast<int32_t*>(at(w.inv));
+    unsigned* err = err_word();
+    const int sms = num_sms();
+
+    stage_mark(0, false, stream);
+    cudaError_t e = jmoe::launch_permute(ids, A, E, jmoe::kPrefillTileM, offsets, poff, perm, inv,
+                                         err, stream);
+    stage_mark(0, true, stream);
+    if (e != cudaSuccess) return JMOE_ECUDA;
+    if (!prefill) {
+        jmoe::DecodeArgs a{};
+        a.x = x; a.T = T; a.A = A; a.d = d; a.f = f; a.E = E; a.top_k = k;
+        a.wgu = desc->w_gu; a.sgu = desc->s_gu; a.wd = desc->w_d; a.sd = desc->s_d;
+        a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm; a.inv = inv;
+        a.H = at(w.H); a.P = static_cast<float*>(at(w.P)); a.nsplit = w.nsplit;
+        a.max_per_expert = T;  // distinct experts per token: at most T rows each
+        a.out = out; a.num_sms = sms;
+        a.mark = stage_mark;
+        return from_cuda(jmoe::launch_decode(a, stream));
+    }
+    jmoe::PrefillArgs p{};
+    p.x = x; p.T = T; p.A = A; p.d = d; p.f = f; p.E = E; p.top_k = k;
+    p.wgu = desc->w_gu; p.sgu = desc->s_gu; p.wd = desc->w_d; p.sd = desc->s_d;
+    p.ids = ids; p.gates = gates; p.offsets = offsets; p.padded_offsets = poff; p.perm = perm;
+    p.inv = inv; p.xperm = at(w.xperm); p.H = at(w.Hp); p.Yg = static_cast<float*>(at(w.Yg));
+    p.rows_padded = w.rows_padded; p.out = out; p.num_sms = sms; p.err = err;
+    p.mark = stage_mark; p.dense = dense;
+    return from_cuda(jmoe::launch_prefill(p, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* jmoe_status_string(jmoe_status s) {
+    switch (s) {
+        case JMOE_OK: return "JMOE_OK";
+        case JMOE_EINVAL: return "JMOE_EINVAL: invalid argument";
+        case JMOE_EALIGN: return "JMOE_EALIGN: pointer not aligned";
+        case JMOE_EUNSUPPORTED: return "JMOE_EUNSUPPORTED: unsupported shape or option";
+        case JMOE_EWORKSPACE: return "JMOE_EWORKSPACE: workspace too small";
+        case JMOE_ECUDA: return "JMOE_ECUDA: CUDA call or launch failed";
+        case JMOE_ETIMEOUT: return "JMOE_ETIMEOUT: a bounded device wait ran out";
+        case JMOE_EDEVICE: return "JMOE_EDEVICE: invalid expert id seen on the device";
+    }
+    return "unknown jmoe_status";
+}
+
+jmoe_status jmoe_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t* q,
+                          float* scales, void* stream) {
+    if (rows < 0 || cols <= 0) return JMOE_EINVAL;
+    if (cols % 8) return JMOE_EUNSUPPORTED;
+    if (rows == 0) return JMOE_OK;
+    if (rows > 0x7fffffffLL) return JMOE_EUNSUPPORTED;
+    if (!w_bf16 || !q || !scales) return JMOE_EINVAL;
+    if (!aligned16(w_bf16) || !aligned16(q) || !aligned16(scales)) return JMOE_EALIGN;
+    return from_cuda(jmoe::launch_quantize(w_bf16, rows, cols, q, scales, (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
+                       const float* bias, int32_t E, int32_t top_k, int32_t* topk_ids,
+                       float* topk_w, float* logits, void* stream) {
+    if (T < 0 || d <= 0) return JMOE_EINVAL;
+    if (E < 1 || E > 16 || top_k < 1 || top_k > 2 || top_k > E) return JMOE_EUNSUPPORTED;
+    if (d % 64) return JMOE_EUNSUPPORTED;
+    if (T == 0) return JMOE_OK;
+    if (!x_bf16 || !w_router || !topk_ids || !topk_w) return JMOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(w_router) || !aligned16(topk_ids) || !aligned16(topk_w) ||
+        (bias && !aligned16(bias)) || (logits && !aligned16(logits)))
+        return JMOE_EALIGN;
+    return from_cuda(jmoe::launch_route(x_bf16, T, d, w_router, bias, E, top_k, topk_ids, topk_w,
+                                        logits, num_sms(), (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int32_t E,
+                         int32_t* offsets, int32_t* perm, int32_t* inv, void* stream) {
+    if (T < 0) return JMOE_EINVAL;
+    if (E < 1 || E > 16 || top_k < 1 || top_k > 2) return JMOE_EUNSUPPORTED;
+    if (T * top_k > (1LL << 24)) return JMOE_EUNSUPPORTED;
+    if (!offsets) return JMOE_EINVAL;
+    if (T > 0 && (!topk_ids || !perm || !inv)) return JMOE_EINVAL;
+    if (!aligned16(offsets) || (T > 0 && (!aligned16(topk_ids) || !aligned16(perm) ||
+                                          !aligned16(inv))))
+        return JMOE_EALIGN;
+    return from_cuda(jmoe::launch_permute(topk_ids, T * top_k, E, jmoe::kPrefillTileM, offsets,
+                                          nullptr, perm, inv, err_word(), (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_forward_workspace_size(const jmoe_moe_desc* desc, int64_t T, size_t* bytes) {
+    if (!bytes || !desc) return JMOE_EINVAL;
+    if (T < 0) return JMOE_EINVAL;
+    if (desc->E < 1 || desc->E > 16 || desc->top_k < 1 || desc->top_k > 2 ||
+        desc->top_k > desc->E)
+        return JMOE_EUNSUPPORTED;
+    if (desc->d_model <= 0 || desc->d_ff <= 0) return JMOE_EINVAL;
+    if (desc->d_model % 64 || desc->d_ff % 64) return JMOE_EUNSUPPORTED;
+    if (desc->path < JMOE_PATH_AUTO || desc->path > JMOE_PATH_PREFILL) return JMOE_EINVAL;
+    const int64_t A = T * desc->top_k;
+    *bytes = plan(T, A, desc->E, desc->d_model, desc->d_ff, use_prefill(desc->path, A)).total;
+    return JMOE_OK;
+}
+
+jmoe_status jmoe_forward(const jmoe_moe_desc* desc, const void* x_bf16, int64_t T,
+                         const int32_t* topk_ids, const float* topk_w, void* out_bf16,
+                         void* workspace, size_t ws_bytes, void* stream) {
+    jmoe_status st = check_desc(desc);
+    if (st != JMOE_OK) return st;
+    if (T < 0) return JMOE_EINVAL;
+    if (T == 0) return JMOE_OK;
+    if (T * desc->top_k > (1LL << 24)) return JMOE_EUNSUPPORTED;
+    if (!x_bf16 || !topk_ids || !topk_w || !out_bf16) return JMOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(out_bf16))
+        return JMOE_EALIGN;
+    return run_experts(desc, x_bf16, T, topk_ids, topk_w, out_bf16, workspace, ws_bytes, false,
+                       (cudaStream_t)stream);
+}
+
+jmoe_status jmoe_mlp_workspace_size(int64_t T, int64_t d_model, int64_t d_ff, int32_t path,
+                                    size_t* bytes) {
+    if (!bytes) return JMOE_EINVAL;
+    jmoe_moe_desc desc{};
+    desc.E = 1;
+    desc.top_k = 1;
+    desc.d_model = d_model;
+    desc.d_ff = d_ff;
+    desc.path = path;
+    size_t inner = 0;
+    const jmoe_status st = jmoe_forward_workspace_size(&desc, T, &inner);
+    if (st != JMOE_OK) return st;
+    // ids and gates tables of the single-expert routing, then the MoE workspace
+    *bytes = 2 * round_up(sizeof(float) * (size_t)(T > 0 ? T : 0), 256) + inner;
+    return JMOE_OK;
+}
+
+jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int64_t d_ff,
+                             const int8_t* w_gu, const float* s_gu, const int8_t* w_d,
+                             const float* s_d, void* out_bf16, void* workspace, size_t ws_bytes,
+                             int32_t path, void* stream) {
+    jmoe_moe_desc desc{};
+    desc.E = 1;
+    desc.top_k = 1;
+    desc.d_model = d_model;
+    desc.d_ff = d_ff;
+    desc.w_gu = w_gu;
+    desc.s_gu = s_gu;
+    desc.w_d = w_d;
+    desc.s_d = s_d;
+    desc.path = path;
+    jmoe_status st = check_desc(&desc);
+    if (st != JMOE_OK) return st;
+    if (T < 0) return JMOE_EINVAL;
+    if (T == 0) return JMOE_OK;
+    if (T > (1LL << 24)) return JMOE_EUNSUPPORTED;
+    if (!x_bf16 || !out_bf16) return JMOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(out_bf16)) return JMOE_EALIGN;
+    size_t need = 0;
+    st = jmoe_mlp_workspace_size(T, d_model, d_ff, path, &need);
+    if (st != JMOE_OK) return st;
+    if (!workspace || ws_bytes < need) return JMOE_EWORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return JMOE_EALIGN;
+    // The dense layer is the MoE machinery with one expert, every token
+    // routed to it with gate 1: ids (all 0) and gates (all 1) live at the
+    // front of the workspace, filled on the stream.
+    char* base = static_cast<char*>(workspace);
+    const size_t tbl = round_up(sizeof(float) * (size_t)T, 256);
+    int32_t* ids = reinterpret_cast<int32_t*>(base);
+    float* gates = reinterpret_cast<float*>(base + tbl);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemsetAsync(ids, 0, sizeof(int32_t) * (size_t)T, s) != cudaSuccess) return JMOE_ECUDA;
+    if (jmoe::launch_fill_f32(gates, 1.0f, T, s) != cudaSuccess) return JMOE_ECUDA;
+    return run_experts(&desc, x_bf16, T, ids, gates, out_bf16, base + 2 * tbl, ws_bytes - 2 * tbl,
+                       true, s);
+}
+
+jmoe_status jmoe_profile_events(void* const* events, int32_t n) {
+    if (n == 0 || events == nullptr) {
+        g_profile_on.store(false);
+        return JMOE_OK;
+    }
+    if (n != 2 * kStages) return JMOE_EINVAL;
+    for (int i = 0; i < n; ++i) {
+        if (!events[i]) return JMOE_EINVAL;
+        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    g_profile_on.store(true);
+    return JMOE_OK;
+}
+
+jmoe_status jmoe_last_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return JMOE_ECUDA;
+    unsigned* p = err_word();
+    if (!p) return JMOE_ECUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return JMOE_ECUDA;
+    if (v != 0 && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return JMOE_ECUDA;
+    if (v & jmoe::kErrBadExpert) return JMOE_EDEVICE;
+    if (v & jmoe::kErrTimeout) return JMOE_ETIMEOUT;
+    return JMOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// Device helpers shared by the jmoe kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+
+namespace jmoe {
+
+__device__ __forceinline__ void flag_error(unsigned* err, unsigned bit) {
+    if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// Two int8 values (bytes 0,1 or 2,3 of `w`) to a packed bf16x2, exactly.
+//
+// For a byte b (two's complement), let m = b & 0x7f and s = b & 0x80.  The
+// bf16 pattern 0x4300 | m is the number 128 + m (exponent 2^7, mantissa m),
+// and 0x4300 | s is 128 (s = 0) or 256 (s = 0x80).  Their difference is
+// m - 128*[s != 0] = b, which is exactly representable (|b| <= 128 needs 8
+// significant bits), so one round-to-nearest bf16x2 subtraction is exact.
+// Cost: one byte permute, two logic ops and one bf16x2 subtract per pair.
+template <int kHigh>
+__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w) {
+    // byte layout of t: [b_lo, 0x43, b_hi, 0x43] -> halves 0x43bb
+    const uint32_t t = __byte_perm(w, 0x43u, kHigh ? 0x4342u : 0x4140u);
+    const uint32_t v = t & 0xff7fff7fu;                // 0x43 | m  -> 128 + m
+    const uint32_t c = (t & 0x00800080u) | 0x43004300u;  // 128 or 256
+    __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v),
+                               *reinterpret_cast<const __nv_bfloat162*>(&c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// 16 bytes of int8 -> 8 packed bf16x2 words (element order preserved).
+__device__ __forceinline__ void i8x16_to_bf16x16(const uint4& q, uint32_t (&o)[8]) {
+    o[0] = i8x2_to_bf16x2<0>(q.x);
+    o[1] = i8x2_to_bf16x2<1>(q.x);
+    o[2] = i8x2_to_bf16x2<0>(q.y);
+    o[3] = i8x2_to_bf16x2<1>(q.y);
+    o[4] = i8x2_to_bf16x2<0>(q.z);
+    o[5] = i8x2_to_bf16x2<1>(q.z);
+    o[6] = i8x2_to_bf16x2<0>(q.w);
+    o[7] = i8x2_to_bf16x2<1>(q.w);
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Streaming load for weights that are read exactly once.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// D = A * B + D for one m16n8k16 tile, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float silu_f32(float z) {
+    return z / (1.0f + __expf(-z));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+}  // namespace jmoe

@@ -1,0 +1,63 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace jmoe {
+
+// Bits of the sticky device error word (see jmoe_last_error).
+enum : unsigned {
+    kErrTimeout = 1u,    // a bounded wait ran out
+    kErrBadExpert = 2u,  // an expert id outside [0, E)
+};
+
+// Rows of the tensor-core path's M tile; expert groups are padded to it.
+constexpr int kPrefillTileM = 128;
+
+cudaError_t launch_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t* q,
+                            float* scales, cudaStream_t stream);
+
+cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
+                         const float* bias, int E, int top_k, int32_t* ids, float* gates,
+                         float* logits, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_t* offsets,
+                           int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,
+                           cudaStream_t stream);
+
+cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
+                               const int32_t* offsets, const int32_t* padded_offsets,
+                               const int32_t* perm, int64_t max_rows, void* x_perm, int num_sms,
+                               cudaStream_t stream);
+
+// Optional stage-timing callback (see jmoe_profile_events).
+using StageMark = void (*)(int stage, bool after, cudaStream_t stream);
+
+struct DecodeArgs {
+    const void* x;        // bf16 [T][d]
+    int64_t T, A, d, f;
+    int E, top_k;
+    const int8_t* wgu;    // int8 [E][2f][d]
+    const float* sgu;     // [E][2f]
+    const int8_t* wd;     // int8 [E][d][f]
+    const float* sd;      // [E][d]
+    const int32_t* ids;   // [T][top_k]
+    const float* gates;   // [T][top_k]
+    const int32_t* offsets;  // [E+1]
+    const int32_t* perm;     // [A]
+    const int32_t* inv;      // [A]
+    void* H;              // bf16 [A][f]   (workspace)
+    float* P;             // fp32 [nsplit][A][d] (workspace)
+    int nsplit;
+    int64_t max_per_expert;  // host-side bound used to size register tiles
+    void* out;            // bf16 [T][d]
+    int num_sms;
+    StageMark mark;
+};
+
+int decode_split_for(int64_t f);
+cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace jmoe

@@ -1,0 +1,164 @@
+// Grouping of token->expert assignments by expert, and the row gather that
+// feeds the tensor-core path.
+//
+// The fused MoE kernel of "Jamba-1.5: Hybrid Transformer-Mamba Models at
+// Scale" (paper summary, section "Innovation 2") fuses expert routing with
+// the expert computation; here routing is split into this bit-exact
+// counting sort and the expert GEMMs that consume its output.
+//
+// k_permute: one CTA of 1024 threads.
+//   pass 1: per-expert counts (shared-memory atomics; order-independent);
+//   scan:   offsets[e] = exclusive prefix; padded offsets (each count rounded
+//           up to the tensor-core path's row tile) for the gather;
+//   pass 2: the assignments are visited in ascending order, 1024 at a time;
+//           inside a warp, __match_any_sync groups lanes with the same expert
+//           and a popcount of the lower lanes gives the stable rank; per-warp
+//           counts are prefix-summed across the 32 warps.  perm and inv come
+//           out identical to a stable counting sort.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace jmoe {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxE = 16;
+
+__global__ void __launch_bounds__(kThreads)
+    k_permute(const int32_t* __restrict__ ids, int64_t A, int E, int pad, int32_t* __restrict__ offsets,
+              int32_t* __restrict__ padded_offsets, int32_t* __restrict__ perm,
+              int32_t* __restrict__ inv, unsigned* err) {
+    __shared__ int s_count[kMaxE];
+    __shared__ int s_cursor[kMaxE];
+    __shared__ int s_warp_count[kWarps][kMaxE];
+    __shared__ int s_warp_base[kWarps][kMaxE];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    if (tid < kMaxE) s_count[tid] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int64_t a = tid; a < A; a += kThreads) {
+        const int e = ids[a];
+        if (e >= 0 && e < E)
+            atomicAdd(&s_count[e], 1);
+        else
+            bad = true;
+    }
+    if (bad) flag_error(err, kErrBadExpert);
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0, prun = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = run;
+            if (padded_offsets) padded_offsets[e] = prun;
+            s_cursor[e] = run;
+            run += s_count[e];
+            prun += (s_count[e] + pad - 1) / pad * pad;
+        }
+        offsets[E] = run;
+        if (padded_offsets) padded_offsets[E] = prun;
+    }
+    for (int i = tid; i < kWarps * kMaxE; i += kThreads) (&s_warp_count[0][0])[i] = 0;
+    __syncthreads();
+
+    for (int64_t base = 0; base < A; base += kThreads) {
+        const int64_t a = base + tid;
+        int e = a < A ? ids[a] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        if (e >= 0 && rank == 0) s_warp_count[warp][e] = __popc(peers);
+        __syncthreads();
+        if (tid < E) {
+            int run = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                s_warp_base[w][tid] = run;
+                run += s_warp_count[w][tid];
+                s_warp_count[w][tid] = 0;
+            }
+            s_count[tid] = run;  // this chunk's total for expert tid
+        }
+        __syncthreads();
+        if (e >= 0) {
+            const int pos = s_cursor[e] + s_warp_base[warp][e] + rank;
+            perm[pos] = (int32_t)a;
+            if (inv) inv[a] = pos;
+        } else if (a < A && inv) {
+            inv[a] = -1;
+        }
+        __syncthreads();
+        if (tid < E) s_cursor[tid] += s_count[tid];
+        __syncthreads();
+    }
+}
+
+// x_perm[padded_offsets[e] + r] = x[perm[offsets[e] + r] / top_k] for
+// r < count_e, zero rows up to the padded end.  One warp per row, 16-B moves.
+__global__ void __launch_bounds__(256)
+    k_gather_rows(const uint16_t* __restrict__ x, int64_t d, int top_k, int E,
+                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ padded_offsets,
+                  const int32_t* __restrict__ perm, int64_t max_rows, uint16_t* __restrict__ x_perm) {
+    __shared__ int s_off[kMaxE + 1], s_poff[kMaxE + 1];
+    if (threadIdx.x <= E) {
+        s_off[threadIdx.x] = offsets[threadIdx.x];
+        s_poff[threadIdx.x] = padded_offsets[threadIdx.x];
+    }
+    __syncthreads();
+    const int64_t total = s_poff[E];
+    const int lane = threadIdx.x & 31;
+    const int64_t nvec = d / 8;
+    for (int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); row < total && row < max_rows;
+         row += (int64_t)gridDim.x * 8) {
+        int e = 0;
+        while (e + 1 < E && s_poff[e + 1] <= row) ++e;
+        const int64_t r = row - s_poff[e];
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + row * d);
+        if (r < s_off[e + 1] - s_off[e]) {
+            const int64_t t = perm[s_off[e] + r] / top_k;
+            const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+            for (int64_t i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
+        } else {
+            for (int64_t i = lane; i < nvec; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__global__ void k_fill_f32(float* __restrict__ p, float v, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = v;
+}
+
+}  // namespace
+
+cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    k_fill_f32<<<(unsigned)blocks, 256, 0, stream>>>(p, v, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_t* offsets,
+                           int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,
+                           cudaStream_t stream) {
+    k_permute<<<1, kThreads, 0, stream>>>(ids, A, E, pad, offsets, padded_offsets, perm, inv, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
+                               const int32_t* offsets, const int32_t* padded_offsets,
+                               const int32_t* perm, int64_t max_rows, void* x_perm, int num_sms,
+                               cudaStream_t stream) {
+    if (max_rows == 0) return cudaSuccess;
+    int64_t blocks = (max_rows + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 16;
+    if (blocks > cap) blocks = cap;
+    k_gather_rows<<<(unsigned)blocks, 256, 0, stream>>>((const uint16_t*)x_bf16, d, top_k, E,
+                                                        offsets, padded_offsets, perm, max_rows,
+                                                        (uint16_t*)x_perm);
+    return cudaGetLastError();
+}
+
+}  // namespace jmoe

@@ -1,0 +1,299 @@
+"""CUDA path vs the CPU oracle, on the same seeded inputs, through the C ABI.
+
+Bit-exact: INT8 weights and scales, router logits and top-k ids, the
+permutation.  Floating-point outputs: max |d| <= 2e-2 max |ref| and
+sum |d| / sum |ref| <= 5e-3 (bf16 I/O, fp32 accumulation); gates within 1e-6.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from exact import bf16_bits
+from layers import DeviceLayer, OracleLayer, assert_close, bf16_to_f64
+from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DENSE,
+                             MINI_PREFILL, TINY, Workload)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import int8_weight_moe_b200 as jm  # noqa: E402
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def cuda_bf16(bits: np.ndarray):
+    return torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).cuda()
+
+
+# ----------------------------------------------------------------------------- quantisation
+
+
+def test_quantize_golden_rows_bitexact():
+    with open(os.path.join(GOLDEN, "quantize_rows.json")) as fh:
+        rows = json.load(fh)["rows"]
+    for row in rows:
+        vals = np.array(row["values"], dtype=np.float32)
+        pad = (-len(vals)) % 8  # the device kernel wants 16-byte rows
+        bits = bf16_bits(np.concatenate([vals, np.zeros(pad, np.float32)]))[None, :]
+        q, s = jm.jmoe_quantize(cuda_bf16(bits))
+        qo, so = oracle.quantize(bits)
+        assert np.array_equal(q.cpu().numpy(), qo), row["name"]
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32)), row["name"]
+
+
+def test_quantize_tiny_all_weights_bitexact():
+    dev = DeviceLayer(TINY)
+    ora = OracleLayer(TINY)
+    for e in range(TINY.E):
+        qg, sg, qd, sd = ora.expert(e)
+        assert np.array_equal(dev.w_gu[e].cpu().numpy(), qg)
+        assert np.array_equal(dev.s_gu[e].cpu().numpy().view(np.uint32), sg.view(np.uint32))
+        assert np.array_equal(dev.w_d[e].cpu().numpy(), qd)
+        assert np.array_equal(dev.s_d[e].cpu().numpy().view(np.uint32), sd.view(np.uint32))
+
+
+@pytest.mark.parametrize("wl", [MINI_DECODE, LARGE_DECODE], ids=lambda w: w.name)
+def test_quantize_full_size_sampled_rows_bitexact(wl):
+    """Full-size expert matrices quantised on the GPU; 3 experts x 48 sampled
+    rows of each matrix re-derived by the oracle."""
+    dev = DeviceLayer(wl, T=8)
+    ora = OracleLayer(wl, T=8)
+    rng = np.random.default_rng(0)
+    f, d = wl.d_ff, wl.d_model
+    for e in (0, wl.E // 2, wl.E - 1):
+        for r in rng.integers(0, 2 * f, size=48):
+            q, s = oracle.quantize(ora.gate_up_rows(e, int(r), 1))
+            assert np.array_equal(dev.w_gu[e, r].cpu().numpy(), q[0])
+            assert dev.s_gu[e, r].item() == s[0]
+        for r in rng.integers(0, d, size=48):
+            q, s = oracle.quantize(ora.down_rows(e, int(r), 1))
+            assert np.array_equal(dev.w_d[e, r].cpu().numpy(), q[0])
+            assert dev.s_d[e, r].item() == s[0]
+
+
+def test_quantize_roundtrip_bound_on_device():
+    w = synth.normal_bf16_gpu(77, synth.WD, 0.02, (512, 1024))
+    q, s = jm.jmoe_quantize(w)
+    wv = w.float().double()
+    err = (wv - q.double() * s.double()[:, None]).abs()
+    assert bool((err <= s.double()[:, None] / 2 * (1 + 2.0 ** -16)).all())
+    assert int(q.abs().max(dim=1).values.min()) == 127
+
+
+# ----------------------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("wl", [TINY, MINI_DECODE, LARGE_DECODE, MINI_PREFILL, LARGE_PREFILL_SKEW],
+                         ids=lambda w: w.name)
+def test_route_bitexact(wl):
+    dev = DeviceLayer(Workload(wl.name, wl.index, wl.T, wl.d_model, 64, wl.E, wl.top_k, wl.bias))
+    ora = OracleLayer(wl)
+    ids, g, logits = jm.jmoe_route(dev.x, dev.w_router, wl.top_k, dev.bias, want_logits=True)
+    lo, io, go = ora.route()
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    gg = g.cpu().numpy().astype(np.float64)
+    assert np.abs(gg - go).max() <= 1e-6
+    assert np.abs(gg.sum(axis=1) - 1.0).max() <= 2.0 ** -21
+    if wl.bias is not None:
+        frac = float(np.isin(io, [0, 1]).mean())
+        assert 0.33 <= frac <= 0.47, frac
+
+
+def test_route_top1_and_ties():
+    d, E = 256, 16
+    x = synth.normal_bf16_gpu(3, synth.X, 1.0, (40, d))
+    wr = synth.normal_f32_gpu(3, synth.WR, 0.02, (E, d))
+    wr[7] = wr[3]
+    bias = torch.zeros(E, dtype=torch.float32, device="cuda")
+    bias[3] = bias[7] = 4.0
+    ids, g = jm.jmoe_route(x, wr, 2, bias)
+    assert bool((ids[:, 0] == 3).all()) and bool((ids[:, 1] == 7).all())
+    assert bool((g == 0.5).all())
+    ids1, g1 = jm.jmoe_route(x, wr, 1, None)
+    _, io, _ = oracle.route(x.view(torch.int16).cpu().numpy().view(np.uint16),
+                            wr.cpu().numpy(), 1, None)
+    assert np.array_equal(ids1.cpu().numpy(), io)
+    assert bool((g1 == 1.0).all())
+    z = torch.zeros((4, d), dtype=torch.bfloat16, device="cuda")
+    idz, gz = jm.jmoe_route(z, wr, 2, None)
+    assert idz.cpu().numpy().tolist() == [[0, 1]] * 4 and bool((gz == 0.5).all())
+
+
+# ----------------------------------------------------------------------------- permutation
+
+
+@pytest.mark.parametrize("T,k,E,mode", [(64, 2, 16, "uniform"), (37, 2, 16, "skew"),
+                                         (1, 2, 16, "uniform"), (5000, 2, 16, "skew"),
+                                         (16384, 2, 16, "uniform"), (300, 1, 1, "uniform"),
+                                         (129, 2, 16, "one")])
+def test_permute_bitexact(T, k, E, mode):
+    rng = np.random.default_rng(T + k + E)
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    if mode == "skew":
+        ids[:, 0] = np.minimum(ids[:, 0], 1)
+    if mode == "one":
+        ids[:] = 5
+    off, perm, inv = jm.jmoe_permute(torch.from_numpy(ids).cuda(), E)
+    oo, po, io = oracle.permute(ids, E)
+    assert np.array_equal(off.cpu().numpy(), oo)
+    assert np.array_equal(perm.cpu().numpy(), po)
+    assert np.array_equal(inv.cpu().numpy(), io)
+
+
+# ----------------------------------------------------------------------------- forward
+
+
+def run_layer(dev, path=0):
+    ids, g = jm.jmoe_route(dev.x, dev.w_router, dev.wl.top_k, dev.bias)
+    out = jm.jmoe_forward(dev.desc(path), dev.x, ids, g)
+    torch.cuda.synchronize()
+    return ids, g, out
+
+
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+def test_forward_tiny_all_tokens(path):
+    dev, ora = DeviceLayer(TINY), OracleLayer(TINY)
+    ids, g, out = run_layer(dev, path)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    ref = ora.forward_tokens(np.arange(TINY.T), io, go)
+    assert_close(bf16_to_f64(out), ref, "tiny")
+
+
+def test_forward_mini_decode_all_tokens():
+    dev, ora = DeviceLayer(MINI_DECODE), OracleLayer(MINI_DECODE)
+    ids, g, out = run_layer(dev)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    ref = ora.forward_tokens(np.arange(MINI_DECODE.T), io, go)
+    assert_close(bf16_to_f64(out), ref, "mini decode")
+
+
+def test_forward_large_decode_sampled():
+    dev, ora = DeviceLayer(LARGE_DECODE), OracleLayer(LARGE_DECODE)
+    ids, g, out = run_layer(dev)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    tokens = [0, 31]
+    ref = ora.forward_tokens(tokens, io, go)
+    assert_close(bf16_to_f64(out)[tokens], ref, "large decode")
+
+
+@pytest.mark.parametrize("wl,tokens", [
+    (MINI_PREFILL, [0, 1, 2, 511, 4097, 9000, 16382, 16383]),
+    (LARGE_PREFILL_SKEW, [0, 4095, 8191]),
+], ids=["mini_prefill", "large_prefill_skewed"])
+def test_forward_prefill_sampled(wl, tokens):
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g, out = run_layer(dev)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    ref = ora.forward_tokens(tokens, io, go)
+    assert_close(bf16_to_f64(out)[tokens], ref, wl.name)
+
+
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+def test_dense_mlp_tiny(path):
+    wl = Workload("tiny_dense", 0, 64, 256, 512, E=1, top_k=1, dense=True)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    out = jm.jmoe_mlp_forward(dev.x, dev.w_gu[0], dev.s_gu[0], dev.w_d[0], dev.s_d[0], path=path)
+    torch.cuda.synchronize()
+    assert_close(bf16_to_f64(out), ora.dense_forward_tokens(np.arange(64)), "tiny dense")
+
+
+def test_dense_mlp_mini_sampled():
+    dev, ora = DeviceLayer(MINI_DENSE), OracleLayer(MINI_DENSE)
+    out = jm.jmoe_mlp_forward(dev.x, dev.w_gu[0], dev.s_gu[0], dev.w_d[0], dev.s_d[0])
+    torch.cuda.synchronize()
+    tokens = [0, 100, 8191, 16383]
+    assert_close(bf16_to_f64(out)[tokens], ora.dense_forward_tokens(tokens), "mini dense")
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+
+@pytest.mark.parametrize("T", [1, 2, 37, 129])
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+def test_forward_ragged_token_counts(T, path):
+    wl = Workload(f"ragged_T{T}", 7, T, 256, 576, bias=None)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g, out = run_layer(dev, path)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(T), io, go), f"T={T}")
+
+
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+def test_forced_routing_one_expert_and_zero_input(path):
+    wl = Workload("forced", 8, 200, 256, 512)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids = np.full((wl.T, 2), 5, dtype=np.int32)
+    ids[::3, 1] = 9
+    gates = np.tile(np.array([0.75, 0.25], dtype=np.float32), (wl.T, 1))
+    out = jm.jmoe_forward(dev.desc(path), dev.x, torch.from_numpy(ids).cuda(),
+                          torch.from_numpy(gates).cuda())
+    torch.cuda.synchronize()
+    ref = ora.forward_tokens(np.arange(wl.T), ids, gates.astype(np.float64))
+    assert_close(bf16_to_f64(out), ref, "forced")
+    zero = torch.zeros_like(dev.x)
+    outz = jm.jmoe_forward(dev.desc(path), zero, torch.from_numpy(ids).cuda(),
+                           torch.from_numpy(gates).cuda())
+    torch.cuda.synchronize()
+    assert bool((outz.float() == 0).all())
+
+
+def test_forward_top1_and_single_expert():
+    wl = Workload("top1", 9, 50, 256, 512, E=16, top_k=1)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g, out = run_layer(dev)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(wl.T), io, go), "top1")
+    wl1 = Workload("E1", 10, 30, 256, 512, E=1, top_k=1)
+    dev1, ora1 = DeviceLayer(wl1), OracleLayer(wl1)
+    ids1, g1, out1 = run_layer(dev1)
+    assert bool((ids1 == 0).all()) and bool((g1 == 1).all())
+    assert_close(bf16_to_f64(out1), ora1.dense_forward_tokens(np.arange(30)), "E=1")
+
+
+def test_zero_tokens_is_a_noop():
+    dev = DeviceLayer(TINY, T=1)
+    x = dev.x[:0]
+    ids = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    g = torch.empty((0, 2), dtype=torch.float32, device="cuda")
+    out = jm.jmoe_forward(dev.desc(), x, ids, g)
+    assert out.shape == (0, TINY.d_model)
+
+
+# ----------------------------------------------------------------------------- invariants
+
+
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+def test_token_permutation_and_determinism(path):
+    wl = Workload("perm", 11, 96, 256, 512)
+    dev = DeviceLayer(wl)
+    ids, g, out = run_layer(dev, path)
+    _, _, out2 = run_layer(dev, path)
+    assert torch.equal(out, out2)  # run-to-run bitwise identical
+    tp = torch.randperm(wl.T, generator=torch.Generator().manual_seed(0)).cuda()
+    outp = jm.jmoe_forward(dev.desc(path), dev.x[tp].contiguous(), ids[tp].contiguous(),
+                           g[tp].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(outp, out[tp])
+
+
+def test_invalid_expert_id_sets_device_error_word():
+    assert jm.jmoe_last_error() in (jm.JMOE_OK, jm.JMOE_EDEVICE)
+    dev = DeviceLayer(Workload("bad", 12, 8, 256, 512))
+    ids = torch.full((8, 2), 1, dtype=torch.int32, device="cuda")
+    ids[3, 1] = 99
+    g = torch.full((8, 2), 0.5, dtype=torch.float32, device="cuda")
+    out = jm.jmoe_forward(dev.desc(jm.JMOE_PATH_DECODE), dev.x, ids, g)
+    assert jm.jmoe_last_error() == jm.JMOE_EDEVICE
+    assert jm.jmoe_last_error() == jm.JMOE_OK  # cleared by the read
+    assert bool(torch.isfinite(out.float()).all())

@@ -68,7 +68,7 @@ class ClockSampler(threading.Thread):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         self.handle = None
         try:
             import pynvml
@@ -95,7 +95,7 @@ class ClockSampler(threading.Thread):
         if self.handle is None:
             return
         n = self.nvml
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
                 self.reasons |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
@@ -104,7 +104,7 @@ class ClockSampler(threading.Thread):
             time.sleep(self.period)
 
     def stop(self):
-        self._stop.set()
+        self._halt.set()
         self.join(timeout=2)
         if self.handle is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"]}
@@ -210,15 +210,22 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
 
         dist.barrier()
     torch.cuda.synchronize()
+    if profile:
+        # torch creates the CUDA event handle on the first record: record every
+        # event once now so the library can re-record them inside the steps
+        for _ in range(steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+            for ev in evs:
+                ev.record()
+            stage_events.append(evs)
+        torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     launches = 0
     start.record()
-    for _ in range(steps):
+    for i in range(steps):
         if profile:
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
-            jm.jmoe_profile_events(evs)
-            stage_events.append(evs)
+            jm.jmoe_profile_events(stage_events[i])
         launches += layer.step()
     stop.record()
     jm.jmoe_profile_events(None)
@@ -230,15 +237,20 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
     total_ms = start.elapsed_time(stop)
     stages = {}
     for i, name in enumerate(jm.STAGES):
-        times = []
-        for evs in stage_events:
-            try:
-                times.append(evs[2 * i].elapsed_time(evs[2 * i + 1]))
-            except RuntimeError:
-                pass  # this stage did not run on this path
-        if times:
+        times = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for evs in stage_events]
+        # a stage that does not run on this path leaves its pre-recorded pair,
+        # which spans no step: report only stages whose events moved
+        if times and min(times) >= 0 and stage_ran(stage_events, i, start):
             stages[name] = sum(times) / len(times)
     return total_ms, stages, launches
+
+
+def stage_ran(stage_events, i, start):
+    """True when stage i's events were re-recorded inside the timed region."""
+    try:
+        return all(start.elapsed_time(evs[2 * i]) >= 0 for evs in stage_events)
+    except RuntimeError:
+        return False
 
 
 def roofline_entry(layer: Layer, stages: dict, peaks: dict, traffic=None):

@@ -1,7 +1,521 @@
-// Tensor-core expert path (placeholder until the tcgen05 kernels land).
+// Tensor-core path of the expert MLPs (many tokens per expert): a persistent
+// grouped GEMM on the 5th-generation tensor cores (tcgen05, accumulators in
+// TMEM), with the ExpertsInt8 dequantisation inside the kernel.
+//
+// "Jamba-1.5: Hybrid Transformer-Mamba Models at Scale" (paper summary),
+// section "ExpertsInt8 Quantization (Section 3.1)", step 3: the INT8 weights
+// are turned back into BF16 inside the fused MoE kernel as they move from HBM
+// to on-chip memory, by a scaling and a cast.  Here: TMA brings each INT8
+// weight tile HBM -> shared memory (1 byte per weight), converter warps turn
+// it exactly into BF16 in the 128-byte-swizzled K-major layout the tensor core
+// reads, and the per-output-channel scale is applied once in the epilogue
+// (sum_k x_k (q_k s) = s sum_k x_k q_k).  Activations stay BF16 (step 4);
+// accumulation is fp32 in TMEM.
+//
+// One CTA per SM, 15 warps:
+//   warp 0      TMA producer of the activation tile A [128 rows x 64 k] bf16
+//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warp 2      TMA producer of the INT8 weight tile [256 rows x 64 k]
+//   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled)
+//   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
+// Rings: A + converted B share 3 stages (48 KB each), the INT8 tiles have 4
+// stages (16 KB each); two 128 x 256 fp32 accumulators (512 TMEM columns)
+// let the epilogue of one tile overlap the main loop of the next.
+//
+// Tiles: 128 expert-grouped rows (each expert's rows are padded to a
+// multiple of 128, so a tile never mixes experts) x 256 MMA columns.  Gate/up
+// mode: the 256 columns are 128 gate channels and the same 128 up channels,
+// so the SwiGLU pairs sit in one thread.  Down mode: 256 output channels; the
+// epilogue multiplies by the routing gate and writes one fp32 row per
+// token->expert assignment.  Tiles are visited expert by expert, m fastest,
+// so the CTAs of a wave share weight tiles and activation rows in L2.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
 #include "prefill.h"
+#include "sm100.cuh"
 
 namespace jmoe {
-bool prefill_available() { return false; }
-cudaError_t launch_prefill(const PrefillArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kStagesAB = 3, kStages8 = 4;
+constexpr int kABytes = BM * BK * 2;    // 16 KB
+constexpr int kBbfBytes = BN * BK * 2;  // 32 KB
+constexpr int kB8Bytes = BN * BK;       // 16 KB
+constexpr int kABStage = kABytes + kBbfBytes;
+constexpr int kSmemAB = kStagesAB * kABStage;
+constexpr int kSmem8 = kStages8 * kB8Bytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
+
+constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
+constexpr int kConvWarp0 = 3, kConvWarps = 8;
+constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps, kEpiWarps = 4;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+constexpr int kMaxE = 16;
+
+enum Mode { kGateUp = 0, kDown = 1 };
+
+struct GemmParams {
+    int E;
+    int K;                // contraction length (d_model or d_ff)
+    int n_valid;          // valid output channels (d_ff or d_model)
+    int n_tiles;          // N tiles per expert
+    int w_rows;           // weight rows per expert (2 d_ff or d_model)
+    int up_offset;        // d_ff (gate/up mode)
+    const int32_t* poff;  // [E+1] padded row offsets
+    const int32_t* off;   // [E+1] assignment offsets
+    const int32_t* perm;  // [A]
+    const float* scale;   // [E][w_rows]
+    const float* gates;   // [A]
+    uint16_t* H;          // gate/up output, bf16 [rows_padded][d_ff]
+    float* Y;             // down output, fp32 [A][d_model]
+    unsigned* err;
+};
+
+struct Shared {
+    uint64_t ab_full_a[kStagesAB], ab_full_b[kStagesAB], ab_empty[kStagesAB];
+    uint64_t b8_full[kStages8], b8_empty[kStages8];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int poff[kMaxE + 1];
+    int off[kMaxE + 1];
+    int tile_start[kMaxE + 1];
+};
+
+constexpr int kSmemBytes = kSmemAB + kSmem8 + (int)sizeof(Shared) + 1024;
+
+struct Tile {
+    int e, row0, n;
+};
+
+__device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int tile) {
+    int e = 0;
+    while (e + 1 < E && s.tile_start[e + 1] <= tile) ++e;
+    const int local = tile - s.tile_start[e];
+    const int mt = (s.poff[e + 1] - s.poff[e]) / BM;
+    Tile t;
+    t.e = e;
+    t.n = local / mt;
+    t.row0 = s.poff[e] + (local % mt) * BM;
+    return t;
+}
+
+// Bounded wait that ignores the abort flag (used only while draining).
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    Shared& S = *reinterpret_cast<Shared*>(smem + kSmemAB + kSmem8);
+    auto tileA = [&](int s) { return smem + s * kABStage; };
+    auto tileBbf = [&](int s) { return smem + s * kABStage + kABytes; };
+    auto tileB8 = [&](int s) { return smem + kSmemAB + s * kB8Bytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int KB = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStagesAB; ++i) {
+            mbar_init(&S.ab_full_a[i], 1);
+            mbar_init(&S.ab_full_b[i], kConvWarps);
+            mbar_init(&S.ab_empty[i], 1);
+        }
+        for (int i = 0; i < kStages8; ++i) {
+            mbar_init(&S.b8_full[i], 1);
+            mbar_init(&S.b8_empty[i], kConvWarps);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_empty[i], kEpiWarps);
+        }
+        mbar_init(&S.drain, 1);
+        S.abort = 0;
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= E) {
+        S.poff[threadIdx.x] = p.poff[threadIdx.x];
+        S.off[threadIdx.x] = p.off[threadIdx.x];
+    }
+    if (warp == kWarpProdA && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            S.tile_start[e] = run;
+            run += (S.poff[e + 1] - S.poff[e]) / BM * p.n_tiles;
+        }
+        S.tile_start[E] = run;
+    }
+    if (warp == kWarpMMA) {
+        tmem_alloc(&S.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    const int total = S.tile_start[E];
+    volatile int* abort = &S.abort;
+
+    if (warp == kWarpProdA) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+                const Tile t = decode_tile(S, E, tile);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStagesAB;
+                    const uint32_t ph = (g / kStagesAB) & 1;
+                    if (!mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) break;
+                    mbar_arrive_expect_tx(&S.ab_full_a[s], kABytes);
+                    tma_load_2d(tileA(s), &tmA, &S.ab_full_a[s], kb * BK, t.row0);
+                }
+            }
+            // make sure no copy is still landing in shared memory when the CTA exits
+            for (uint32_t h = (g > (uint32_t)kStagesAB ? g - kStagesAB : 0); h < g; ++h)
+                wait_drain(&S.ab_full_a[h % kStagesAB], (h / kStagesAB) & 1);
+        }
+    } else if (warp == kWarpProdB) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+                const Tile t = decode_tile(S, E, tile);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStages8;
+                    const uint32_t ph = (g / kStages8) & 1;
+                    if (!mbar_wait(&S.b8_empty[s], ph ^ 1, abort)) break;
+                    mbar_arrive_expect_tx(&S.b8_full[s], kB8Bytes);
+                    if (MODE == kGateUp) {
+                        const int y = t.e * p.w_rows + t.n * (BN / 2);
+                        tma_load_2d(tileB8(s), &tmB, &S.b8_full[s], kb * BK, y);
+                        tma_load_2d(tileB8(s) + kB8Bytes / 2, &tmB, &S.b8_full[s], kb * BK,
+                                    y + p.up_offset);
+                    } else {
+                        tma_load_2d(tileB8(s), &tmB, &S.b8_full[s], kb * BK,
+                                    t.e * p.w_rows + t.n * BN);
+                    }
+                }
+            }
+            for (uint32_t h = (g > (uint32_t)kStages8 ? g - kStages8 : 0); h < g; ++h)
+                wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1);
+        }
+    } else if (warp == kWarpMMA) {
+        if (lane == 0) {
+            uint32_t g = 0;
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+                const int buf = it & 1;
+                if (!mbar_wait(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * BN;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStagesAB;
+                    const uint32_t ph = (g / kStagesAB) & 1;
+                    if (!mbar_wait(&S.ab_full_a[s], ph, abort) ||
+                        !mbar_wait(&S.ab_full_b[s], ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(tileA(s)), b0 = smem_u32(tileBbf(s));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_ss(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
+                                    kIdesc, (kb | kk) != 0);
+                    mma_commit(&S.ab_empty[s]);
+                }
+                if (!ok) break;
+                mma_commit(&S.acc_full[buf]);
+            }
+            mma_commit(&S.drain);
+            wait_drain(&S.drain, 0);
+        }
+    } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
+        const int ct = threadIdx.x - kConvWarp0 * 32;  // 0..255
+        const int chunk = ct & 7;
+        uint32_t g = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok && !*abort; tile += gridDim.x) {
+            for (int kb = 0; kb < KB; ++kb, ++g) {
+                const int s = g % kStagesAB;
+                const uint32_t ph = (g / kStagesAB) & 1;
+                const int s8 = g % kStages8;
+                const uint32_t ph8 = (g / kStages8) & 1;
+                if (!mbar_wait(&S.b8_full[s8], ph8, abort) ||
+                    !mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* src = tileB8(s8);
+                uint8_t* dst = tileBbf(s);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int row = (ct >> 3) + 32 * j;
+                    const uint2 v = *reinterpret_cast<const uint2*>(src + row * BK + chunk * 8);
+                    uint4 o;
+                    o.x = i8x2_to_bf16x2<0>(v.x);
+                    o.y = i8x2_to_bf16x2<1>(v.x);
+                    o.z = i8x2_to_bf16x2<0>(v.y);
+                    o.w = i8x2_to_bf16x2<1>(v.y);
+                    *reinterpret_cast<uint4*>(dst + (row >> 3) * 1024 + (row & 7) * 128 +
+                                              ((chunk ^ (row & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&S.ab_full_b[s]);
+                    mbar_arrive(&S.b8_empty[s8]);
+                }
+            }
+        }
+    } else {
+        // epilogue warps: TMEM lane quadrant = warp % 4
+        const int quad = warp & 3;
+        const int rloc = quad * 32 + lane;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+            const Tile t = decode_tile(S, E, tile);
+            const int buf = it & 1;
+            if (!mbar_wait(&S.acc_full[buf], (it >> 1) & 1, abort)) break;
+            tc_fence_after();
+            __syncwarp();
+            const uint32_t taddr = tmem + buf * BN + ((uint32_t)(quad * 32) << 16);
+            const int row = t.row0 + rloc;
+            if (MODE == kGateUp) {
+                const int n0 = t.n * (BN / 2);
+                const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
+                const float* su = sg + p.up_offset;
+#pragma unroll 1
+                for (int c = 0; c < BN / 2 / 32; ++c) {
+                    uint32_t gv[32], uv[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, gv);
+                    tmem_ld_32x32b_x32(taddr + BN / 2 + c * 32, uv);
+                    tmem_ld_wait();
+                    const int ch = n0 + c * 32;
+                    if (ch < p.n_valid) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const float g0 = __ldg(sg + c * 32 + j) * __uint_as_float(gv[j]);
+                            const float g1 = __ldg(sg + c * 32 + j + 1) * __uint_as_float(gv[j + 1]);
+                            const float u0 = __ldg(su + c * 32 + j) * __uint_as_float(uv[j]);
+                            const float u1 = __ldg(su + c * 32 + j + 1) * __uint_as_float(uv[j + 1]);
+                            packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                                packed[4 * q + 3]);
+                    }
+                }
+            } else {
+                const int m0 = t.n * BN;
+                const int r = row - S.poff[t.e];
+                const bool valid = r < S.off[t.e + 1] - S.off[t.e];
+                const int a = valid ? p.perm[S.off[t.e] + r] : 0;
+                const float gate = valid ? p.gates[a] : 0.0f;
+                const float* sd = p.scale + (size_t)t.e * p.w_rows;
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    tmem_ld_wait();
+                    const int m = m0 + c * 32;
+                    if (valid && m < p.n_valid) {
+                        float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + q);
+                            float4 o;
+                            o.x = gate * (s4.x * __uint_as_float(v[4 * q]));
+                            o.y = gate * (s4.y * __uint_as_float(v[4 * q + 1]));
+                            o.z = gate * (s4.z * __uint_as_float(v[4 * q + 2]));
+                            o.w = gate * (s4.w * __uint_as_float(v[4 * q + 3]));
+                            dst[q] = o;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && S.abort) flag_error(p.err, kErrTimeout);
+    if (warp == kWarpMMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// out[t] = bf16( sum_j Y[t*top_k + j] ) over the valid assignments of token t.
+__global__ void __launch_bounds__(256)
+    k_finalize(const float* __restrict__ Y, int64_t T, int64_t d, int top_k, int E,
+               const int32_t* __restrict__ ids, uint16_t* __restrict__ out) {
+    const int64_t nvec = d / 4;
+    const int64_t total = T * nvec;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = v / nvec, m = (v % nvec) * 4;
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < top_k; ++j) {
+            const int64_t a = t * top_k + j;
+            const int e = ids[a];
+            if (e < 0 || e >= E) continue;
+            const float4 y = *reinterpret_cast<const float4*>(Y + a * d + m);
+            o[0] += y.x;
+            o[1] += y.y;
+            o[2] += y.z;
+            o[3] += y.w;
+        }
+        uint2 r;
+        r.x = pack_bf16x2(o[0], o[1]);
+        r.y = pack_bf16x2(o[2], o[3]);
+        *reinterpret_cast<uint2*>(out + t * d + m) = r;
+    }
+}
+
+// ----------------------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Row-major 2-D tensor [rows][cols]; a box of box_rows x box_cols elements.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
+              uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+              CUtensorMapSwizzle swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
+                        int num_sms, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    k_grouped_gemm<MODE><<<num_sms, kThreads, kSmemBytes, stream>>>(a, b, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_available() { return encode_fn() != nullptr; }
+
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
+    if (a.T == 0) return cudaSuccess;
+    if (a.d > INT32_MAX / 2 || a.f > INT32_MAX / 2 || a.rows_padded > INT32_MAX)
+        return cudaErrorInvalidValue;
+    cudaError_t err;
+    // 1. gather the routed activation rows, grouped by expert, padded per expert
+    if (a.mark) a.mark(1, false, stream);
+    err = launch_gather_rows(a.x, a.d, a.top_k, a.E, a.offsets, a.padded_offsets, a.perm,
+                             a.rows_padded, a.xperm, a.num_sms, stream);
+    if (a.mark) a.mark(1, true, stream);
+    if (err != cudaSuccess) return err;
+
+    CUtensorMap mA1, mB1, mA2, mB2;
+    const bool ok =
+        make_map(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BM, BK,
+                 CU_TENSOR_MAP_SWIZZLE_128B) &&
+        make_map(&mB1, a.wgu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * 2 * a.f, a.d,
+                 BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        make_map(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BM, BK,
+                 CU_TENSOR_MAP_SWIZZLE_128B) &&
+        make_map(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BN, BK,
+                 CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
+
+    // 2. gate/up GEMM + SwiGLU -> H (bf16, grouped rows)
+    GemmParams g1{};
+    g1.E = a.E;
+    g1.K = (int)a.d;
+    g1.n_valid = (int)a.f;
+    g1.n_tiles = (int)((a.f + BN / 2 - 1) / (BN / 2));
+    g1.w_rows = (int)(2 * a.f);
+    g1.up_offset = (int)a.f;
+    g1.poff = a.padded_offsets;
+    g1.off = a.offsets;
+    g1.perm = a.perm;
+    g1.scale = a.sgu;
+    g1.gates = a.gates;
+    g1.H = static_cast<uint16_t*>(a.H);
+    g1.err = a.err;
+    if (a.mark) a.mark(2, false, stream);
+    err = launch_gemm<kGateUp>(mA1, mB1, g1, a.num_sms, stream);
+    if (a.mark) a.mark(2, true, stream);
+    if (err != cudaSuccess) return err;
+
+    // 3. down GEMM, scale and routing gate -> Y (fp32, one row per assignment)
+    GemmParams g2 = g1;
+    g2.K = (int)a.f;
+    g2.n_valid = (int)a.d;
+    g2.n_tiles = (int)((a.d + BN - 1) / BN);
+    g2.w_rows = (int)a.d;
+    g2.up_offset = 0;
+    g2.scale = a.sd;
+    g2.H = nullptr;
+    g2.Y = a.Yg;
+    if (a.mark) a.mark(3, false, stream);
+    err = launch_gemm<kDown>(mA2, mB2, g2, a.num_sms, stream);
+    if (a.mark) a.mark(3, true, stream);
+    if (err != cudaSuccess) return err;
+
+    // 4. out[t] = bf16(sum over the token's assignments)
+    const int64_t total = a.T * (a.d / 4);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)a.num_sms * 8) blocks = (int64_t)a.num_sms * 8;
+    if (a.mark) a.mark(4, false, stream);
+    k_finalize<<<(unsigned)blocks, 256, 0, stream>>>(a.Yg, a.T, a.d, a.top_k, a.E, a.ids,
+                                                     static_cast<uint16_t*>(a.out));
+    if (a.mark) a.mark(4, true, stream);
+    return cudaGetLastError();
+}
+
 }  // namespace jmoe

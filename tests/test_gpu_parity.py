@@ -155,7 +155,10 @@ def run_layer(dev, path=0):
     return ids, g, out
 
 
-@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+PATHS = [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_PREFILL, jm.JMOE_PATH_AUTO]
+
+
+@pytest.mark.parametrize("path", PATHS)
 def test_forward_tiny_all_tokens(path):
     dev, ora = DeviceLayer(TINY), OracleLayer(TINY)
     ids, g, out = run_layer(dev, path)
@@ -163,6 +166,8 @@ def test_forward_tiny_all_tokens(path):
     assert np.array_equal(ids.cpu().numpy(), io)
     ref = ora.forward_tokens(np.arange(TINY.T), io, go)
     assert_close(bf16_to_f64(out), ref, "tiny")
+    if path == jm.JMOE_PATH_PREFILL:
+        assert jm.jmoe_last_error() == jm.JMOE_OK  # no bounded wait ran out
 
 
 def test_forward_mini_decode_all_tokens():
@@ -197,7 +202,7 @@ def test_forward_prefill_sampled(wl, tokens):
     assert_close(bf16_to_f64(out)[tokens], ref, wl.name)
 
 
-@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+@pytest.mark.parametrize("path", PATHS)
 def test_dense_mlp_tiny(path):
     wl = Workload("tiny_dense", 0, 64, 256, 512, E=1, top_k=1, dense=True)
     dev, ora = DeviceLayer(wl), OracleLayer(wl)
@@ -217,10 +222,13 @@ def test_dense_mlp_mini_sampled():
 # ----------------------------------------------------------------------------- edge cases
 
 
-@pytest.mark.parametrize("T", [1, 2, 37, 129])
-@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
-def test_forward_ragged_token_counts(T, path):
-    wl = Workload(f"ragged_T{T}", 7, T, 256, 576, bias=None)
+@pytest.mark.parametrize("T,d,f", [(1, 256, 576), (2, 256, 576), (37, 320, 576),
+                                   (129, 256, 576), (300, 320, 448)])
+@pytest.mark.parametrize("path", PATHS)
+def test_forward_ragged_token_counts(T, d, f, path):
+    """Ragged token counts and ragged N tiles (d_model 320 is not a multiple of
+    the 256-wide down tile, d_ff 576 / 448 not of the 128-channel gate/up tile)."""
+    wl = Workload(f"ragged_T{T}_d{d}_f{f}", 7, T, d, f, bias=None)
     dev, ora = DeviceLayer(wl), OracleLayer(wl)
     ids, g, out = run_layer(dev, path)
     _, io, go = ora.route()
@@ -228,7 +236,7 @@ def test_forward_ragged_token_counts(T, path):
     assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(T), io, go), f"T={T}")
 
 
-@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+@pytest.mark.parametrize("path", PATHS)
 def test_forced_routing_one_expert_and_zero_input(path):
     wl = Workload("forced", 8, 200, 256, 512)
     dev, ora = DeviceLayer(wl), OracleLayer(wl)
@@ -273,7 +281,7 @@ def test_zero_tokens_is_a_noop():
 # ----------------------------------------------------------------------------- invariants
 
 
-@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_AUTO])
+@pytest.mark.parametrize("path", PATHS)
 def test_token_permutation_and_determinism(path):
     wl = Workload("perm", 11, 96, 256, 512)
     dev = DeviceLayer(wl)

@@ -155,6 +155,40 @@ jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int
                              const float* s_d, void* out_bf16, void* workspace,
                              size_t ws_bytes, int32_t path, void* stream);
 
+/* Allocation-free variant of jmoe_forward.
+ * This call has no counterpart in the method's sources; it exists for callers
+ * that cannot obtain device memory at call time -- for example a plugin inside
+ * a serving engine whose memory planner has already handed every byte of HBM
+ * to its own pool, or a latency-critical path that must not pay the implicit
+ * device-wide synchronisation cudaMalloc/cudaFree can cause.  Such a caller
+ * still passes its inputs and its output buffer, but no workspace.
+ *
+ * It runs the decode (GEMV-like) kernels of jmoe_forward, whatever desc->path
+ * says, with their scratch (grouping tables, the hidden activations and the
+ * split-K partial sums) placed in one fixed array of JMOE_NOALLOC_SCRATCH_BYTES
+ * bytes that is part of the library image: every GPU on which the library is
+ * used holds that array until the process exits.  The call allocates nothing
+ * and calls no allocating routine.
+ *  - Size limit: if the scratch jmoe_forward_workspace_size would report for
+ *    the decode kernels exceeds JMOE_NOALLOC_SCRATCH_BYTES, the call returns
+ *    JMOE_EWORKSPACE before launching anything.  Roughly: the partial sums
+ *    take up to 8 * T*top_k * d_model * 4 bytes and the hidden activations
+ *    T*top_k * d_ff * 2 bytes (for example, 32 tokens at d_model 8192,
+ *    d_ff 24576 and top-2 fit; 64 tokens at those sizes do not).
+ *  - The first call on a device looks up the array's device address for that
+ *    device (with that device current) and caches it; make that first call
+ *    before capturing any stream work on the device.
+ *  - All calls share the one array and it keeps whatever the last call left
+ *    there.  Nothing in it has to start at zero for these kernels, so nothing
+ *    is cleared.  Two calls whose work overlaps on the GPU (different
+ *    streams, or different host threads without ordering) race on the array
+ *    and give wrong results: order them on one stream or synchronise.
+ * Arguments, layouts, validation and results are those of jmoe_forward. */
+#define JMOE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, int64_t T,
+                                 const int32_t* topk_ids, const float* topk_w, void* out_bf16,
+                                 void* stream);
+
 /* Stage timing hook (diagnostics).  Registers `n` CUDA events (cudaEvent_t
  * handles passed as void*) that the following jmoe_forward / jmoe_mlp_forward
  * calls record on their stream around their kernels: events[2*i] before and

@@ -25,8 +25,9 @@ JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 
 # Every C entry point the header declares.
 EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_permute", "jmoe_forward_workspace_size",
-            "jmoe_forward", "jmoe_mlp_workspace_size", "jmoe_mlp_forward", "jmoe_profile_events",
-            "jmoe_last_error", "jmoe_status_string")
+            "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
+            "jmoe_profile_events", "jmoe_last_error", "jmoe_status_string")
+NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
 STAGES = ("permute", "gather", "gate_up", "down", "combine")
 
 
@@ -67,6 +68,7 @@ def load() -> ctypes.CDLL:
     lib.jmoe_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
     lib.jmoe_forward_workspace_size.argtypes = [ctypes.POINTER(MoeDesc), i64, ctypes.POINTER(sz)]
     lib.jmoe_forward.argtypes = [ctypes.POINTER(MoeDesc), vp, i64, vp, vp, vp, vp, sz, vp]
+    lib.jmoe_forward_noalloc.argtypes = [ctypes.POINTER(MoeDesc), vp, i64, vp, vp, vp, vp]
     lib.jmoe_mlp_workspace_size.argtypes = [i64, i64, i64, i32, ctypes.POINTER(sz)]
     lib.jmoe_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i32, vp]
     lib.jmoe_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
@@ -214,6 +216,23 @@ def jmoe_forward(desc: MoeDesc, x, topk_ids, topk_w, out=None, workspace=None):
     _check("jmoe_forward", load().jmoe_forward(ctypes.byref(desc), _ptr(x), T, _ptr(topk_ids),
                                                _ptr(topk_w), _ptr(out), _ptr(workspace),
                                                workspace.numel(), _stream(x)))
+    return out
+
+
+def jmoe_forward_noalloc(desc: MoeDesc, x, topk_ids, topk_w, out=None):
+    """jmoe_forward without a workspace: for callers that cannot allocate device
+    memory when they call the layer; the scratch is a fixed array inside the
+    library (see jmoe.h for its size limit and sharing rules)."""
+    import torch
+
+    _need(x, torch.bfloat16, "x")
+    _need(topk_ids, torch.int32, "topk_ids")
+    _need(topk_w, torch.float32, "topk_w")
+    if out is None:
+        out = torch.empty_like(x)
+    _check("jmoe_forward_noalloc",
+           load().jmoe_forward_noalloc(ctypes.byref(desc), _ptr(x), x.shape[0], _ptr(topk_ids),
+                                       _ptr(topk_w), _ptr(out), _stream(x)))
     return out
 
 

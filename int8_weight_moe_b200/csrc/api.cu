@@ -171,6 +171,27 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
     return from_cuda(jmoe::launch_prefill(p, stream));
 }
 
+// Scratch of jmoe_forward_noalloc: a fixed array in the library image, one
+// per device.  In host code its name is only a stand-in for the symbol; the
+// device address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[JMOE_NOALLOC_SCRATCH_BYTES];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+// The array's device address on the current device (looked up once per
+// device, with that device current), or nullptr if the lookup failed.
+void* noalloc_scratch() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = g_noalloc_ptr[dev].load();
+    if (!p) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return nullptr;
+        g_noalloc_ptr[dev].store(addr);
+        p = addr;
+    }
+    return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -313,6 +334,28 @@ jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int
     if (jmoe::launch_fill_f32(gates, 1.0f, T, s) != cudaSuccess) return JMOE_ECUDA;
     return run_experts(&desc, x_bf16, T, ids, gates, out_bf16, base + 2 * tbl, ws_bytes - 2 * tbl,
                        true, s);
+}
+
+jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, int64_t T,
+                                 const int32_t* topk_ids, const float* topk_w, void* out_bf16,
+                                 void* stream) {
+    jmoe_status st = check_desc(desc);
+    if (st != JMOE_OK) return st;
+    if (T < 0) return JMOE_EINVAL;
+    if (T == 0) return JMOE_OK;
+    if (T * desc->top_k > (1LL << 24)) return JMOE_EUNSUPPORTED;
+    if (!x_bf16 || !topk_ids || !topk_w || !out_bf16) return JMOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(topk_ids) || !aligned16(topk_w) || !aligned16(out_bf16))
+        return JMOE_EALIGN;
+    jmoe_moe_desc dec = *desc;
+    dec.path = JMOE_PATH_DECODE;
+    const size_t need =
+        plan(T, T * dec.top_k, dec.E, dec.d_model, dec.d_ff, /*prefill=*/false).total;
+    if (need > JMOE_NOALLOC_SCRATCH_BYTES) return JMOE_EWORKSPACE;
+    void* scratch = noalloc_scratch();
+    if (!scratch) return JMOE_ECUDA;
+    return run_experts(&dec, x_bf16, T, topk_ids, topk_w, out_bf16, scratch,
+                       JMOE_NOALLOC_SCRATCH_BYTES, false, (cudaStream_t)stream);
 }
 
 jmoe_status jmoe_profile_events(void* const* events, int32_t n) {

@@ -149,7 +149,7 @@ class Layer:
             self.ws = torch.empty(jm.jmoe_forward_workspace_size(self.desc, wl.T),
                                   dtype=torch.uint8, device=device)
 
-    def step(self, x=None, out=None):
+    def step(self, x=None, out=None, route_events=None):
         """One pass of the hot path on the current stream; returns #kernel launches."""
         import int8_weight_moe_b200 as jm
 
@@ -161,8 +161,12 @@ class Layer:
             # fill (unit gates), grouping, gate/up, down, combine/finalize (+ gather on the
             # tensor-core path)
             return 6 if self.prefill_path() else 5
+        if route_events:
+            route_events[0].record()
         jm.jmoe_route(x, self.w_router, self.wl.top_k, self.bias, topk_ids=self.ids,
                       topk_w=self.gates)
+        if route_events:
+            route_events[1].record()
         jm.jmoe_forward(self.desc, x, self.ids, self.gates, out=out, workspace=self.ws)
         return 6 if self.prefill_path() else 5
 
@@ -210,6 +214,7 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
 
         dist.barrier()
     torch.cuda.synchronize()
+    route_events = []
     if profile:
         # torch creates the CUDA event handle on the first record: record every
         # event once now so the library can re-record them inside the steps
@@ -218,6 +223,7 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
             for ev in evs:
                 ev.record()
             stage_events.append(evs)
+            route_events.append([torch.cuda.Event(enable_timing=True) for _ in range(2)])
         torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
@@ -226,7 +232,7 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
     for i in range(steps):
         if profile:
             jm.jmoe_profile_events(stage_events[i])
-        launches += layer.step()
+        launches += layer.step(route_events=route_events[i] if profile else None)
     stop.record()
     jm.jmoe_profile_events(None)
     torch.cuda.synchronize()
@@ -236,6 +242,8 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
         dist.barrier()
     total_ms = start.elapsed_time(stop)
     stages = {}
+    if profile and not layer.wl.dense:
+        stages["route"] = sum(a.elapsed_time(b) for a, b in route_events) / len(route_events)
     for i, name in enumerate(jm.STAGES):
         times = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for evs in stage_events]
         # a stage that does not run on this path leaves its pre-recorded pair,

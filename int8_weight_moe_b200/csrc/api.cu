@@ -70,10 +70,9 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the size query and the forward calls.
 struct Workspace {
     size_t offsets, padded_offsets, perm, inv;  // routing tables
-    size_t H, P;                                // decode path
+    size_t H, Y;                                // decode path
     size_t xperm, Hp, Yg;                       // tensor-core path
     size_t total;
-    int nsplit;
     int64_t rows_padded;  // upper bound of the padded expert-grouped rows
 };
 
@@ -91,9 +90,8 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     w.inv = take(sizeof(int32_t) * (size_t)A);
     (void)T;
     if (!prefill) {
-        w.nsplit = jmoe::decode_split_for(f);
         w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
-        w.P = take(sizeof(float) * (size_t)w.nsplit * (size_t)A * (size_t)d);
+        w.Y = take(sizeof(float) * (size_t)A * (size_t)d);
     } else {
         const int64_t tm = jmoe::kPrefillTileM;
         w.rows_padded = (A + (int64_t)E * (tm - 1) + tm - 1) / tm * tm;
@@ -154,8 +152,8 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         jmoe::DecodeArgs a{};
         a.x = x; a.T = T; a.A = A; a.d = d; a.f = f; a.E = E; a.top_k = k;
         a.wgu = desc->w_gu; a.sgu = desc->s_gu; a.wd = desc->w_d; a.sd = desc->s_d;
-        a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm; a.inv = inv;
-        a.H = at(w.H); a.P = static_cast<float*>(at(w.P)); a.nsplit = w.nsplit;
+        a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm;
+        a.H = at(w.H); a.Y = static_cast<float*>(at(w.Y));
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;

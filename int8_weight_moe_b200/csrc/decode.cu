@@ -1,39 +1,82 @@
-// Decode path of the expert MLPs: few tokens per expert, so the work is a
+// Decode path of the expert MLPs: few tokens per expert, so the work is one
 // stream over the INT8 weights of the experts that some token selected
-// (HBM-bound; weights of untouched experts are never read).
+// (HBM-bound; the weights of untouched experts are never read).
 //
 // ExpertsInt8 ("Jamba-1.5: Hybrid Transformer-Mamba Models at Scale", paper
 // summary, section "ExpertsInt8 Quantization (Section 3.1)", steps 3-4): the
-// INT8 weights cross HBM once and are turned back into BF16 on chip, the
-// activations stay BF16.  Here each weight byte goes HBM -> registers, is
+// INT8 weights cross HBM once and are turned back into BF16 on chip; the
+// activations stay BF16.  Here every weight byte goes HBM -> registers, is
 // converted exactly to bf16 (the scale is applied once per output channel
-// after the dot product, an exact refactoring of sum_k x_k (q_k s)), and
-// feeds an mma.sync m16n8k16 whose 8 columns are up to 8 tokens of the
-// expert; accumulation is fp32.
+// after the dot product, an exact refactoring of sum_k x_k (q_k s)), and feeds
+// an mma.sync m16n8k16 whose 8 columns are up to 8 tokens of the expert;
+// accumulation is fp32.
 //
 // Fragment trick: the dot product does not care in which order k is summed,
 // so the 16 k-columns of every MMA step are a permutation of the 64-wide
 // k-block chosen such that thread (g = lane/4, c = lane%4) needs exactly
-// bytes [16c, 16c+16) of weight rows g and g+8 for all four MMA steps of the
-// block -- one 16-byte load per row -- and the matching 16 consecutive bf16
-// of its token.  Step s uses physical k = 16c + 4s + {0,1} for the fragment
+// bytes [16c, 16c+16) of weight rows g and g+8 for the block's four MMA
+// steps -- one 16-byte load per row -- and the matching 16 consecutive bf16
+// of its token.  Step s uses physical k = 16c + 4s + {0,1} for fragment
 // columns 2c, 2c+1 and 16c + 4s + {2,3} for columns 2c+8, 2c+9.
 //
-// Kernels:
-//   k_decode_gateup : h = silu(s_g * x.q_g) * (s_u * x.q_u) for every
-//                     (expert, 16 channels) per warp, h stored bf16 in
-//                     expert-grouped slot order;
-//   k_decode_down   : raw partial sums of h.q_d over one K split;
-//   k_decode_combine: out_t = bf16( sum_j g_tj * s_d[m] * sum_splits ).
+// Work decomposition (persistent, one 16-warp CTA per SM): a work unit is
+// (touched expert, 16 output channels, one pass of up to 8*NCH tokens).  The
+// CTA's 16 warps split the unit's K range into equal contiguous pieces, so a
+// unit is small (a 16-row weight slab) and the units divide evenly over the
+// CTAs; each warp keeps a ring of kDepth weight steps in registers that runs
+// ahead across unit boundaries, so HBM never waits for a reduction.  At the
+// end of a unit the 16 partial accumulators are summed through shared memory
+// in warp order (deterministic) and warp 0 writes the result:
+//   k_gemv_gateup : h = silu(s_g * x.q_g) * (s_u * x.q_u) -> H (bf16, slot order)
+//   k_gemv_down   : y = gate * (s_d * h.q_d)               -> Y (fp32, one row per
+//                                                             token->expert assignment)
+// and launch_finalize sums each token's rows of Y into the bf16 output.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace jmoe {
 namespace {
 
-constexpr int kWarpsPerBlock = 4;
-constexpr int kChPerWarp = 16;
-constexpr int kDepth = 3;  // weight steps in flight per warp (ring of registers)
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kDepth = 4;  // ring slots per warp: three 64-wide k steps in flight
+constexpr int kMaxE = 16;
+
+// Units of one launch, built by every CTA from the expert offsets.
+struct Units {
+    int start[kMaxE + 1];  // first unit of expert e
+    int groups;            // 16-channel groups per expert
+};
+
+__device__ __forceinline__ void build_units(Units& u, const int32_t* offsets, int E, int groups,
+                                            int tokens_per_pass) {
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int cnt = offsets[e + 1] - offsets[e];
+            const int passes = cnt > 0 ? (cnt + tokens_per_pass - 1) / tokens_per_pass : 0;
+            u.start[e] = run;
+            run += passes * groups;
+        }
+        u.start[E] = run;
+        u.groups = groups;
+    }
+}
+
+struct Unit {
+    int e, group, pass;
+};
+
+__device__ __forceinline__ Unit decode_unit(const Units& u, int E, int unit) {
+    int e = 0;
+    while (e + 1 < E && u.start[e + 1] <= unit) ++e;
+    const int local = unit - u.start[e];
+    Unit r;
+    r.e = e;
+    r.group = local % u.groups;
+    r.pass = local / u.groups;
+    return r;
+}
 
 // x (or h) fragment for one token row: 16 consecutive bf16 starting at p.
 __device__ __forceinline__ void load_b(const uint16_t* p, uint32_t (&b)[8]) {
@@ -62,180 +105,273 @@ __device__ __forceinline__ void mma_block(float (&acc)[4], const uint4& q0, cons
 }
 
 template <int NCH>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    k_decode_gateup(const uint16_t* __restrict__ x, int top_k, int64_t d, int64_t f,
-                    const int8_t* __restrict__ wgu, const float* __restrict__ sgu,
-                    const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
-                    uint16_t* __restrict__ H) {
-    const int e = blockIdx.y;
-    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const int64_t ch0 = ((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * kChPerWarp;
-    if (ch0 >= f) return;
-    const int base = offsets[e];
-    const int cnt = offsets[e + 1] - base;
-    if (cnt <= 0) return;
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemv_gateup(const uint16_t* __restrict__ x, int top_k, int E, int64_t d, int64_t f,
+                  const int8_t* __restrict__ wgu, const float* __restrict__ sgu,
+                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+                  uint16_t* __restrict__ H) {
+    __shared__ Units U;
+    __shared__ int s_off[kMaxE + 1];
+    // partial sums of the 16 warps, double-buffered by unit parity (dynamic:
+    // 32 KB per token chunk)
+    extern __shared__ float red_raw[];
+    auto red = reinterpret_cast<float(*)[kWarps][32][NCH][8]>(red_raw);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, c = lane & 3;
+    if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
+    build_units(U, offsets, E, (int)(f / 16), 8 * NCH);
+    __syncthreads();
+    const int n_units = U.start[E];
+    const int G = gridDim.x;
+    const int n_mine = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
+    const int S = (int)(d / 64);
+    const int nw = (S + kWarps - 1) / kWarps;
+    const int s_lo = warp * nw;
+    const int s_hi = min(S, s_lo + nw);
+    const int64_t total = (int64_t)n_mine * nw;
 
-    const int8_t* wg0 = wgu + ((int64_t)e * 2 * f + ch0 + g) * d + 16 * c;
-    const int8_t* wg1 = wg0 + 8 * d;
-    const int8_t* wu0 = wg0 + f * d;
-    const int8_t* wu1 = wu0 + 8 * d;
-    const int64_t nsteps = d / 64;
+    // ---- prefetch cursor (unit iteration pi, step pj) and its slab pointers
+    int pi = 0, pj = 0;
+    const int8_t* pw[4] = {nullptr, nullptr, nullptr, nullptr};
+    auto set_prefetch_unit = [&](int it) {
+        const Unit u = decode_unit(U, E, blockIdx.x + it * G);
+        const int8_t* base = wgu + ((int64_t)u.e * 2 * f + u.group * 16 + g) * d + 16 * c +
+                             (int64_t)s_lo * 64;
+        pw[0] = base;
+        pw[1] = base + 8 * d;
+        pw[2] = base + f * d;
+        pw[3] = base + f * d + 8 * d;
+    };
+    uint4 ring[kDepth][4];
+    auto issue = [&](int slot) {
+        // load step (pi, pj) into ring[slot]; the padding steps of short K pieces load nothing
+        if (s_lo + pj < s_hi) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) ring[slot][m] = ldg_stream_v4(pw[m] + (int64_t)pj * 64);
+        }
+        if (++pj == nw) {
+            pj = 0;
+            if (++pi < n_mine) set_prefetch_unit(pi);
+        }
+    };
+    if (n_mine > 0) set_prefetch_unit(0);
+#pragma unroll
+    for (int p = 0; p < kDepth - 1; ++p)
+        if (p < total) issue(p);
 
-    for (int pass = 0; pass * NCH * 8 < cnt; ++pass) {
-        const int nch = min(NCH, (cnt - pass * NCH * 8 + 7) / 8);  // warp-uniform
-        const uint16_t* xp[NCH];
+    // ---- consumer state
+    float ag[NCH][4], au[NCH][4];
+#pragma unroll
+    for (int n = 0; n < NCH; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ag[n][i] = au[n][i] = 0.0f;
+    Unit cu{};
+    const uint16_t* xp[NCH];
+    int cnt_pass = 0;
+    int ci = 0, cj = 0;
+    auto set_consumer_unit = [&](int it) {
+        cu = decode_unit(U, E, blockIdx.x + it * G);
+        const int base = s_off[cu.e];
+        const int cnt = s_off[cu.e + 1] - base;
+        const int t0 = cu.pass * 8 * NCH;
+        cnt_pass = min(8 * NCH, cnt - t0);
 #pragma unroll
         for (int n = 0; n < NCH; ++n) {
-            const int slot = (pass * NCH + n) * 8 + g;
-            xp[n] = slot < cnt ? x + (int64_t)(perm[base + slot] / top_k) * d + 16 * c : nullptr;
+            const int slot = n * 8 + g;
+            xp[n] = slot < cnt_pass
+                        ? x + (int64_t)(perm[base + t0 + slot] / top_k) * d + 16 * c + s_lo * 64
+                        : nullptr;
         }
-        float ag[NCH][4], au[NCH][4];
-#pragma unroll
-        for (int n = 0; n < NCH; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) ag[n][i] = au[n][i] = 0.0f;
+    };
+    if (n_mine > 0) set_consumer_unit(0);
 
-        uint4 ring[kDepth][4];
+    for (int64_t q0 = 0; q0 < total; q0 += kDepth) {
 #pragma unroll
-        for (int p = 0; p < kDepth - 1; ++p) {
-            if (p < nsteps) {
-                ring[p][0] = ldg_stream_v4(wg0 + p * 64);
-                ring[p][1] = ldg_stream_v4(wg1 + p * 64);
-                ring[p][2] = ldg_stream_v4(wu0 + p * 64);
-                ring[p][3] = ldg_stream_v4(wu1 + p * 64);
-            }
-        }
-        for (int64_t i0 = 0; i0 < nsteps; i0 += kDepth) {
-#pragma unroll
-            for (int j = 0; j < kDepth; ++j) {
-                const int64_t i = i0 + j;
-                if (i < nsteps) {
-                    const int64_t ip = i + kDepth - 1;
-                    if (ip < nsteps) {
-                        const int slot = (j + kDepth - 1) % kDepth;
-                        ring[slot][0] = ldg_stream_v4(wg0 + ip * 64);
-                        ring[slot][1] = ldg_stream_v4(wg1 + ip * 64);
-                        ring[slot][2] = ldg_stream_v4(wu0 + ip * 64);
-                        ring[slot][3] = ldg_stream_v4(wu1 + ip * 64);
-                    }
+        for (int jj = 0; jj < kDepth; ++jj) {
+            const int64_t q = q0 + jj;
+            if (q < total) {
+                if (q + kDepth - 1 < total) issue((jj + kDepth - 1) % kDepth);
+                if (s_lo + cj < s_hi) {
 #pragma unroll
                     for (int n = 0; n < NCH; ++n) {
-                        if (n < nch) {
+                        if (n * 8 < cnt_pass) {
                             uint32_t b[8];
-                            load_b(xp[n] ? xp[n] + i * 64 : nullptr, b);
-                            mma_block(ag[n], ring[j][0], ring[j][1], b);
-                            mma_block(au[n], ring[j][2], ring[j][3], b);
+                            load_b(xp[n] ? xp[n] + cj * 64 : nullptr, b);
+                            mma_block(ag[n], ring[jj][0], ring[jj][1], b);
+                            mma_block(au[n], ring[jj][2], ring[jj][3], b);
                         }
                     }
                 }
-            }
-        }
-        // epilogue: rows = channels (g, g+8), cols = token slots (2c, 2c+1)
-        const float sg0 = sgu[(int64_t)e * 2 * f + ch0 + g];
-        const float sg1 = sgu[(int64_t)e * 2 * f + ch0 + g + 8];
-        const float su0 = sgu[(int64_t)e * 2 * f + f + ch0 + g];
-        const float su1 = sgu[(int64_t)e * 2 * f + f + ch0 + g + 8];
+                if (++cj == nw) {
+                    // end of unit: reduce the 16 warps' partials, warp 0 writes h
+                    const int buf = ci & 1;
 #pragma unroll
-        for (int n = 0; n < NCH; ++n) {
+                    for (int n = 0; n < NCH; ++n)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int slot = (pass * NCH + n) * 8 + 2 * c + (i & 1);
-                const int row = g + (i >> 1) * 8;
-                if (n < nch && slot < cnt) {
-                    const float gs = (i >> 1) ? sg1 : sg0;
-                    const float us = (i >> 1) ? su1 : su0;
-                    const float h = silu_f32(gs * ag[n][i]) * (us * au[n][i]);
-                    H[(int64_t)(base + slot) * f + ch0 + row] =
-                        __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                        for (int i = 0; i < 4; ++i) {
+                            red[buf][warp][lane][n][i] = ag[n][i];
+                            red[buf][warp][lane][n][4 + i] = au[n][i];
+                            ag[n][i] = au[n][i] = 0.0f;
+                        }
+                    __syncthreads();
+                    if (warp == 0) {
+                        const int base = s_off[cu.e] + cu.pass * 8 * NCH;
+                        const int64_t ch0 = (int64_t)cu.group * 16;
+                        const float* sg = sgu + (int64_t)cu.e * 2 * f + ch0;
+#pragma unroll
+                        for (int n = 0; n < NCH; ++n) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float vg = 0.f, vu = 0.f;
+                                for (int w2 = 0; w2 < kWarps; ++w2) {
+                                    vg += red[buf][w2][lane][n][i];
+                                    vu += red[buf][w2][lane][n][4 + i];
+                                }
+                                const int slot = n * 8 + 2 * c + (i & 1);
+                                const int row = g + (i >> 1) * 8;
+                                if (slot < cnt_pass) {
+                                    const float h = silu_f32(sg[row] * vg) * (sg[f + row] * vu);
+                                    H[(int64_t)(base + slot) * f + ch0 + row] =
+                                        __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                                }
+                            }
+                        }
+                    }
+                    cj = 0;
+                    if (++ci < n_mine) set_consumer_unit(ci);
                 }
             }
         }
     }
 }
 
-// Raw partial sums P[z][slot][m] = sum over k in split z of h[slot][k] q_d[m][k].
 template <int NCH>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    k_decode_down(const uint16_t* __restrict__ H, int64_t d, int64_t f, int64_t ksplit,
-                  const int8_t* __restrict__ wd, const int32_t* __restrict__ offsets, int64_t A,
-                  float* __restrict__ P) {
-    const int e = blockIdx.y;
-    const int z = blockIdx.z;
-    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const int64_t m0 = ((int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * kChPerWarp;
-    if (m0 >= d) return;
-    const int base = offsets[e];
-    const int cnt = offsets[e + 1] - base;
-    if (cnt <= 0) return;
-    const int64_t k_begin = (int64_t)z * ksplit;
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemv_down(const uint16_t* __restrict__ H, int E, int64_t d, int64_t f,
+                const int8_t* __restrict__ wd, const float* __restrict__ sd,
+                const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+                const float* __restrict__ gates, float* __restrict__ Y) {
+    __shared__ Units U;
+    __shared__ int s_off[kMaxE + 1];
+    __shared__ float red[2][kWarps][32][NCH][4];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, c = lane & 3;
+    if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
+    build_units(U, offsets, E, (int)(d / 16), 8 * NCH);
+    __syncthreads();
+    const int n_units = U.start[E];
+    const int G = gridDim.x;
+    const int n_mine = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
+    const int S = (int)(f / 64);
+    const int nw = (S + kWarps - 1) / kWarps;
+    const int s_lo = warp * nw;
+    const int s_hi = min(S, s_lo + nw);
+    const int64_t total = (int64_t)n_mine * nw;
 
-    const int8_t* w0 = wd + ((int64_t)e * d + m0 + g) * f + k_begin + 16 * c;
-    const int8_t* w1 = w0 + 8 * f;
-    const int64_t nsteps = ksplit / 64;
+    int pi = 0, pj = 0;
+    const int8_t* pw[2] = {nullptr, nullptr};
+    auto set_prefetch_unit = [&](int it) {
+        const Unit u = decode_unit(U, E, blockIdx.x + it * G);
+        const int8_t* base =
+            wd + ((int64_t)u.e * d + u.group * 16 + g) * f + 16 * c + (int64_t)s_lo * 64;
+        pw[0] = base;
+        pw[1] = base + 8 * f;
+    };
+    uint4 ring[kDepth][2];
+    auto issue = [&](int slot) {
+        if (s_lo + pj < s_hi) {
+            ring[slot][0] = ldg_stream_v4(pw[0] + (int64_t)pj * 64);
+            ring[slot][1] = ldg_stream_v4(pw[1] + (int64_t)pj * 64);
+        }
+        if (++pj == nw) {
+            pj = 0;
+            if (++pi < n_mine) set_prefetch_unit(pi);
+        }
+    };
+    if (n_mine > 0) set_prefetch_unit(0);
+#pragma unroll
+    for (int p = 0; p < kDepth - 1; ++p)
+        if (p < total) issue(p);
 
-    for (int pass = 0; pass * NCH * 8 < cnt; ++pass) {
-        const int nch = min(NCH, (cnt - pass * NCH * 8 + 7) / 8);
-        const uint16_t* hp[NCH];
+    float acc[NCH][4];
+#pragma unroll
+    for (int n = 0; n < NCH; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
+    Unit cu{};
+    const uint16_t* hp[NCH];
+    int cnt_pass = 0;
+    int ci = 0, cj = 0;
+    auto set_consumer_unit = [&](int it) {
+        cu = decode_unit(U, E, blockIdx.x + it * G);
+        const int base = s_off[cu.e];
+        const int cnt = s_off[cu.e + 1] - base;
+        const int t0 = cu.pass * 8 * NCH;
+        cnt_pass = min(8 * NCH, cnt - t0);
 #pragma unroll
         for (int n = 0; n < NCH; ++n) {
-            const int slot = (pass * NCH + n) * 8 + g;
-            hp[n] = slot < cnt ? H + (int64_t)(base + slot) * f + k_begin + 16 * c : nullptr;
+            const int slot = n * 8 + g;
+            hp[n] = slot < cnt_pass ? H + (int64_t)(base + t0 + slot) * f + 16 * c + s_lo * 64
+                                    : nullptr;
         }
-        float acc[NCH][4];
-#pragma unroll
-        for (int n = 0; n < NCH; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
+    };
+    if (n_mine > 0) set_consumer_unit(0);
 
-        uint4 ring[kDepth][2];
+    for (int64_t q0 = 0; q0 < total; q0 += kDepth) {
 #pragma unroll
-        for (int p = 0; p < kDepth - 1; ++p) {
-            if (p < nsteps) {
-                ring[p][0] = ldg_stream_v4(w0 + p * 64);
-                ring[p][1] = ldg_stream_v4(w1 + p * 64);
-            }
-        }
-        for (int64_t i0 = 0; i0 < nsteps; i0 += kDepth) {
-#pragma unroll
-            for (int j = 0; j < kDepth; ++j) {
-                const int64_t i = i0 + j;
-                if (i < nsteps) {
-                    const int64_t ip = i + kDepth - 1;
-                    if (ip < nsteps) {
-                        const int slot = (j + kDepth - 1) % kDepth;
-                        ring[slot][0] = ldg_stream_v4(w0 + ip * 64);
-                        ring[slot][1] = ldg_stream_v4(w1 + ip * 64);
-                    }
+        for (int jj = 0; jj < kDepth; ++jj) {
+            const int64_t q = q0 + jj;
+            if (q < total) {
+                if (q + kDepth - 1 < total) issue((jj + kDepth - 1) % kDepth);
+                if (s_lo + cj < s_hi) {
 #pragma unroll
                     for (int n = 0; n < NCH; ++n) {
-                        if (n < nch) {
+                        if (n * 8 < cnt_pass) {
                             uint32_t b[8];
-                            load_b(hp[n] ? hp[n] + i * 64 : nullptr, b);
-                            mma_block(acc[n], ring[j][0], ring[j][1], b);
+                            load_b(hp[n] ? hp[n] + cj * 64 : nullptr, b);
+                            mma_block(acc[n], ring[jj][0], ring[jj][1], b);
                         }
                     }
                 }
-            }
-        }
+                if (++cj == nw) {
+                    const int buf = ci & 1;
 #pragma unroll
-        for (int n = 0; n < NCH; ++n) {
+                    for (int n = 0; n < NCH; ++n)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int slot = (pass * NCH + n) * 8 + 2 * c + (i & 1);
-                const int row = g + (i >> 1) * 8;
-                if (n < nch && slot < cnt)
-                    P[((int64_t)z * A + base + slot) * d + m0 + row] = acc[n][i];
+                        for (int i = 0; i < 4; ++i) {
+                            red[buf][warp][lane][n][i] = acc[n][i];
+                            acc[n][i] = 0.0f;
+                        }
+                    __syncthreads();
+                    if (warp == 0) {
+                        const int base = s_off[cu.e] + cu.pass * 8 * NCH;
+                        const int64_t m0 = (int64_t)cu.group * 16;
+                        const float* s = sd + (int64_t)cu.e * d + m0;
+#pragma unroll
+                        for (int n = 0; n < NCH; ++n) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float v = 0.f;
+                                for (int w2 = 0; w2 < kWarps; ++w2) v += red[buf][w2][lane][n][i];
+                                const int slot = n * 8 + 2 * c + (i & 1);
+                                const int row = g + (i >> 1) * 8;
+                                if (slot < cnt_pass) {
+                                    const int a = perm[base + slot];
+                                    Y[(int64_t)a * d + m0 + row] = gates[a] * (s[row] * v);
+                                }
+                            }
+                        }
+                    }
+                    cj = 0;
+                    if (++ci < n_mine) set_consumer_unit(ci);
+                }
             }
         }
     }
 }
 
-// out[t][m] = bf16( sum_j g_tj * (s_d[e_j][m] * sum_z P[z][inv[a]][m]) ), a = t*top_k + j.
+// out[t] = bf16( sum_j Y[t*top_k + j] ) over the token's valid assignments.
 __global__ void __launch_bounds__(256)
-    k_decode_combine(const float* __restrict__ P, int nsplit, int64_t A, int64_t T, int64_t d,
-                     int top_k, int E, const int32_t* __restrict__ ids,
-                     const float* __restrict__ gates, const int32_t* __restrict__ inv,
-                     const float* __restrict__ sd, uint16_t* __restrict__ out) {
+    k_finalize(const float* __restrict__ Y, int64_t T, int64_t d, int top_k, int E,
+               const int32_t* __restrict__ ids, uint16_t* __restrict__ out) {
     const int64_t nvec = d / 4;
     const int64_t total = T * nvec;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -245,19 +381,12 @@ __global__ void __launch_bounds__(256)
         for (int j = 0; j < top_k; ++j) {
             const int64_t a = t * top_k + j;
             const int e = ids[a];
-            const int slot = inv[a];
-            if (e < 0 || e >= E || slot < 0) continue;
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int z = 0; z < nsplit; ++z) {
-                const float4 p = *reinterpret_cast<const float4*>(P + ((int64_t)z * A + slot) * d + m);
-                y[0] += p.x; y[1] += p.y; y[2] += p.z; y[3] += p.w;
-            }
-            const float4 s = *reinterpret_cast<const float4*>(sd + (int64_t)e * d + m);
-            const float gw = gates[a];
-            o[0] += gw * (s.x * y[0]);
-            o[1] += gw * (s.y * y[1]);
-            o[2] += gw * (s.z * y[2]);
-            o[3] += gw * (s.w * y[3]);
+            if (e < 0 || e >= E) continue;
+            const float4 y = *reinterpret_cast<const float4*>(Y + a * d + m);
+            o[0] += y.x;
+            o[1] += y.y;
+            o[2] += y.z;
+            o[3] += y.w;
         }
         uint2 r;
         r.x = pack_bf16x2(o[0], o[1]);
@@ -268,51 +397,47 @@ __global__ void __launch_bounds__(256)
 
 template <int NCH>
 cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
-    dim3 g1((unsigned)((a.f + kWarpsPerBlock * kChPerWarp - 1) / (kWarpsPerBlock * kChPerWarp)),
-            (unsigned)a.E);
-    if (a.mark) a.mark(2, false, stream);
-    k_decode_gateup<NCH><<<g1, kWarpsPerBlock * 32, 0, stream>>>(
-        (const uint16_t*)a.x, a.top_k, a.d, a.f, a.wgu, a.sgu, a.offsets, a.perm, (uint16_t*)a.H);
-    if (a.mark) a.mark(2, true, stream);
-    cudaError_t err = cudaGetLastError();
+    const int grid = a.num_sms;
+    const int red_bytes = (int)(2 * kWarps * 32 * NCH * 8 * sizeof(float));
+    cudaError_t err = cudaFuncSetAttribute(k_gemv_gateup<NCH>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, red_bytes);
     if (err != cudaSuccess) return err;
-    dim3 g2((unsigned)((a.d + kWarpsPerBlock * kChPerWarp - 1) / (kWarpsPerBlock * kChPerWarp)),
-            (unsigned)a.E, (unsigned)a.nsplit);
+    if (a.mark) a.mark(2, false, stream);
+    k_gemv_gateup<NCH><<<grid, kThreads, red_bytes, stream>>>((const uint16_t*)a.x, a.top_k, a.E, a.d,
+                                                      a.f, a.wgu, a.sgu, a.offsets, a.perm,
+                                                      (uint16_t*)a.H);
+    if (a.mark) a.mark(2, true, stream);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
     if (a.mark) a.mark(3, false, stream);
-    k_decode_down<NCH><<<g2, kWarpsPerBlock * 32, 0, stream>>>(
-        (const uint16_t*)a.H, a.d, a.f, a.f / a.nsplit, a.wd, a.offsets, a.A, a.P);
+    k_gemv_down<NCH><<<grid, kThreads, 0, stream>>>((const uint16_t*)a.H, a.E, a.d, a.f, a.wd,
+                                                    a.sd, a.offsets, a.perm, a.gates, a.Y);
     if (a.mark) a.mark(3, true, stream);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int decode_split_for(int64_t f) {
-    // largest power of two <= 8 that keeps each K split a multiple of 64
-    int s = 8;
-    while (s > 1 && (f % (64 * s)) != 0) s >>= 1;
-    return s;
+cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int E,
+                            const int32_t* ids, void* out, int num_sms, cudaStream_t stream) {
+    const int64_t total = T * (d / 4);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    if (blocks < 1) blocks = 1;
+    k_finalize<<<(unsigned)blocks, 256, 0, stream>>>(Y, T, d, top_k, E, ids,
+                                                     static_cast<uint16_t*>(out));
+    return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (a.T == 0) return cudaSuccess;
-    cudaError_t err;
-    if (a.max_per_expert <= 8)
-        err = launch_decode_nch<1>(a, stream);
-    else if (a.max_per_expert <= 16)
-        err = launch_decode_nch<2>(a, stream);
-    else
-        err = launch_decode_nch<4>(a, stream);
+    cudaError_t err = a.max_per_expert <= 8 ? launch_decode_nch<1>(a, stream)
+                                            : launch_decode_nch<2>(a, stream);
     if (err != cudaSuccess) return err;
-    const int64_t total = a.T * (a.d / 4);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > (int64_t)a.num_sms * 8) blocks = (int64_t)a.num_sms * 8;
     if (a.mark) a.mark(4, false, stream);
-    k_decode_combine<<<(unsigned)blocks, 256, 0, stream>>>(a.P, a.nsplit, a.A, a.T, a.d, a.top_k,
-                                                           a.E, a.ids, a.gates, a.inv, a.sd,
-                                                           (uint16_t*)a.out);
+    err = launch_finalize(a.Y, a.T, a.d, a.top_k, a.E, a.ids, a.out, a.num_sms, stream);
     if (a.mark) a.mark(4, true, stream);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace jmoe

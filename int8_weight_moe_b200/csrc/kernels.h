@@ -46,17 +46,16 @@ struct DecodeArgs {
     const float* gates;   // [T][top_k]
     const int32_t* offsets;  // [E+1]
     const int32_t* perm;     // [A]
-    const int32_t* inv;      // [A]
-    void* H;              // bf16 [A][f]   (workspace)
-    float* P;             // fp32 [nsplit][A][d] (workspace)
-    int nsplit;
+    void* H;              // bf16 [A][f], expert-grouped slot order (workspace)
+    float* Y;             // fp32 [A][d], one row per assignment (workspace)
     int64_t max_per_expert;  // host-side bound used to size register tiles
     void* out;            // bf16 [T][d]
     int num_sms;
     StageMark mark;
 };
 
-int decode_split_for(int64_t f);
+cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int E,
+                            const int32_t* ids, void* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 

@@ -372,33 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// out[t] = bf16( sum_j Y[t*top_k + j] ) over the valid assignments of token t.
-__global__ void __launch_bounds__(256)
-    k_finalize(const float* __restrict__ Y, int64_t T, int64_t d, int top_k, int E,
-               const int32_t* __restrict__ ids, uint16_t* __restrict__ out) {
-    const int64_t nvec = d / 4;
-    const int64_t total = T * nvec;
-    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
-         v += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = v / nvec, m = (v % nvec) * 4;
-        float o[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < top_k; ++j) {
-            const int64_t a = t * top_k + j;
-            const int e = ids[a];
-            if (e < 0 || e >= E) continue;
-            const float4 y = *reinterpret_cast<const float4*>(Y + a * d + m);
-            o[0] += y.x;
-            o[1] += y.y;
-            o[2] += y.z;
-            o[3] += y.w;
-        }
-        uint2 r;
-        r.x = pack_bf16x2(o[0], o[1]);
-        r.y = pack_bf16x2(o[2], o[3]);
-        *reinterpret_cast<uint2*>(out + t * d + m) = r;
-    }
-}
-
 // ----------------------------------------------------------------------------- host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -508,13 +481,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
 
     // 4. out[t] = bf16(sum over the token's assignments)
-    const int64_t total = a.T * (a.d / 4);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > (int64_t)a.num_sms * 8) blocks = (int64_t)a.num_sms * 8;
     if (a.mark) a.mark(4, false, stream);
-    k_finalize<<<(unsigned)blocks, 256, 0, stream>>>(a.Yg, a.T, a.d, a.top_k, a.E, a.ids,
-                                                     static_cast<uint16_t*>(a.out));
+    err = launch_finalize(a.Yg, a.T, a.d, a.top_k, a.E, a.ids, a.out, a.num_sms, stream);
     if (a.mark) a.mark(4, true, stream);
+    if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 

@@ -6,52 +6,82 @@
 // g = softmax(W_r h) with W_r of shape [n, d]; the top K = 2 experts are
 // selected and their probabilities renormalised over the selected set.
 //
-// One warp per token.  Lane j accumulates the fp64 partial sum
-// p_j = sum over k = j, j+32, ... (ascending) of x_k * w_ek for every expert;
-// the 32 partial sums are then combined by the halving tree
-// p_j += p_{j+o}, o = 16, 8, 4, 2, 1 (a shuffle-down reduction), the bias is
-// added in fp64 and the result rounded once to fp32.  The products are exact
-// in fp64, so this fixed order makes the logits -- and the top-k ids chosen
-// from them -- reproducible bit for bit.  Softmax and gates are fp32.
+// Summation order (fixed, so the logits -- and the top-k ids chosen from them
+// -- are reproducible bit for bit): for every (token, expert), lane j of a
+// warp accumulates in fp64 the partial sum p_j = sum over k = j, j+32, ...
+// (ascending) of x_k * w_ek; the 32 partial sums are combined by the halving
+// tree p_j += p_{j+o}, o = 16, 8, 4, 2, 1 (a shuffle-down reduction); the bias
+// is added in fp64 and the result rounded once to fp32.  The products are
+// exact in fp64 (8-bit x 24-bit significands).
+//
+// Work split: a CTA of 4 warps handles kTok tokens; warp w owns experts
+// w, w+4, w+8, w+12, so each lane keeps 4 x kTok independent fp64
+// accumulators and every router weight it loads serves kTok tokens.  The
+// k loop is unrolled so the loads of several steps are in flight together.
+// Softmax (fp32) and top-k run in the first threads of the CTA afterwards.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace jmoe {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;
 constexpr int kMaxE = 16;
+constexpr int kPerWarp = kMaxE / kWarps;
 
+template <int kTok>
 __global__ void __launch_bounds__(kWarps * 32)
     k_route(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
             const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
             float* __restrict__ gates, float* __restrict__ logits) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp_global = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
-    const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-    for (int64_t t = warp_global; t < T; t += nwarps) {
-        const uint16_t* xr = x + t * d;
-        double acc[kMaxE];
+    __shared__ float s_logit[kTok][kMaxE];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int64_t t0 = (int64_t)blockIdx.x * kTok; t0 < T; t0 += (int64_t)gridDim.x * kTok) {
+        double acc[kTok][kPerWarp];
 #pragma unroll
-        for (int e = 0; e < kMaxE; ++e) acc[e] = 0.0;
+        for (int t = 0; t < kTok; ++t)
+#pragma unroll
+            for (int i = 0; i < kPerWarp; ++i) acc[t][i] = 0.0;
+        const uint16_t* xr[kTok];
+#pragma unroll
+        for (int t = 0; t < kTok; ++t) xr[t] = x + min(t0 + t, T - 1) * d;  // clamp: tail tokens
+#pragma unroll 4
         for (int64_t k = lane; k < d; k += 32) {
-            const double xk = (double)bf16_bits_to_f32(__ldg(xr + k));
+            double xk[kTok];
 #pragma unroll
-            for (int e = 0; e < kMaxE; ++e)
-                if (e < E) acc[e] = fma(xk, (double)__ldg(wr + (int64_t)e * d + k), acc[e]);
-        }
+            for (int t = 0; t < kTok; ++t) xk[t] = (double)bf16_bits_to_f32(__ldg(xr[t] + k));
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
+            for (int i = 0; i < kPerWarp; ++i) {
+                const int e = warp + kWarps * i;
+                if (e < E) {
+                    const double w = (double)__ldg(wr + (int64_t)e * d + k);
 #pragma unroll
-            for (int e = 0; e < kMaxE; ++e) acc[e] += __shfl_down_sync(0xffffffffu, acc[e], o);
-        }
-        if (lane == 0) {
-            float l[kMaxE];
-#pragma unroll
-            for (int e = 0; e < kMaxE; ++e) {
-                const double b = (bias && e < E) ? (double)bias[e] : 0.0;
-                l[e] = e < E ? __double2float_rn(acc[e] + b) : -INFINITY;
+                    for (int t = 0; t < kTok; ++t) acc[t][i] = fma(xk[t], w, acc[t][i]);
+                }
             }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int t = 0; t < kTok; ++t)
+#pragma unroll
+                for (int i = 0; i < kPerWarp; ++i)
+                    acc[t][i] += __shfl_down_sync(0xffffffffu, acc[t][i], o);
+        if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < kPerWarp; ++i) {
+                const int e = warp + kWarps * i;
+                if (e < E) {
+                    const double b = bias ? (double)bias[e] : 0.0;
+#pragma unroll
+                    for (int t = 0; t < kTok; ++t) s_logit[t][e] = __double2float_rn(acc[t][i] + b);
+                }
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x < kTok && t0 + threadIdx.x < T) {
+            const int64_t t = t0 + threadIdx.x;
+            const float* l = s_logit[threadIdx.x];
             if (logits)
                 for (int e = 0; e < E; ++e) logits[t * E + e] = l[e];
             // top-k on the fp32 logits: strict '>' keeps the lower index on ties
@@ -59,11 +89,10 @@ __global__ void __launch_bounds__(kWarps * 32)
             for (int e = 1; e < E; ++e)
                 if (l[e] > l[e1]) e1 = e;
             int e2 = -1;
-            if (top_k == 2) {
+            if (top_k == 2)
                 for (int e = 0; e < E; ++e)
                     if (e != e1 && (e2 < 0 || l[e] > l[e2])) e2 = e;
-            }
-            // fp32 softmax over all E experts
+            // fp32 softmax over all E experts, renormalised over the selection
             float p[kMaxE];
             const float m = l[e1];
             float z = 0.0f;
@@ -83,6 +112,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                 gates[2 * t + 1] = p[e2] / sel;
             }
         }
+        __syncthreads();
     }
 }
 
@@ -92,11 +122,19 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
                          const float* bias, int E, int top_k, int32_t* ids, float* gates,
                          float* logits, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    int64_t blocks = (T + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)num_sms * 16;
-    if (blocks > cap) blocks = cap;
-    k_route<<<(unsigned)blocks, kWarps * 32, 0, stream>>>((const uint16_t*)x_bf16, T, d, w_router,
-                                                          bias, E, top_k, ids, gates, logits);
+    // Few tokens: one token per CTA spreads them over more SMs (latency);
+    // many tokens: 4 per CTA cuts the router-weight traffic fourfold.
+    if (T < (int64_t)num_sms * 8) {
+        int64_t blocks = T;
+        k_route<1><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+            (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, ids, gates, logits);
+    } else {
+        int64_t blocks = (T + 3) / 4;
+        const int64_t cap = (int64_t)num_sms * 16;
+        if (blocks > cap) blocks = cap;
+        k_route<4><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+            (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, ids, gates, logits);
+    }
     return cudaGetLastError();
 }
 

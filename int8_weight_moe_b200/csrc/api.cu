@@ -157,6 +157,7 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;
+        a.err = err;
         return from_cuda(jmoe::launch_decode(a, stream));
     }
     jmoe::PrefillArgs p{};

@@ -5,63 +5,79 @@
 // ExpertsInt8 ("Jamba-1.5: Hybrid Transformer-Mamba Models at Scale", paper
 // summary, section "ExpertsInt8 Quantization (Section 3.1)", steps 3-4): the
 // INT8 weights cross HBM once and are turned back into BF16 on chip; the
-// activations stay BF16.  Here every weight byte goes HBM -> registers, is
-// converted exactly to bf16 (the scale is applied once per output channel
-// after the dot product, an exact refactoring of sum_k x_k (q_k s)), and feeds
-// an mma.sync m16n8k16 whose 8 columns are up to 8 tokens of the expert;
-// accumulation is fp32.
+// activations stay BF16.  Here the weight bytes go HBM -> shared memory by
+// bulk asynchronous copies (1 byte per weight), are converted exactly to bf16
+// in registers (the scale is applied once per output channel after the dot
+// product, an exact refactoring of sum_k x_k (q_k s)), and feed mma.sync
+// m16n8k16 tiles whose 8 columns are up to 8 tokens of the expert; fp32
+// accumulation.
 //
+// One CTA per SM, persistent: 1 producer warp + 16 consumer warps.
+//  - A work unit is (touched expert, 16 output channels, one pass of up to
+//    8*NCH tokens): a slab of R weight rows (gate/up: 16 gate + the matching
+//    16 up rows; down: 16 rows) over the whole contraction length K.  Units
+//    are dealt to the CTAs round-robin; they are small, so the CTAs finish
+//    together.
+//  - The producer streams each slab in stages of R rows x KC bytes (32 KB),
+//    one cp.async.bulk per row (lane r copies row r), into a ring of 4-5
+//    stages: about 130-160 KB of weights in flight per SM, independent of
+//    what the consumers are doing.
+//  - Consumer warp w takes k-blocks [w*KB_W, (w+1)*KB_W) of every stage (64 B
+//    each) and accumulates its partial dot products over the whole unit.  Rows
+//    sit at a pitch of KC + 64 bytes, which spreads the 16-byte fragment reads
+//    of a warp over all banks.
+//  - At the end of a unit the 16 partials go to shared memory (double
+//    buffered by unit parity), an mbarrier collects the 16 warps, and all 512
+//    consumer threads sum them in warp order (deterministic) and write:
+//      gate/up : h = silu(s_g * x.q_g) * (s_u * x.q_u) -> H (bf16, slot order)
+//      down    : y = gate * (s_d * h.q_d)               -> Y (fp32, one row per
+//                                                          token->expert assignment)
+//    launch_finalize then sums each token's rows of Y into the bf16 output.
 // Fragment trick: the dot product does not care in which order k is summed,
-// so the 16 k-columns of every MMA step are a permutation of the 64-wide
-// k-block chosen such that thread (g = lane/4, c = lane%4) needs exactly
-// bytes [16c, 16c+16) of weight rows g and g+8 for the block's four MMA
-// steps -- one 16-byte load per row -- and the matching 16 consecutive bf16
-// of its token.  Step s uses physical k = 16c + 4s + {0,1} for fragment
-// columns 2c, 2c+1 and 16c + 4s + {2,3} for columns 2c+8, 2c+9.
-//
-// Work decomposition (persistent, one 16-warp CTA per SM): a work unit is
-// (touched expert, 16 output channels, one pass of up to 8*NCH tokens).  The
-// CTA's 16 warps split the unit's K range into equal contiguous pieces, so a
-// unit is small (a 16-row weight slab) and the units divide evenly over the
-// CTAs; each warp keeps a ring of kDepth weight steps in registers that runs
-// ahead across unit boundaries, so HBM never waits for a reduction.  At the
-// end of a unit the 16 partial accumulators are summed through shared memory
-// in warp order (deterministic) and warp 0 writes the result:
-//   k_gemv_gateup : h = silu(s_g * x.q_g) * (s_u * x.q_u) -> H (bf16, slot order)
-//   k_gemv_down   : y = gate * (s_d * h.q_d)               -> Y (fp32, one row per
-//                                                             token->expert assignment)
-// and launch_finalize sums each token's rows of Y into the bf16 output.
+// so the 16 k-columns of an MMA step are a permutation of the 64-wide k-block
+// chosen such that thread (g = lane/4, c = lane%4) reads exactly bytes
+// [16c, 16c+16) of rows g and g+8 for the block's four MMA steps, and the
+// matching 16 consecutive bf16 of its token.  Step s uses physical
+// k = 16c + 4s + {0,1} for fragment columns 2c, 2c+1 and 16c + 4s + {2,3} for
+// columns 2c+8, 2c+9.
+// Every wait is bounded (a stuck wait raises the abort flag, sets the device
+// error word and lets all warps leave).
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace jmoe {
 namespace {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;
-constexpr int kDepth = 4;  // ring slots per warp: three 64-wide k steps in flight
-constexpr int kMaxE = 16;
+using namespace sm100;
 
-// Units of one launch, built by every CTA from the expert offsets.
+constexpr int kConsumers = 16;
+constexpr int kProducer = kConsumers;  // warp index of the producer
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kPad = 64;
+constexpr int kMaxE = 16;
+constexpr int kMaxStages = 5;
+
+enum { kGateUp = 0, kDown = 1 };
+
+template <int MODE, int NCH>
+struct Cfg {
+    static constexpr int R = MODE == kGateUp ? 32 : 16;       // slab rows
+    static constexpr int KC = MODE == kGateUp ? 1024 : 2048;  // stage bytes per row
+    static constexpr int KBW = KC / 64 / kConsumers;          // 64-B k-blocks per warp per stage
+    static constexpr int kPitch = KC + kPad;
+    static constexpr int kStage = R * kPitch;
+    static constexpr int kStages = NCH == 1 ? 5 : 4;
+    static constexpr int NMAT = MODE == kGateUp ? 2 : 1;  // weight matrices per slab
+    static constexpr int kAcc = NMAT * 4;                 // fp32 per token chunk per thread
+    static constexpr int kRedFloats = 2 * kConsumers * NCH * kAcc * 32;
+    static constexpr int kSmem = kStages * kStage + kRedFloats * 4;
+};
+
 struct Units {
     int start[kMaxE + 1];  // first unit of expert e
     int groups;            // 16-channel groups per expert
 };
-
-__device__ __forceinline__ void build_units(Units& u, const int32_t* offsets, int E, int groups,
-                                            int tokens_per_pass) {
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < E; ++e) {
-            const int cnt = offsets[e + 1] - offsets[e];
-            const int passes = cnt > 0 ? (cnt + tokens_per_pass - 1) / tokens_per_pass : 0;
-            u.start[e] = run;
-            run += passes * groups;
-        }
-        u.start[E] = run;
-        u.groups = groups;
-    }
-}
 
 struct Unit {
     int e, group, pass;
@@ -104,268 +120,202 @@ __device__ __forceinline__ void mma_block(float (&acc)[4], const uint4& q0, cons
     }
 }
 
-template <int NCH>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemv_gateup(const uint16_t* __restrict__ x, int top_k, int E, int64_t d, int64_t f,
-                  const int8_t* __restrict__ wgu, const float* __restrict__ sgu,
-                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
-                  uint16_t* __restrict__ H) {
+struct GemvParams {
+    int E, top_k;
+    int64_t d, f;
+    const int8_t* w;        // gate/up [E][2f][d] or down [E][d][f]
+    const float* scale;     // [E][2f] or [E][d]
+    const int32_t* offsets; // [E+1]
+    const int32_t* perm;    // [A]
+    const float* gates;     // [A]        (down)
+    const uint16_t* b_src;  // x [T][d] (gate/up) or H [A][f] (down)
+    uint16_t* H;            // out of gate/up: bf16 [A][f]
+    float* Y;               // out of down: fp32 [A][d]
+    unsigned* err;
+};
+
+template <int MODE, int NCH>
+__global__ void __launch_bounds__(kThreads, 1) k_gemv(const GemvParams p) {
+    using C = Cfg<MODE, NCH>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* red = reinterpret_cast<float*>(smem + C::kStages * C::kStage);
+    __shared__ uint64_t full[kMaxStages], empty[kMaxStages], red_full[2];
     __shared__ Units U;
     __shared__ int s_off[kMaxE + 1];
-    // partial sums of the 16 warps, double-buffered by unit parity (dynamic:
-    // 32 KB per token chunk)
-    extern __shared__ float red_raw[];
-    auto red = reinterpret_cast<float(*)[kWarps][32][NCH][8]>(red_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, c = lane & 3;
-    if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
-    build_units(U, offsets, E, (int)(f / 16), 8 * NCH);
+    __shared__ int s_abort;
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int E = p.E;
+    const int64_t K = MODE == kGateUp ? p.d : p.f;
+    const int64_t rows_out = MODE == kGateUp ? p.f : p.d;  // output channels per expert
+    const int nst = (int)((K + C::KC - 1) / C::KC);       // stages per unit
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumers);
+        }
+        mbar_init(&red_full[0], kConsumers);
+        mbar_init(&red_full[1], kConsumers);
+        s_abort = 0;
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            const int cnt = p.offsets[e + 1] - p.offsets[e];
+            U.start[e] = run;
+            run += cnt > 0 ? (cnt + 8 * NCH - 1) / (8 * NCH) * (int)(rows_out / 16) : 0;
+        }
+        U.start[E] = run;
+        U.groups = (int)(rows_out / 16);
+        fence_mbar_init();
+    }
+    if (threadIdx.x <= E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
     __syncthreads();
+    volatile int* abort = &s_abort;
     const int n_units = U.start[E];
     const int G = gridDim.x;
     const int n_mine = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
-    const int S = (int)(d / 64);
-    const int nw = (S + kWarps - 1) / kWarps;
-    const int s_lo = warp * nw;
-    const int s_hi = min(S, s_lo + nw);
-    const int64_t total = (int64_t)n_mine * nw;
 
-    // ---- prefetch cursor (unit iteration pi, step pj) and its slab pointers
-    int pi = 0, pj = 0;
-    const int8_t* pw[4] = {nullptr, nullptr, nullptr, nullptr};
-    auto set_prefetch_unit = [&](int it) {
-        const Unit u = decode_unit(U, E, blockIdx.x + it * G);
-        const int8_t* base = wgu + ((int64_t)u.e * 2 * f + u.group * 16 + g) * d + 16 * c +
-                             (int64_t)s_lo * 64;
-        pw[0] = base;
-        pw[1] = base + 8 * d;
-        pw[2] = base + f * d;
-        pw[3] = base + f * d + 8 * d;
-    };
-    uint4 ring[kDepth][4];
-    auto issue = [&](int slot) {
-        // load step (pi, pj) into ring[slot]; the padding steps of short K pieces load nothing
-        if (s_lo + pj < s_hi) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) ring[slot][m] = ldg_stream_v4(pw[m] + (int64_t)pj * 64);
-        }
-        if (++pj == nw) {
-            pj = 0;
-            if (++pi < n_mine) set_prefetch_unit(pi);
-        }
-    };
-    if (n_mine > 0) set_prefetch_unit(0);
-#pragma unroll
-    for (int p = 0; p < kDepth - 1; ++p)
-        if (p < total) issue(p);
-
-    // ---- consumer state
-    float ag[NCH][4], au[NCH][4];
-#pragma unroll
-    for (int n = 0; n < NCH; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) ag[n][i] = au[n][i] = 0.0f;
-    Unit cu{};
-    const uint16_t* xp[NCH];
-    int cnt_pass = 0;
-    int ci = 0, cj = 0;
-    auto set_consumer_unit = [&](int it) {
-        cu = decode_unit(U, E, blockIdx.x + it * G);
-        const int base = s_off[cu.e];
-        const int cnt = s_off[cu.e + 1] - base;
-        const int t0 = cu.pass * 8 * NCH;
-        cnt_pass = min(8 * NCH, cnt - t0);
-#pragma unroll
-        for (int n = 0; n < NCH; ++n) {
-            const int slot = n * 8 + g;
-            xp[n] = slot < cnt_pass
-                        ? x + (int64_t)(perm[base + t0 + slot] / top_k) * d + 16 * c + s_lo * 64
-                        : nullptr;
-        }
-    };
-    if (n_mine > 0) set_consumer_unit(0);
-
-    for (int64_t q0 = 0; q0 < total; q0 += kDepth) {
-#pragma unroll
-        for (int jj = 0; jj < kDepth; ++jj) {
-            const int64_t q = q0 + jj;
-            if (q < total) {
-                if (q + kDepth - 1 < total) issue((jj + kDepth - 1) % kDepth);
-                if (s_lo + cj < s_hi) {
-#pragma unroll
-                    for (int n = 0; n < NCH; ++n) {
-                        if (n * 8 < cnt_pass) {
-                            uint32_t b[8];
-                            load_b(xp[n] ? xp[n] + cj * 64 : nullptr, b);
-                            mma_block(ag[n], ring[jj][0], ring[jj][1], b);
-                            mma_block(au[n], ring[jj][2], ring[jj][3], b);
-                        }
-                    }
+    if (warp == kProducer) {
+        uint32_t g = 0;
+        bool ok = true;
+        for (int it = 0; it < n_mine && ok; ++it) {
+            const Unit u = decode_unit(U, E, blockIdx.x + it * G);
+            const int8_t* src = nullptr;
+            if (lane < C::R) {
+                int64_t row;
+                if (MODE == kGateUp)
+                    row = (int64_t)u.e * 2 * p.f + (lane < 16 ? 0 : p.f) + u.group * 16 + (lane & 15);
+                else
+                    row = (int64_t)u.e * p.d + u.group * 16 + lane;
+                src = p.w + row * K;
+            }
+            for (int st = 0; st < nst; ++st, ++g) {
+                const int s = g % C::kStages;
+                const uint32_t ph = (g / C::kStages) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort)) {
+                    ok = false;
+                    break;
                 }
-                if (++cj == nw) {
-                    // end of unit: reduce the 16 warps' partials, warp 0 writes h
-                    const int buf = ci & 1;
+                const int64_t k0 = (int64_t)st * C::KC;
+                const uint32_t bytes = (uint32_t)min((int64_t)C::KC, K - k0);
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], C::R * bytes);
+                __syncwarp();
+                if (lane < C::R) bulk_load(smem + s * C::kStage + lane * C::kPitch, src + k0, bytes,
+                                           &full[s]);
+            }
+        }
+        // do not leave while a copy may still be landing in shared memory
+        for (uint32_t h = (g > (uint32_t)C::kStages ? g - C::kStages : 0); h < g; ++h) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&full[h % C::kStages], (h / C::kStages) & 1))
+                if (clock64() - t0 > kWaitCycles) break;
+        }
+    } else {
+        const int g8 = lane >> 2, c = lane & 3;
+        float acc[NCH][C::NMAT][4];
 #pragma unroll
-                    for (int n = 0; n < NCH; ++n)
+        for (int n = 0; n < NCH; ++n)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            red[buf][warp][lane][n][i] = ag[n][i];
-                            red[buf][warp][lane][n][4 + i] = au[n][i];
-                            ag[n][i] = au[n][i] = 0.0f;
+            for (int m = 0; m < C::NMAT; ++m)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[n][m][i] = 0.0f;
+        uint32_t g = 0;
+        bool ok = true;
+        for (int it = 0; it < n_mine && ok; ++it) {
+            const Unit u = decode_unit(U, E, blockIdx.x + it * G);
+            const int base = s_off[u.e] + u.pass * 8 * NCH;
+            const int cnt_pass = min(8 * NCH, s_off[u.e + 1] - base);
+            const uint16_t* bp[NCH];
+#pragma unroll
+            for (int n = 0; n < NCH; ++n) {
+                const int slot = n * 8 + g8;
+                if (slot < cnt_pass) {
+                    const int64_t row =
+                        MODE == kGateUp ? (int64_t)(p.perm[base + slot] / p.top_k) : base + slot;
+                    bp[n] = p.b_src + row * K + 16 * c;
+                } else {
+                    bp[n] = nullptr;
+                }
+            }
+            for (int st = 0; st < nst; ++st, ++g) {
+                const int s = g % C::kStages;
+                const uint32_t ph = (g / C::kStages) & 1;
+                if (!mbar_wait(&full[s], ph, abort)) {
+                    ok = false;
+                    break;
+                }
+                const int64_t k0 = (int64_t)st * C::KC;
+                const int valid = (int)min((int64_t)C::KC, K - k0);
+                const uint8_t* stage = smem + s * C::kStage;
+#pragma unroll
+                for (int kb = 0; kb < C::KBW; ++kb) {
+                    const int kbyte = (warp * C::KBW + kb) * 64;
+                    if (kbyte < valid) {
+                        const uint8_t* r0 = stage + g8 * C::kPitch + kbyte + 16 * c;
+                        const uint4 q0 = *reinterpret_cast<const uint4*>(r0);
+                        const uint4 q1 = *reinterpret_cast<const uint4*>(r0 + 8 * C::kPitch);
+                        uint4 q2, q3;
+                        if (MODE == kGateUp) {
+                            q2 = *reinterpret_cast<const uint4*>(r0 + 16 * C::kPitch);
+                            q3 = *reinterpret_cast<const uint4*>(r0 + 24 * C::kPitch);
                         }
-                    __syncthreads();
-                    if (warp == 0) {
-                        const int base = s_off[cu.e] + cu.pass * 8 * NCH;
-                        const int64_t ch0 = (int64_t)cu.group * 16;
-                        const float* sg = sgu + (int64_t)cu.e * 2 * f + ch0;
 #pragma unroll
                         for (int n = 0; n < NCH; ++n) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                float vg = 0.f, vu = 0.f;
-                                for (int w2 = 0; w2 < kWarps; ++w2) {
-                                    vg += red[buf][w2][lane][n][i];
-                                    vu += red[buf][w2][lane][n][4 + i];
-                                }
-                                const int slot = n * 8 + 2 * c + (i & 1);
-                                const int row = g + (i >> 1) * 8;
-                                if (slot < cnt_pass) {
-                                    const float h = silu_f32(sg[row] * vg) * (sg[f + row] * vu);
-                                    H[(int64_t)(base + slot) * f + ch0 + row] =
-                                        __bfloat16_as_ushort(__float2bfloat16_rn(h));
-                                }
+                            if (n * 8 < cnt_pass) {
+                                uint32_t b[8];
+                                load_b(bp[n] ? bp[n] + k0 + kbyte : nullptr, b);
+                                mma_block(acc[n][0], q0, q1, b);
+                                if (MODE == kGateUp) mma_block(acc[n][C::NMAT - 1], q2, q3, b);
                             }
                         }
                     }
-                    cj = 0;
-                    if (++ci < n_mine) set_consumer_unit(ci);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
+            if (!ok) break;
+            // ---- end of unit: partials -> shared, then 512 threads finish
+            const int buf = it & 1;
+            float* rb = red + buf * (kConsumers * NCH * C::kAcc * 32);
+#pragma unroll
+            for (int n = 0; n < NCH; ++n)
+#pragma unroll
+                for (int m = 0; m < C::NMAT; ++m)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        rb[((warp * NCH + n) * C::kAcc + 4 * m + i) * 32 + lane] = acc[n][m][i];
+                        acc[n][m][i] = 0.0f;
+                    }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_full[buf]);
+            if (!mbar_wait(&red_full[buf], (it >> 1) & 1, abort)) break;
+            const int pos = threadIdx.x;  // 0..511: (n, i, lane') with lane' fastest
+            if (pos < NCH * 4 * 32) {
+                const int ln = pos & 31, i = (pos >> 5) & 3, n = pos >> 7;
+                float v0 = 0.f, v1 = 0.f;
+                for (int w2 = 0; w2 < kConsumers; ++w2) {
+                    v0 += rb[((w2 * NCH + n) * C::kAcc + i) * 32 + ln];
+                    if (MODE == kGateUp) v1 += rb[((w2 * NCH + n) * C::kAcc + 4 + i) * 32 + ln];
+                }
+                const int slot = n * 8 + 2 * (ln & 3) + (i & 1);
+                const int row = (ln >> 2) + (i >> 1) * 8;
+                const int64_t ch = (int64_t)u.group * 16 + row;
+                if (slot < cnt_pass) {
+                    if (MODE == kGateUp) {
+                        const float* sg = p.scale + (int64_t)u.e * 2 * p.f;
+                        const float h = silu_f32(sg[ch] * v0) * (sg[p.f + ch] * v1);
+                        p.H[(int64_t)(base + slot) * p.f + ch] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                    } else {
+                        const int a = p.perm[base + slot];
+                        p.Y[(int64_t)a * p.d + ch] =
+                            p.gates[a] * (p.scale[(int64_t)u.e * p.d + ch] * v0);
+                    }
                 }
             }
         }
     }
-}
-
-template <int NCH>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemv_down(const uint16_t* __restrict__ H, int E, int64_t d, int64_t f,
-                const int8_t* __restrict__ wd, const float* __restrict__ sd,
-                const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
-                const float* __restrict__ gates, float* __restrict__ Y) {
-    __shared__ Units U;
-    __shared__ int s_off[kMaxE + 1];
-    __shared__ float red[2][kWarps][32][NCH][4];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, c = lane & 3;
-    if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
-    build_units(U, offsets, E, (int)(d / 16), 8 * NCH);
-    __syncthreads();
-    const int n_units = U.start[E];
-    const int G = gridDim.x;
-    const int n_mine = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
-    const int S = (int)(f / 64);
-    const int nw = (S + kWarps - 1) / kWarps;
-    const int s_lo = warp * nw;
-    const int s_hi = min(S, s_lo + nw);
-    const int64_t total = (int64_t)n_mine * nw;
-
-    int pi = 0, pj = 0;
-    const int8_t* pw[2] = {nullptr, nullptr};
-    auto set_prefetch_unit = [&](int it) {
-        const Unit u = decode_unit(U, E, blockIdx.x + it * G);
-        const int8_t* base =
-            wd + ((int64_t)u.e * d + u.group * 16 + g) * f + 16 * c + (int64_t)s_lo * 64;
-        pw[0] = base;
-        pw[1] = base + 8 * f;
-    };
-    uint4 ring[kDepth][2];
-    auto issue = [&](int slot) {
-        if (s_lo + pj < s_hi) {
-            ring[slot][0] = ldg_stream_v4(pw[0] + (int64_t)pj * 64);
-            ring[slot][1] = ldg_stream_v4(pw[1] + (int64_t)pj * 64);
-        }
-        if (++pj == nw) {
-            pj = 0;
-            if (++pi < n_mine) set_prefetch_unit(pi);
-        }
-    };
-    if (n_mine > 0) set_prefetch_unit(0);
-#pragma unroll
-    for (int p = 0; p < kDepth - 1; ++p)
-        if (p < total) issue(p);
-
-    float acc[NCH][4];
-#pragma unroll
-    for (int n = 0; n < NCH; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
-    Unit cu{};
-    const uint16_t* hp[NCH];
-    int cnt_pass = 0;
-    int ci = 0, cj = 0;
-    auto set_consumer_unit = [&](int it) {
-        cu = decode_unit(U, E, blockIdx.x + it * G);
-        const int base = s_off[cu.e];
-        const int cnt = s_off[cu.e + 1] - base;
-        const int t0 = cu.pass * 8 * NCH;
-        cnt_pass = min(8 * NCH, cnt - t0);
-#pragma unroll
-        for (int n = 0; n < NCH; ++n) {
-            const int slot = n * 8 + g;
-            hp[n] = slot < cnt_pass ? H + (int64_t)(base + t0 + slot) * f + 16 * c + s_lo * 64
-                                    : nullptr;
-        }
-    };
-    if (n_mine > 0) set_consumer_unit(0);
-
-    for (int64_t q0 = 0; q0 < total; q0 += kDepth) {
-#pragma unroll
-        for (int jj = 0; jj < kDepth; ++jj) {
-            const int64_t q = q0 + jj;
-            if (q < total) {
-                if (q + kDepth - 1 < total) issue((jj + kDepth - 1) % kDepth);
-                if (s_lo + cj < s_hi) {
-#pragma unroll
-                    for (int n = 0; n < NCH; ++n) {
-                        if (n * 8 < cnt_pass) {
-                            uint32_t b[8];
-                            load_b(hp[n] ? hp[n] + cj * 64 : nullptr, b);
-                            mma_block(acc[n], ring[jj][0], ring[jj][1], b);
-                        }
-                    }
-                }
-                if (++cj == nw) {
-                    const int buf = ci & 1;
-#pragma unroll
-                    for (int n = 0; n < NCH; ++n)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            red[buf][warp][lane][n][i] = acc[n][i];
-                            acc[n][i] = 0.0f;
-                        }
-                    __syncthreads();
-                    if (warp == 0) {
-                        const int base = s_off[cu.e] + cu.pass * 8 * NCH;
-                        const int64_t m0 = (int64_t)cu.group * 16;
-                        const float* s = sd + (int64_t)cu.e * d + m0;
-#pragma unroll
-                        for (int n = 0; n < NCH; ++n) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                float v = 0.f;
-                                for (int w2 = 0; w2 < kWarps; ++w2) v += red[buf][w2][lane][n][i];
-                                const int slot = n * 8 + 2 * c + (i & 1);
-                                const int row = g + (i >> 1) * 8;
-                                if (slot < cnt_pass) {
-                                    const int a = perm[base + slot];
-                                    Y[(int64_t)a * d + m0 + row] = gates[a] * (s[row] * v);
-                                }
-                            }
-                        }
-                    }
-                    cj = 0;
-                    if (++ci < n_mine) set_consumer_unit(ci);
-                }
-            }
-        }
-    }
+    if (s_abort && threadIdx.x == kProducer * 32) flag_error(p.err, kErrTimeout);
 }
 
 // out[t] = bf16( sum_j Y[t*top_k + j] ) over the token's valid assignments.
@@ -395,25 +345,44 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+template <int MODE, int NCH>
+cudaError_t launch_gemv(const GemvParams& p, int grid, cudaStream_t stream) {
+    using C = Cfg<MODE, NCH>;
+    cudaError_t err = cudaFuncSetAttribute(k_gemv<MODE, NCH>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (err != cudaSuccess) return err;
+    k_gemv<MODE, NCH><<<grid, kThreads, C::kSmem, stream>>>(p);
+    return cudaGetLastError();
+}
+
 template <int NCH>
 cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
-    const int grid = a.num_sms;
-    const int red_bytes = (int)(2 * kWarps * 32 * NCH * 8 * sizeof(float));
-    cudaError_t err = cudaFuncSetAttribute(k_gemv_gateup<NCH>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, red_bytes);
-    if (err != cudaSuccess) return err;
+    GemvParams p{};
+    p.E = a.E;
+    p.top_k = a.top_k;
+    p.d = a.d;
+    p.f = a.f;
+    p.offsets = a.offsets;
+    p.perm = a.perm;
+    p.gates = a.gates;
+    p.err = a.err;
+    p.w = a.wgu;
+    p.scale = a.sgu;
+    p.b_src = static_cast<const uint16_t*>(a.x);
+    p.H = static_cast<uint16_t*>(a.H);
     if (a.mark) a.mark(2, false, stream);
-    k_gemv_gateup<NCH><<<grid, kThreads, red_bytes, stream>>>((const uint16_t*)a.x, a.top_k, a.E, a.d,
-                                                      a.f, a.wgu, a.sgu, a.offsets, a.perm,
-                                                      (uint16_t*)a.H);
+    cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
     if (a.mark) a.mark(2, true, stream);
-    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
+    p.w = a.wd;
+    p.scale = a.sd;
+    p.b_src = static_cast<const uint16_t*>(a.H);
+    p.H = nullptr;
+    p.Y = a.Y;
     if (a.mark) a.mark(3, false, stream);
-    k_gemv_down<NCH><<<grid, kThreads, 0, stream>>>((const uint16_t*)a.H, a.E, a.d, a.f, a.wd,
-                                                    a.sd, a.offsets, a.perm, a.gates, a.Y);
+    err = launch_gemv<kDown, NCH>(p, a.num_sms, stream);
     if (a.mark) a.mark(3, true, stream);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace

@@ -52,6 +52,7 @@ struct DecodeArgs {
     void* out;            // bf16 [T][d]
     int num_sms;
     StageMark mark;
+    unsigned* err;        // device error word
 };
 
 cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int E,

@@ -420,6 +420,8 @@ def main():
     ap.add_argument("--no-also", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--only", default=None, help="run only this workload (name) as headline")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the token count of --only (profiling runs on smaller cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -449,6 +451,10 @@ def main():
         from synth.workloads import BY_NAME
 
         wl = BY_NAME[args.only]
+        if args.tokens:
+            import dataclasses
+
+            wl = dataclasses.replace(wl, T=args.tokens, name=f"{wl.name}@T{args.tokens}")
     layer = Layer(wl, torch.device("cuda", local))
 
     sampler = ClockSampler(local)

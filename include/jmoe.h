@@ -171,10 +171,11 @@ jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int
  * and calls no allocating routine.
  *  - Size limit: if the scratch jmoe_forward_workspace_size would report for
  *    the decode kernels exceeds JMOE_NOALLOC_SCRATCH_BYTES, the call returns
- *    JMOE_EWORKSPACE before launching anything.  Roughly: the per-assignment
- *    output rows take T*top_k * d_model * 4 bytes and the hidden activations
- *    T*top_k * d_ff * 2 bytes (for example, 128 tokens at d_model 8192,
- *    d_ff 24576 and top-2 fit; 256 tokens at those sizes do not).
+ *    JMOE_EWORKSPACE before launching anything.  Roughly: the hidden
+ *    activations take T*top_k * d_ff * 2 bytes and the split-K partial sums
+ *    of the two projections up to 24 MB, or at least T*top_k * (2*d_ff +
+ *    d_model) * 4 bytes (for example, 32 tokens at d_model 8192, d_ff 24576
+ *    and top-2 fit; 64 tokens at those sizes do not).
  *  - The first call on a device looks up the array's device address for that
  *    device (with that device current) and caches it; make that first call
  *    before capturing any stream work on the device.

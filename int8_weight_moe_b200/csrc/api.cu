@@ -70,7 +70,8 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the size query and the forward calls.
 struct Workspace {
     size_t offsets, padded_offsets, perm, inv;  // routing tables
-    size_t H, Y;                                // decode path
+    size_t H, Pgu, Pd;                          // decode path
+    int split_gu, split_d;
     size_t xperm, Hp, Yg;                       // tensor-core path
     size_t total;
     int64_t rows_padded;  // upper bound of the padded expert-grouped rows
@@ -90,8 +91,20 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     w.inv = take(sizeof(int32_t) * (size_t)A);
     (void)T;
     if (!prefill) {
+        // K pieces: about 16 work items per warp on a 148-SM GPU, with the
+        // partial-sum buffers capped at 16 MB (gate/up) and 8 MB (down).
+        const int64_t target = 148LL * 16 * 16;
+        const int64_t touched = A < E ? A : E;
+        const int64_t units_gu = touched * (f / 16), units_d = touched * (d / 16);
+        const int64_t row_gu = A * 2 * f * (int64_t)sizeof(float);
+        const int64_t row_d = A * d * (int64_t)sizeof(float);
+        w.split_gu = jmoe::decode_split(d, units_gu > 0 ? (target + units_gu - 1) / units_gu : 1,
+                                        row_gu > 0 ? (16LL << 20) / row_gu : 1);
+        w.split_d = jmoe::decode_split(f, units_d > 0 ? (target + units_d - 1) / units_d : 1,
+                                       row_d > 0 ? (8LL << 20) / row_d : 1);
         w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
-        w.Y = take(sizeof(float) * (size_t)A * (size_t)d);
+        w.Pgu = take((size_t)w.split_gu * (size_t)row_gu);
+        w.Pd = take((size_t)w.split_d * (size_t)row_d);
     } else {
         const int64_t tm = jmoe::kPrefillTileM;
         w.rows_padded = (A + (int64_t)E * (tm - 1) + tm - 1) / tm * tm;
@@ -152,8 +165,10 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         jmoe::DecodeArgs a{};
         a.x = x; a.T = T; a.A = A; a.d = d; a.f = f; a.E = E; a.top_k = k;
         a.wgu = desc->w_gu; a.sgu = desc->s_gu; a.wd = desc->w_d; a.sd = desc->s_d;
-        a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm;
-        a.H = at(w.H); a.Y = static_cast<float*>(at(w.Y));
+        a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm; a.inv = inv;
+        a.H = at(w.H); a.P_gu = static_cast<float*>(at(w.Pgu));
+        a.P_d = static_cast<float*>(at(w.Pd));
+        a.split_gu = w.split_gu; a.split_d = w.split_d;
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;

@@ -46,8 +46,11 @@ struct DecodeArgs {
     const float* gates;   // [T][top_k]
     const int32_t* offsets;  // [E+1]
     const int32_t* perm;     // [A]
+    const int32_t* inv;      // [A]
     void* H;              // bf16 [A][f], expert-grouped slot order (workspace)
-    float* Y;             // fp32 [A][d], one row per assignment (workspace)
+    float* P_gu;          // fp32 [split_gu][A][2f] partial sums (workspace)
+    float* P_d;           // fp32 [split_d][A][d] partial sums (workspace)
+    int split_gu, split_d;   // K pieces of the two GEMVs
     int64_t max_per_expert;  // host-side bound used to size register tiles
     void* out;            // bf16 [T][d]
     int num_sms;
@@ -55,6 +58,9 @@ struct DecodeArgs {
     unsigned* err;        // device error word
 };
 
+// K pieces for a decode GEMV: the smallest divisor s of K/64 with s >= want
+// (and K/s >= 512 B, s <= cap); if there is none, the largest allowed one.
+int decode_split(int64_t K, int64_t want, int64_t cap);
 cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int E,
                             const int32_t* ids, void* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream);

@@ -13,22 +13,26 @@
 // accumulation is fp32 in TMEM.
 //
 // One CTA per SM, 15 warps:
-//   warp 0      TMA producer of the activation tile A [128 rows x 64 k] bf16
+//   warp 0      TMA producer of the activation tile A [256 rows x 64 k] bf16
+//               (two 128-row boxes; the second is skipped when the expert ends)
 //   warp 1      TMEM allocator and MMA issuer (one thread)
-//   warp 2      TMA producer of the INT8 weight tile [256 rows x 64 k]
+//   warp 2      TMA producer of the INT8 weight tile [128 rows x 64 k]
 //   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled)
 //   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
-// Rings: A + converted B share 3 stages (48 KB each), the INT8 tiles have 4
-// stages (16 KB each); two 128 x 256 fp32 accumulators (512 TMEM columns)
-// let the epilogue of one tile overlap the main loop of the next.
+// Rings: A + converted B share 3 stages (48 KB each); the INT8 tiles, which
+// come from HBM, have 8 stages (8 KB each) to cover its latency.  Each weight tile, once converted, feeds two M = 128
+// MMAs (256 token rows), which halves the conversion work per multiply-add
+// compared with one 128-row MMA.  Two accumulators of 2 x 128 x 128 fp32
+// (512 TMEM columns) let the epilogue of one tile overlap the main loop of
+// the next.
 //
-// Tiles: 128 expert-grouped rows (each expert's rows are padded to a
-// multiple of 128, so a tile never mixes experts) x 256 MMA columns.  Gate/up
-// mode: the 256 columns are 128 gate channels and the same 128 up channels,
-// so the SwiGLU pairs sit in one thread.  Down mode: 256 output channels; the
-// epilogue multiplies by the routing gate and writes one fp32 row per
-// token->expert assignment.  Tiles are visited expert by expert, m fastest,
-// so the CTAs of a wave share weight tiles and activation rows in L2.
+// Tiles: 256 expert-grouped rows (each expert's rows are padded to a
+// multiple of 128, so a tile never mixes experts; its second half may be
+// absent) x 128 MMA columns.  Gate/up mode: the 128 columns are 64 gate
+// channels and the same 64 up channels, so the SwiGLU pairs sit in one
+// thread.  Down mode: 128 output channels; the epilogue multiplies by the
+// routing gate and writes one fp32 row per token->expert assignment.  Tiles
+// are visited expert by expert in groups of 16 m-tiles (see decode_tile).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -41,16 +45,20 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int kStagesAB = 3, kStages8 = 4;
-constexpr int kABytes = BM * BK * 2;    // 16 KB
-constexpr int kBbfBytes = BN * BK * 2;  // 32 KB
-constexpr int kB8Bytes = BN * BK;       // 16 KB
+constexpr int BH = 128;       // rows of one MMA (a "half" of the tile)
+constexpr int BM = 2 * BH;    // token rows per tile: two MMAs share one weight tile
+constexpr int BN = 128, BK = 64;
+constexpr int kStagesAB = 3, kStages8 = 8;
+constexpr int kGroupM = 16;  // m-tiles per raster group (activation rows kept in L2)
+constexpr int kHalfBytes = BH * BK * 2;  // 16 KB
+constexpr int kABytes = 2 * kHalfBytes;  // 32 KB
+constexpr int kBbfBytes = BN * BK * 2;   // 16 KB
+constexpr int kB8Bytes = BN * BK;        // 8 KB
 constexpr int kABStage = kABytes + kBbfBytes;
 constexpr int kSmemAB = kStagesAB * kABStage;
 constexpr int kSmem8 = kStages8 * kB8Bytes;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
+constexpr uint32_t kTmemCols = 512;   // 2 buffers x 2 halves x 128 fp32 columns
+constexpr uint32_t kIdesc = idesc_bf16_f32(BH, BN);
 
 constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
 constexpr int kConvWarp0 = 3, kConvWarps = 8;
@@ -92,18 +100,27 @@ struct Shared {
 constexpr int kSmemBytes = kSmemAB + kSmem8 + (int)sizeof(Shared) + 1024;
 
 struct Tile {
-    int e, row0, n;
+    int e, row0, n, halves;  // halves: 1 or 2 valid 128-row halves
 };
 
-__device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int tile) {
+// Tile order inside an expert: groups of kGroupM m-tiles; within a group all
+// n-tiles, m fastest.  The CTAs of a wave then share a few weight tiles and
+// at most kGroupM x 256 activation rows, which stay in L2.
+__device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int n_tiles, int tile) {
     int e = 0;
     while (e + 1 < E && s.tile_start[e + 1] <= tile) ++e;
     const int local = tile - s.tile_start[e];
-    const int mt = (s.poff[e + 1] - s.poff[e]) / BM;
+    const int nh = (s.poff[e + 1] - s.poff[e]) / BH;  // 128-row halves of this expert
+    const int mt = (nh + 1) / 2;
+    const int mg = local / (kGroupM * n_tiles);
+    const int gm = min(kGroupM, mt - mg * kGroupM);  // m-tiles in this group
+    const int rem = local - mg * kGroupM * n_tiles;
     Tile t;
     t.e = e;
-    t.n = local / mt;
-    t.row0 = s.poff[e] + (local % mt) * BM;
+    t.n = rem / gm;
+    const int m = mg * kGroupM + rem % gm;
+    t.row0 = s.poff[e] + m * BM;
+    t.halves = min(2, nh - 2 * m);
     return t;
 }
 
@@ -161,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int run = 0;
         for (int e = 0; e < E; ++e) {
             S.tile_start[e] = run;
-            run += (S.poff[e + 1] - S.poff[e]) / BM * p.n_tiles;
+            run += ((S.poff[e + 1] - S.poff[e]) / BH + 1) / 2 * p.n_tiles;
         }
         S.tile_start[E] = run;
     }
@@ -180,13 +197,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t g = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
-                const Tile t = decode_tile(S, E, tile);
+                const Tile t = decode_tile(S, E, p.n_tiles, tile);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStagesAB;
                     const uint32_t ph = (g / kStagesAB) & 1;
                     if (!mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) break;
-                    mbar_arrive_expect_tx(&S.ab_full_a[s], kABytes);
+                    mbar_arrive_expect_tx(&S.ab_full_a[s], t.halves * kHalfBytes);
                     tma_load_2d(tileA(s), &tmA, &S.ab_full_a[s], kb * BK, t.row0);
+                    if (t.halves == 2)
+                        tma_load_2d(tileA(s) + kHalfBytes, &tmA, &S.ab_full_a[s], kb * BK,
+                                    t.row0 + BH);
                 }
             }
             // make sure no copy is still landing in shared memory when the CTA exits
@@ -197,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t g = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
-                const Tile t = decode_tile(S, E, tile);
+                const Tile t = decode_tile(S, E, p.n_tiles, tile);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages8;
                     const uint32_t ph = (g / kStages8) & 1;
@@ -222,10 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t g = 0;
             int it = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+                const int t_halves = decode_tile(S, E, p.n_tiles, tile).halves;
                 const int buf = it & 1;
                 if (!mbar_wait(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * BN;
+                const uint32_t d_tmem = tmem + buf * 2 * BN;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStagesAB;
@@ -237,10 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(tileA(s)), b0 = smem_u32(tileBbf(s));
+                    for (int h = 0; h < t_halves; ++h) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_bf16_ss(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
-                                    kIdesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_bf16_ss(d_tmem + h * BN, desc_sw128(a0 + h * kHalfBytes + kk * 32),
+                                        desc_sw128(b0 + kk * 32), kIdesc, (kb | kk) != 0);
+                    }
                     mma_commit(&S.ab_empty[s]);
                 }
                 if (!ok) break;
@@ -268,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* src = tileB8(s8);
                 uint8_t* dst = tileBbf(s);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < BN / 32; ++j) {
                     const int row = (ct >> 3) + 32 * j;
                     const uint2 v = *reinterpret_cast<const uint2*>(src + row * BK + chunk * 8);
                     uint4 o;
@@ -288,70 +311,79 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // epilogue warps: TMEM lane quadrant = warp % 4
+        // epilogue warps: TMEM lane quadrant = warp % 4, both halves of the tile
         const int quad = warp & 3;
-        const int rloc = quad * 32 + lane;
         int it = 0;
         for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
-            const Tile t = decode_tile(S, E, tile);
+            const Tile t = decode_tile(S, E, p.n_tiles, tile);
             const int buf = it & 1;
             if (!mbar_wait(&S.acc_full[buf], (it >> 1) & 1, abort)) break;
             tc_fence_after();
             __syncwarp();
-            const uint32_t taddr = tmem + buf * BN + ((uint32_t)(quad * 32) << 16);
-            const int row = t.row0 + rloc;
-            if (MODE == kGateUp) {
-                const int n0 = t.n * (BN / 2);
-                const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
-                const float* su = sg + p.up_offset;
+            for (int h = 0; h < t.halves; ++h) {
+                const uint32_t taddr =
+                    tmem + buf * 2 * BN + h * BN + ((uint32_t)(quad * 32) << 16);
+                const int row = t.row0 + h * BH + quad * 32 + lane;
+                if (MODE == kGateUp) {
+                    const int n0 = t.n * (BN / 2);
+                    const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
+                    const float* su = sg + p.up_offset;
 #pragma unroll 1
-                for (int c = 0; c < BN / 2 / 32; ++c) {
-                    uint32_t gv[32], uv[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, gv);
-                    tmem_ld_32x32b_x32(taddr + BN / 2 + c * 32, uv);
-                    tmem_ld_wait();
-                    const int ch = n0 + c * 32;
-                    if (ch < p.n_valid) {
-                        uint32_t packed[16];
+                    for (int c = 0; c < BN / 2 / 32; ++c) {
+                        uint32_t gv[32], uv[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, gv);
+                        tmem_ld_32x32b_x32(taddr + BN / 2 + c * 32, uv);
+                        tmem_ld_wait();
+                        const int ch = n0 + c * 32;
+                        if (ch < p.n_valid) {
+                            uint32_t packed[16];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const float g0 = __ldg(sg + c * 32 + j) * __uint_as_float(gv[j]);
-                            const float g1 = __ldg(sg + c * 32 + j + 1) * __uint_as_float(gv[j + 1]);
-                            const float u0 = __ldg(su + c * 32 + j) * __uint_as_float(uv[j]);
-                            const float u1 = __ldg(su + c * 32 + j + 1) * __uint_as_float(uv[j + 1]);
-                            packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                            for (int j = 0; j < 32; j += 4) {
+                                const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
+                                const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
+                                const float g0 = g4.x * __uint_as_float(gv[j]);
+                                const float g1 = g4.y * __uint_as_float(gv[j + 1]);
+                                const float g2 = g4.z * __uint_as_float(gv[j + 2]);
+                                const float g3 = g4.w * __uint_as_float(gv[j + 3]);
+                                const float u0 = u4.x * __uint_as_float(uv[j]);
+                                const float u1 = u4.y * __uint_as_float(uv[j + 1]);
+                                const float u2 = u4.z * __uint_as_float(uv[j + 2]);
+                                const float u3 = u4.w * __uint_as_float(uv[j + 3]);
+                                packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                                packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
+                            }
+                            uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1],
+                                                    packed[4 * q + 2], packed[4 * q + 3]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                                packed[4 * q + 3]);
                     }
-                }
-            } else {
-                const int m0 = t.n * BN;
-                const int r = row - S.poff[t.e];
-                const bool valid = r < S.off[t.e + 1] - S.off[t.e];
-                const int a = valid ? p.perm[S.off[t.e] + r] : 0;
-                const float gate = valid ? p.gates[a] : 0.0f;
-                const float* sd = p.scale + (size_t)t.e * p.w_rows;
+                } else {
+                    const int m0 = t.n * BN;
+                    const int r = row - S.poff[t.e];
+                    const bool valid = r < S.off[t.e + 1] - S.off[t.e];
+                    const int a = valid ? p.perm[S.off[t.e] + r] : 0;
+                    const float gate = valid ? p.gates[a] : 0.0f;
+                    const float* sd = p.scale + (size_t)t.e * p.w_rows;
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(taddr + c * 32, v);
-                    tmem_ld_wait();
-                    const int m = m0 + c * 32;
-                    if (valid && m < p.n_valid) {
-                        float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(taddr + c * 32, v);
+                        tmem_ld_wait();
+                        const int m = m0 + c * 32;
+                        if (valid && m < p.n_valid) {
+                            float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + q);
-                            float4 o;
-                            o.x = gate * (s4.x * __uint_as_float(v[4 * q]));
-                            o.y = gate * (s4.y * __uint_as_float(v[4 * q + 1]));
-                            o.z = gate * (s4.z * __uint_as_float(v[4 * q + 2]));
-                            o.w = gate * (s4.w * __uint_as_float(v[4 * q + 3]));
-                            dst[q] = o;
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + q);
+                                float4 o;
+                                o.x = gate * (s4.x * __uint_as_float(v[4 * q]));
+                                o.y = gate * (s4.y * __uint_as_float(v[4 * q + 1]));
+                                o.z = gate * (s4.z * __uint_as_float(v[4 * q + 2]));
+                                o.w = gate * (s4.w * __uint_as_float(v[4 * q + 3]));
+                                dst[q] = o;
+                            }
                         }
                     }
                 }
@@ -435,11 +467,11 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
 
     CUtensorMap mA1, mB1, mA2, mB2;
     const bool ok =
-        make_map(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BM, BK,
+        make_map(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
         make_map(&mB1, a.wgu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * 2 * a.f, a.d,
                  BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        make_map(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BM, BK,
+        make_map(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
         make_map(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BN, BK,
                  CU_TENSOR_MAP_SWIZZLE_NONE);

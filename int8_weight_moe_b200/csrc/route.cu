@@ -14,11 +14,12 @@
 // is added in fp64 and the result rounded once to fp32.  The products are
 // exact in fp64 (8-bit x 24-bit significands).
 //
-// Work split: a CTA of 4 warps handles kTok tokens; warp w owns experts
-// w, w+4, w+8, w+12, so each lane keeps 4 x kTok independent fp64
-// accumulators and every router weight it loads serves kTok tokens.  The
-// k loop is unrolled so the loads of several steps are in flight together.
-// Softmax (fp32) and top-k run in the first threads of the CTA afterwards.
+// Work split: for many tokens a CTA of 4 warps handles kTok tokens; warp w
+// owns experts w, w+4, w+8, w+12, so each lane keeps 4 x kTok independent
+// fp64 accumulators and every router weight it loads serves kTok tokens.
+// For few tokens (decode) a 16-warp CTA takes one token, one expert per warp.
+// The k loops are unrolled so the loads of several steps are in flight
+// together.  Softmax (fp32) and top-k run in one thread per token afterwards.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,6 +29,63 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kMaxE = 16;
 constexpr int kPerWarp = kMaxE / kWarps;
+
+// Top-k on one token's fp32 logits (strict '>' keeps the lower index on
+// ties), fp32 softmax over all E experts, renormalised over the selection.
+__device__ void select_topk(const float* l, int64_t t, int E, int top_k, int32_t* ids,
+                            float* gates, float* logits) {
+    if (logits)
+        for (int e = 0; e < E; ++e) logits[t * E + e] = l[e];
+    int e1 = 0;
+    for (int e = 1; e < E; ++e)
+        if (l[e] > l[e1]) e1 = e;
+    int e2 = -1;
+    if (top_k == 2)
+        for (int e = 0; e < E; ++e)
+            if (e != e1 && (e2 < 0 || l[e] > l[e2])) e2 = e;
+    float p[kMaxE];
+    const float m = l[e1];
+    float z = 0.0f;
+    for (int e = 0; e < E; ++e) {
+        p[e] = expf(l[e] - m);
+        z += p[e];
+    }
+    for (int e = 0; e < E; ++e) p[e] = p[e] / z;
+    if (top_k == 1) {
+        ids[t] = e1;
+        gates[t] = 1.0f;
+    } else {
+        const float sel = p[e1] + p[e2];
+        ids[2 * t] = e1;
+        ids[2 * t + 1] = e2;
+        gates[2 * t] = p[e1] / sel;
+        gates[2 * t + 1] = p[e2] / sel;
+    }
+}
+
+// Few tokens: one CTA of 16 warps per token, warp e computes expert e's
+// logit (same per-lane order and halving tree), loads deeply unrolled.
+__global__ void __launch_bounds__(kMaxE * 32)
+    k_route_wide(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
+                 const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
+                 float* __restrict__ gates, float* __restrict__ logits) {
+    __shared__ float s_logit[kMaxE];
+    const int lane = threadIdx.x & 31, e = threadIdx.x >> 5;
+    const int64_t t = blockIdx.x;
+    if (e < E) {
+        const uint16_t* xr = x + t * d;
+        const float* w = wr + (int64_t)e * d;
+        double acc = 0.0;
+#pragma unroll 8
+        for (int64_t k = lane; k < d; k += 32)
+            acc = fma((double)bf16_bits_to_f32(__ldg(xr + k)), (double)__ldg(w + k), acc);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o);
+        if (lane == 0) s_logit[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) select_topk(s_logit, t, E, top_k, ids, gates, logits);
+}
 
 template <int kTok>
 __global__ void __launch_bounds__(kWarps * 32)
@@ -79,39 +137,8 @@ __global__ void __launch_bounds__(kWarps * 32)
             }
         }
         __syncthreads();
-        if (threadIdx.x < kTok && t0 + threadIdx.x < T) {
-            const int64_t t = t0 + threadIdx.x;
-            const float* l = s_logit[threadIdx.x];
-            if (logits)
-                for (int e = 0; e < E; ++e) logits[t * E + e] = l[e];
-            // top-k on the fp32 logits: strict '>' keeps the lower index on ties
-            int e1 = 0;
-            for (int e = 1; e < E; ++e)
-                if (l[e] > l[e1]) e1 = e;
-            int e2 = -1;
-            if (top_k == 2)
-                for (int e = 0; e < E; ++e)
-                    if (e != e1 && (e2 < 0 || l[e] > l[e2])) e2 = e;
-            // fp32 softmax over all E experts, renormalised over the selection
-            float p[kMaxE];
-            const float m = l[e1];
-            float z = 0.0f;
-            for (int e = 0; e < E; ++e) {
-                p[e] = expf(l[e] - m);
-                z += p[e];
-            }
-            for (int e = 0; e < E; ++e) p[e] = p[e] / z;
-            if (top_k == 1) {
-                ids[t] = e1;
-                gates[t] = 1.0f;
-            } else {
-                const float sel = p[e1] + p[e2];
-                ids[2 * t] = e1;
-                ids[2 * t + 1] = e2;
-                gates[2 * t] = p[e1] / sel;
-                gates[2 * t + 1] = p[e2] / sel;
-            }
-        }
+        if (threadIdx.x < kTok && t0 + threadIdx.x < T)
+            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, ids, gates, logits);
         __syncthreads();
     }
 }
@@ -122,12 +149,11 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
                          const float* bias, int E, int top_k, int32_t* ids, float* gates,
                          float* logits, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    // Few tokens: one token per CTA spreads them over more SMs (latency);
-    // many tokens: 4 per CTA cuts the router-weight traffic fourfold.
+    // Few tokens: a 16-warp CTA per token (latency); many tokens: 4 tokens per
+    // 4-warp CTA, which cuts the router-weight traffic fourfold.
     if (T < (int64_t)num_sms * 8) {
-        int64_t blocks = T;
-        k_route<1><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-            (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, ids, gates, logits);
+        k_route_wide<<<(unsigned)T, kMaxE * 32, 0, stream>>>((const uint16_t*)x_bf16, d, w_router,
+                                                             bias, E, top_k, ids, gates, logits);
     } else {
         int64_t blocks = (T + 3) / 4;
         const int64_t cap = (int64_t)num_sms * 16;

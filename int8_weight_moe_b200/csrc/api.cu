@@ -70,7 +70,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the size query and the forward calls.
 struct Workspace {
     size_t offsets, padded_offsets, perm, inv;  // routing tables
-    size_t H, Pgu, Pd;                          // decode path
+    size_t H, Pgu, Pd, x16, xexp;               // decode path
     int split_gu, split_d;
     size_t xperm, Hp, Yg;                       // tensor-core path
     size_t total;
@@ -89,7 +89,6 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     w.padded_offsets = take(sizeof(int32_t) * (size_t)(E + 1));
     w.perm = take(sizeof(int32_t) * (size_t)A);
     w.inv = take(sizeof(int32_t) * (size_t)A);
-    (void)T;
     if (!prefill) {
         // K pieces: about 16 work items per warp on a 148-SM GPU, with the
         // partial-sum buffers capped at 16 MB (gate/up) and 8 MB (down).
@@ -103,6 +102,8 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
         w.split_d = jmoe::decode_split(f, units_d > 0 ? (target + units_d - 1) / units_d : 1,
                                        row_d > 0 ? (8LL << 20) / row_d : 1);
         w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
+        w.x16 = take(sizeof(uint16_t) * (size_t)T * (size_t)d);
+        w.xexp = take(sizeof(int32_t) * (size_t)T);
         w.Pgu = take((size_t)w.split_gu * (size_t)row_gu);
         w.Pd = take((size_t)w.split_d * (size_t)row_d);
     } else {
@@ -169,6 +170,7 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         a.H = at(w.H); a.P_gu = static_cast<float*>(at(w.Pgu));
         a.P_d = static_cast<float*>(at(w.Pd));
         a.split_gu = w.split_gu; a.split_d = w.split_d;
+        a.x16 = at(w.x16); a.xexp = static_cast<int32_t*>(at(w.xexp));
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -34,6 +35,33 @@ __device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w) {
     __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v),
                                *reinterpret_cast<const __nv_bfloat162*>(&c));
     return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Four int8 values (one 32-bit word) to two packed f16x2 words, exactly.
+//
+// u = b + 128 (flip the sign bit) is an unsigned byte; the f16 pattern
+// 0x6400 | u is 1024 + u (exponent 2^10, ten mantissa bits hold 0..1023), and
+// subtracting 1152 = 1024 + 128 (0x6480) gives b exactly.  One logic op per
+// word, then one byte permute and one f16x2 subtract per pair.
+__device__ __forceinline__ void i8x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t tlo = __byte_perm(u, 0x64646464u, 0x4140u);  // [u0, 0x64, u1, 0x64]
+    const uint32_t thi = __byte_perm(u, 0x64646464u, 0x4342u);  // [u2, 0x64, u3, 0x64]
+    const uint32_t k = 0x64806480u;
+    __half2 rl = __hsub2(*reinterpret_cast<const __half2*>(&tlo), *reinterpret_cast<const __half2*>(&k));
+    __half2 rh = __hsub2(*reinterpret_cast<const __half2*>(&thi), *reinterpret_cast<const __half2*>(&k));
+    lo = *reinterpret_cast<uint32_t*>(&rl);
+    hi = *reinterpret_cast<uint32_t*>(&rh);
+}
+
+// D = A * B + D for one m16n8k16 tile, f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                              uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // 16 bytes of int8 -> 8 packed bf16x2 words (element order preserved).

@@ -4,13 +4,20 @@
 //
 // ExpertsInt8 ("Jamba-1.5: Hybrid Transformer-Mamba Models at Scale", paper
 // summary, section "ExpertsInt8 Quantization (Section 3.1)", steps 3-4): the
-// INT8 weights cross HBM once and are turned back into BF16 on chip; the
-// activations stay BF16.  Here every weight byte goes HBM -> registers, is
-// converted exactly to bf16 (the scale is applied once per output channel
-// after the dot product, an exact refactoring of sum_k x_k (q_k s)), and feeds
-// an mma.sync m16n8k16 whose 8 columns are up to 8 tokens of the expert; fp32
-// accumulation.
-//
+// INT8 weights cross HBM once and are turned back into 16-bit floating point
+// on chip; the activations keep their BF16 values.  Every weight byte goes
+// HBM -> shared -> registers and is converted exactly (|q| <= 127).  In the
+// gate/up projection (two thirds of the bytes) the weights become fp16 values
+// -- the same numbers BF16 would hold, but the int8 -> fp16 conversion costs
+// half the ALU work -- and the token rows are staged as fp16 after a
+// power-of-two shift per token that brings the row maximum into [2^14, 2^15):
+// a bf16 value has 8 significant bits, so the staged values are exact and
+// every product equals the bf16 one; the shift is undone exactly after the dot
+// product.  The down projection uses bf16 weights against the bf16 hidden
+// activations.  The per-output-channel scale is applied once after the dot
+// product (an exact refactoring of sum_k x_k (q_k s)).  mma.sync m16n8k16
+// (16-bit in, fp32 accumulate), up to 8 tokens of the expert as the columns.
+
 // Fragment trick: the dot product does not care in which order k is summed,
 // so the 16 k-columns of an MMA step are a permutation of the 64-wide k-block
 // chosen such that thread (g = lane/4, c = lane%4) reads exactly bytes
@@ -30,16 +37,19 @@
 // in registers), so there are no bubbles and no barriers at all.  An item
 // stores its raw fp32 partial sums; the small follow-up kernels add the S
 // pieces in a fixed order (deterministic) and apply scales, SwiGLU, gates:
+//   k_prep_x16 -> x16 (fp16, per-token shift)
 //   k_gemv<gate/up> -> P_gu[S][slot][2f] -> k_swiglu -> H (bf16, slot order)
 //   k_gemv<down>    -> P_d [S][slot][d]  -> k_combine -> out (bf16)
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace jmoe {
 namespace {
 
 constexpr int kWarpsPerBlock = 4;
-constexpr int kDepth = 4;  // ring slots per warp: three 64-byte steps in flight
 constexpr int kMaxE = 16;
 
 enum { kGateUp = 0, kDown = 1 };
@@ -53,6 +63,7 @@ struct GemvParams {
     const uint16_t* b_src;     // x [T][d] (gate/up) or H [A][f] (down)
     float* P;                  // partial sums [S][A][cols]
     int64_t A;
+    unsigned* err;
 };
 
 // x (or h) fragment for one token row: 16 consecutive bf16 starting at p.
@@ -70,15 +81,26 @@ __device__ __forceinline__ void load_b(const uint16_t* p, uint32_t (&b)[8]) {
 
 // Four MMA steps of one 64-wide k-block: rows g (q0) and g+8 (q1).  Even and
 // odd steps accumulate into separate tiles (two independent MMA chains).
+// F16: weights converted to fp16 and fp16 MMA (activation operand in fp16);
+// otherwise bf16 conversion and bf16 MMA.
+template <bool F16>
 __device__ __forceinline__ void mma_block(float (&acc)[2][4], const uint4& q0, const uint4& q1,
                                           const uint32_t (&b)[8]) {
     const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w};
     const uint32_t w1[4] = {q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        const uint32_t a[4] = {i8x2_to_bf16x2<0>(w0[s]), i8x2_to_bf16x2<0>(w1[s]),
-                               i8x2_to_bf16x2<1>(w0[s]), i8x2_to_bf16x2<1>(w1[s])};
-        mma_bf16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
+        if (F16) {
+            uint32_t l0, h0, l1, h1;
+            i8x4_to_f16x2x2(w0[s], l0, h0);
+            i8x4_to_f16x2x2(w1[s], l1, h1);
+            const uint32_t a[4] = {l0, l1, h0, h1};
+            mma_f16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
+        } else {
+            const uint32_t a[4] = {i8x2_to_bf16x2<0>(w0[s]), i8x2_to_bf16x2<0>(w1[s]),
+                                   i8x2_to_bf16x2<1>(w0[s]), i8x2_to_bf16x2<1>(w1[s])};
+            mma_bf16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
+        }
     }
 }
 
@@ -86,34 +108,50 @@ struct Item {
     int e, group, pass, z;
 };
 
-// Shared-memory bytes of one ring slot: per lane, 2*NMAT weight and NCH*2
-// activation 16-byte pieces.
-template <int MODE, int NCH>
-constexpr int slot_bytes() {
-    return (2 * (MODE == kGateUp ? 2 : 1) + 2 * NCH) * 32 * 16;
+// The last `slots` slot fills of a warp (the ones whose copies may still be
+// in flight when the warp leaves).
+__device__ __forceinline__ int64_t q_drain_begin(int64_t total, int slots) {
+    return total > slots ? total - slots : 0;
 }
 
-template <int MODE, int NCH>
+constexpr int kNB = 2;     // 64-byte k-blocks per ring slot
+constexpr int kSlots = 3;  // ring slots per warp: two slots (4 KB of gate/up weights) in flight
+
+// Shared memory of one warp: kSlots x [matrix][k-block][16 rows][64 B]; the
+// dense 64-byte row pitch makes the fragment reads of a warp conflict-free.
+template <int MODE>
+constexpr int slot_bytes() {
+    return (MODE == kGateUp ? 2 : 1) * kNB * 16 * 64;
+}
+
+template <int MODE>
 constexpr int gemv_smem() {
-    return kWarpsPerBlock * kDepth * slot_bytes<MODE, NCH>();
+    return kWarpsPerBlock * kSlots * slot_bytes<MODE>();
 }
 
 template <int MODE, int NCH>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
-    k_gemv(const GemvParams p) {
+    k_gemv(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     constexpr int NMAT = MODE == kGateUp ? 2 : 1;
-    constexpr int kPieces = 2 * NMAT + 2 * NCH;  // 16-byte pieces per lane per step
-    extern __shared__ __align__(16) uint4 ring_smem[];
+    constexpr int kSlotBytes = slot_bytes<MODE>();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ uint64_t full[kWarpsPerBlock][kSlots];
     __shared__ int s_start[kMaxE + 1];  // first item of expert e
     __shared__ int s_off[kMaxE + 1];
-    const int lane = threadIdx.x & 31, g8 = lane >> 2, c = lane & 3;
-    // this lane's pieces of slot q: ring[(q * kPieces + piece) * 32]
-    uint4* ring = ring_smem + (threadIdx.x >> 5) * kDepth * kPieces * 32 + lane;
+    __shared__ int s_abort;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, c = lane & 3;
+    uint8_t* ring = smem_raw + warp * kSlots * kSlotBytes;
     const int E = p.E, S = p.S;
     const int64_t K = MODE == kGateUp ? p.d : p.f;
     const int64_t rows_out = MODE == kGateUp ? p.f : p.d;
     const int groups = (int)(rows_out / 16);
     if (threadIdx.x <= E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
+    if (lane == 0)
+        for (int i = 0; i < kSlots; ++i) sm100::mbar_init(&full[warp][i], 1);
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        sm100::fence_mbar_init();
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         int run = 0;
@@ -125,12 +163,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         s_start[E] = run;
     }
     __syncthreads();
+    volatile int* abort = &s_abort;
     const int n_items = s_start[E];
     const int W = gridDim.x * kWarpsPerBlock;
-    const int wid = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+    const int wid = blockIdx.x * kWarpsPerBlock + warp;
     const int n_mine = wid < n_items ? (n_items - 1 - wid) / W + 1 : 0;
-    const int nw = (int)(K / S / 64);  // 64-byte steps per item
-    const int64_t total = (int64_t)n_mine * nw;
+    const int kb_item = (int)(K / 64 / S);            // k-blocks per item
+    const int nsl = (kb_item + kNB - 1) / kNB;        // ring slots per item
+    const int64_t total = (int64_t)n_mine * nsl;
     if (total == 0) return;
 
     auto item_of = [&](int it) {
@@ -146,70 +186,37 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         return r;
     };
 
-    // ---- prefetch cursor (item iteration pi, step pj): weight rows and the
-    // activation (x or h) rows of the item's tokens, both loaded kDepth-1
-    // steps ahead of use
+    // ---- producer cursor (lane 0 issues the TMA boxes of slot-sized pieces)
     int pi = 0, pj = 0;
-    const int8_t* pw[2 * NMAT];
-    const uint16_t* pb[NCH];
+    int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
     auto set_prefetch_item = [&](int it) {
         const Item u = item_of(it);
-        const int64_t kz = (int64_t)u.z * nw * 64;
-        if (MODE == kGateUp) {
-            const int8_t* base = p.w + ((int64_t)u.e * 2 * p.f + u.group * 16 + g8) * K + 16 * c + kz;
-            pw[0] = base;
-            pw[1] = base + 8 * K;
-            pw[NMAT] = base + p.f * K;
-            pw[NMAT + 1] = base + p.f * K + 8 * K;
-        } else {
-            const int8_t* base = p.w + ((int64_t)u.e * p.d + u.group * 16 + g8) * K + 16 * c + kz;
-            pw[0] = base;
-            pw[1] = base + 8 * K;
-        }
-        const int b0 = s_off[u.e] + u.pass * 8 * NCH;
-        const int cp = min(8 * NCH, s_off[u.e + 1] - b0);
-#pragma unroll
-        for (int n = 0; n < NCH; ++n) {
-            const int slot = n * 8 + g8;
-            if (slot < cp) {
-                const int64_t row = MODE == kGateUp ? (int64_t)(p.perm[b0 + slot] / p.top_k)
-                                                    : (int64_t)(b0 + slot);
-                pb[n] = p.b_src + row * K + 16 * c + kz;
-            } else {
-                pb[n] = nullptr;
-            }
-        }
+        prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16 : u.e * (int)p.d + u.group * 16;
+        pk = u.z * kb_item * 64;
     };
-    // each thread copies (cp.async) exactly the pieces it will later read, so
-    // the shared ring needs no synchronisation beyond the thread's own waits
     auto issue = [&](int slot) {
-        uint4* dst = ring + slot * kPieces * 32;
+        if (lane == 0) {
+            uint8_t* dst = ring + slot * kSlotBytes;
+            sm100::mbar_arrive_expect_tx(&full[warp][slot], kSlotBytes);
 #pragma unroll
-        for (int m = 0; m < 2 * NMAT; ++m) {
-            cp_async_16(dst + m * 32, pw[m], 16);
-            pw[m] += 64;
-        }
+            for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-        for (int n = 0; n < NCH; ++n) {
-            const uint16_t* src = pb[n] ? pb[n] : p.b_src;
-            const uint32_t bytes = pb[n] ? 16u : 0u;
-            cp_async_16(dst + (2 * NMAT + 2 * n) * 32, src, bytes);
-            cp_async_16(dst + (2 * NMAT + 2 * n + 1) * 32, src + 8, bytes);
-            if (pb[n]) pb[n] += 64;
+                for (int b = 0; b < kNB; ++b)
+                    sm100::tma_load_2d(dst + (m * kNB + b) * 1024, &tmW, &full[warp][slot],
+                                       pk + (pj * kNB + b) * 64, prow + m * (int)p.f);
         }
-        if (++pj == nw) {
+        if (++pj == nsl) {
             pj = 0;
             if (++pi < n_mine) set_prefetch_item(pi);
         }
     };
     set_prefetch_item(0);
+    if (lane == 0) sm100::tma_prefetch_desc(&tmW);
 #pragma unroll
-    for (int q = 0; q < kDepth - 1; ++q) {
+    for (int q = 0; q < kSlots - 1; ++q)
         if (q < total) issue(q);
-        cp_async_commit();
-    }
 
-    // ---- consumer state
+    // ---- consumer state: activation fragments are loaded one slot ahead
     float acc[NCH][NMAT][2][4];
 #pragma unroll
     for (int n = 0; n < NCH; ++n)
@@ -217,60 +224,121 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[n][m][0][i] = acc[n][m][1][i] = 0.0f;
-    Item cu{};
-    int base = 0, cnt_pass = 0;
-    int ci = 0, cj = 0;
-    auto set_consumer_item = [&](int it) {
-        cu = item_of(it);
-        base = s_off[cu.e] + cu.pass * 8 * NCH;
-        cnt_pass = min(8 * NCH, s_off[cu.e + 1] - base);
+    struct Cur {
+        Item u;
+        int base, cnt_pass;
+        const uint16_t* b[NCH];
     };
-    set_consumer_item(0);
-
-    int cslot = 0, pslot = kDepth - 1;  // consumed slot, next slot to fill
-    for (int64_t q = 0; q < total; ++q) {
-        {
-            if (q + kDepth - 1 < total) issue(pslot);
-            pslot = pslot == kDepth - 1 ? 0 : pslot + 1;
-            cp_async_commit();  // one group per step, empty ones included
-            cp_async_wait<kDepth - 1>();  // step q has landed
-            const uint4* src = ring + cslot * kPieces * 32;
-            cslot = cslot == kDepth - 1 ? 0 : cslot + 1;
-            uint4 wq[2 * NMAT];
+    auto make_cur = [&](int it) {
+        Cur r;
+        r.u = item_of(it);
+        r.base = s_off[r.u.e] + r.u.pass * 8 * NCH;
+        r.cnt_pass = min(8 * NCH, s_off[r.u.e + 1] - r.base);
+        const int64_t kz = (int64_t)r.u.z * kb_item * 64;
 #pragma unroll
-            for (int m = 0; m < 2 * NMAT; ++m) wq[m] = src[m * 32];
+        for (int n = 0; n < NCH; ++n) {
+            const int slot = n * 8 + g8;
+            if (slot < r.cnt_pass) {
+                const int64_t row = MODE == kGateUp ? (int64_t)(p.perm[r.base + slot] / p.top_k)
+                                                    : (int64_t)(r.base + slot);
+                r.b[n] = p.b_src + row * K + 16 * c + kz;
+            } else {
+                r.b[n] = nullptr;
+            }
+        }
+        return r;
+    };
+    uint32_t bn[kNB][NCH][8];
+    auto load_slot_b = [&](const Cur& r, int j) {
+#pragma unroll
+        for (int b = 0; b < kNB; ++b)
 #pragma unroll
             for (int n = 0; n < NCH; ++n) {
-                if (n * 8 < cnt_pass) {
-                    const uint4 b0 = src[(2 * NMAT + 2 * n) * 32];
-                    const uint4 b1 = src[(2 * NMAT + 2 * n + 1) * 32];
-                    const uint32_t b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                    mma_block(acc[n][0], wq[0], wq[1], b);
-                    if (MODE == kGateUp) mma_block(acc[n][NMAT - 1], wq[2], wq[3], b);
+                const int kb = j * kNB + b;
+                load_b(r.b[n] && kb < kb_item ? r.b[n] + kb * 64 : nullptr, bn[b][n]);
+            }
+    };
+    Cur cur = make_cur(0), nxt{};
+    load_slot_b(cur, 0);
+    int ci = 0, cj = 0, cslot = 0;
+    uint32_t cphase = 0;
+    bool ok = true;
+    for (int64_t q = 0; q < total && ok; ++q) {
+        // refill the slot consumed in the previous iteration
+        if (q + kSlots - 1 < total) {
+            __syncwarp();
+            if (lane == 0) sm100::fence_proxy_async_smem();
+            issue((int)((q + kSlots - 1) % kSlots));
+        }
+        uint32_t bc[kNB][NCH][8];
+#pragma unroll
+        for (int b = 0; b < kNB; ++b)
+#pragma unroll
+            for (int n = 0; n < NCH; ++n)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bc[b][n][i] = bn[b][n][i];
+        if (cj + 1 < nsl) {
+            load_slot_b(cur, cj + 1);
+        } else if (ci + 1 < n_mine) {
+            nxt = make_cur(ci + 1);
+            load_slot_b(nxt, 0);
+        }
+        if (!sm100::mbar_wait(&full[warp][cslot], cphase, abort)) {
+            ok = false;
+            break;
+        }
+        const uint8_t* src = ring + cslot * kSlotBytes + g8 * 64 + 16 * c;
+#pragma unroll
+        for (int b = 0; b < kNB; ++b) {
+            if (cj * kNB + b < kb_item) {
+                uint4 wq[2 * NMAT];
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    wq[2 * m] = *reinterpret_cast<const uint4*>(src + (m * kNB + b) * 1024);
+                    wq[2 * m + 1] = *reinterpret_cast<const uint4*>(src + (m * kNB + b) * 1024 + 8 * 64);
+                }
+#pragma unroll
+                for (int n = 0; n < NCH; ++n) {
+                    if (n * 8 < cur.cnt_pass) {
+                        mma_block<MODE == kGateUp>(acc[n][0], wq[0], wq[1], bc[b][n]);
+                        if (MODE == kGateUp) mma_block<true>(acc[n][NMAT - 1], wq[2], wq[3], bc[b][n]);
+                    }
                 }
             }
-                if (++cj == nw) {
-                    // end of item: raw partial sums -> P[z][slot][col]
-                    const int64_t cols = MODE == kGateUp ? 2 * p.f : p.d;
-                    float* P = p.P + (int64_t)cu.z * p.A * cols;
+        }
+        if (++cslot == kSlots) {
+            cslot = 0;
+            cphase ^= 1u;
+        }
+        if (++cj == nsl) {
+            // end of item: raw partial sums -> P[z][slot][col]
+            const int64_t cols = MODE == kGateUp ? 2 * p.f : p.d;
+            float* P = p.P + (int64_t)cur.u.z * p.A * cols;
 #pragma unroll
-                    for (int n = 0; n < NCH; ++n)
+            for (int n = 0; n < NCH; ++n)
 #pragma unroll
-                        for (int m = 0; m < NMAT; ++m)
+                for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int slot = n * 8 + 2 * c + (i & 1);
-                                const int64_t col = (int64_t)m * p.f + cu.group * 16 + g8 + (i >> 1) * 8;
-                                if (slot < cnt_pass)
-                                    P[(int64_t)(base + slot) * cols + col] = acc[n][m][0][i] + acc[n][m][1][i];
-                                acc[n][m][0][i] = acc[n][m][1][i] = 0.0f;
-                            }
-                    cj = 0;
-                    if (++ci < n_mine) set_consumer_item(ci);
-                }
+                    for (int i = 0; i < 4; ++i) {
+                        const int slot = n * 8 + 2 * c + (i & 1);
+                        const int64_t col = (int64_t)m * p.f + cur.u.group * 16 + g8 + (i >> 1) * 8;
+                        if (slot < cur.cnt_pass)
+                            P[(int64_t)(cur.base + slot) * cols + col] = acc[n][m][0][i] + acc[n][m][1][i];
+                        acc[n][m][0][i] = acc[n][m][1][i] = 0.0f;
+                    }
+            cj = 0;
+            if (++ci < n_mine) cur = nxt;
         }
     }
-    cp_async_wait<0>();
+    // leave only when no copy is still landing in this warp's ring
+    if (lane == 0) {
+        for (int64_t h = q_drain_begin(total, kSlots); h < total; ++h) {
+            const long long t0 = clock64();
+            while (!sm100::mbar_try_wait(&full[warp][h % kSlots], (uint32_t)((h / kSlots) & 1)))
+                if (clock64() - t0 > sm100::kWaitCycles) break;
+        }
+        if (!ok && p.err) flag_error(p.err, kErrTimeout);
+    }
 }
 
 // Expert of a grouped slot (offsets[e] <= slot < offsets[e+1]).
@@ -280,10 +348,64 @@ __device__ __forceinline__ int expert_of_slot(const int* off, int E, int slot) {
     return e;
 }
 
-// H[slot][n] = bf16( silu(s_g * sum_z Pg) * (s_u * sum_z Pu) ), pieces in order.
+// Power-of-two shift that puts the largest |value| of a row (biased fp32 /
+// bf16 exponent field emax) into [2^14, 2^15), inside fp16's normal range.
+__device__ __forceinline__ int row_shift(int emax) {
+    if (emax == 0) return 0;
+    return max(emax - 127 - 14, -100);
+}
+
+__device__ __forceinline__ int block_max_int(int v, int* red) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int m = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m = max(m, red[i]);
+    __syncthreads();
+    return m;
+}
+
+// x16[t] = fp16(x[t] * 2^-xexp[t]).  A bf16 value has 8 significant bits, so
+// the scaled value is exactly representable in fp16 unless it falls below
+// fp16's normal range (2^-14, i.e. 2^28 times smaller than the row maximum).
 __global__ void __launch_bounds__(256)
-    k_swiglu(const float* __restrict__ P, int S, int64_t A, int64_t f, int E,
-             const int32_t* __restrict__ offsets, const float* __restrict__ sgu,
+    k_prep_x16(const uint16_t* __restrict__ x, int64_t d, uint16_t* __restrict__ x16,
+               int32_t* __restrict__ xexp) {
+    __shared__ int red[8];
+    const int64_t t = blockIdx.x;
+    const uint16_t* xr = x + t * d;
+    int m = 0;
+    for (int64_t k = threadIdx.x * 8; k < d; k += 256 * 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, (int)max((u[i] >> 7) & 0xffu, (u[i] >> 23) & 0xffu));
+    }
+    const int sh = row_shift(block_max_int(m, red));
+    if (threadIdx.x == 0) xexp[t] = sh;
+    const float scale = ldexpf(1.0f, -sh);
+    for (int64_t k = threadIdx.x * 8; k < d; k += 256 * 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __half2 h = __floats2half2_rn(__uint_as_float(u[i] << 16) * scale,
+                                                __uint_as_float(u[i] & 0xffff0000u) * scale);
+            o[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(x16 + t * d + k) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// H[slot][n] = bf16( silu(s_g * u_g) * (s_u * u_u) ), u = 2^xexp[token] *
+// sum_z P (pieces in order; the power-of-two factor undoes the fp16 staging
+// of x exactly).
+__global__ void __launch_bounds__(256)
+    k_swiglu(const float* __restrict__ P, int S, int64_t A, int64_t f, int E, int top_k,
+             const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
+             const int32_t* __restrict__ xexp, const float* __restrict__ sgu,
              uint16_t* __restrict__ H) {
     __shared__ int s_off[kMaxE + 1];
     if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
@@ -294,15 +416,16 @@ __global__ void __launch_bounds__(256)
         const int slot = (int)(v / f);
         const int64_t n = v % f;
         const int e = expert_of_slot(s_off, E, slot);
+        const float sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
         float vg = 0.f, vu = 0.f;
         for (int z = 0; z < S; ++z) {
             const float* row = P + ((int64_t)z * A + slot) * 2 * f;
             vg += row[n];
             vu += row[f + n];
         }
-        const float* s = sgu + (int64_t)e * 2 * f;
-        H[(int64_t)slot * f + n] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(silu_f32(s[n] * vg) * (s[f + n] * vu)));
+        const float* sg = sgu + (int64_t)e * 2 * f;
+        H[(int64_t)slot * f + n] = __bfloat16_as_ushort(
+            __float2bfloat16_rn(silu_f32(sg[n] * (vg * sx)) * (sg[f + n] * (vu * sx))));
     }
 }
 
@@ -376,30 +499,39 @@ int grid_for(int64_t work, int num_sms, int per_sm) {
     return (int)(blocks < 1 ? 1 : blocks);
 }
 
-// One full wave: the resident CTAs per SM at the kernel's register use.
+// One full wave: the resident CTAs per SM at the kernel's register and
+// shared-memory use.
 template <int MODE, int NCH>
 int gemv_grid(int num_sms) {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv<MODE, NCH>,
                                                       kWarpsPerBlock * 32,
-                                                      gemv_smem<MODE, NCH>()) != cudaSuccess ||
+                                                      gemv_smem<MODE>()) != cudaSuccess ||
         per_sm < 1)
         per_sm = 2;
     return num_sms * per_sm;
 }
 
 template <int MODE, int NCH>
-cudaError_t set_gemv_smem() {
-    return cudaFuncSetAttribute(k_gemv<MODE, NCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                gemv_smem<MODE, NCH>());
+cudaError_t launch_gemv(const GemvParams& p, int num_sms, cudaStream_t stream) {
+    // weights [rows][K] int8, boxes of 64 bytes x 16 rows
+    const int64_t K = MODE == kGateUp ? p.d : p.f;
+    const int64_t rows = MODE == kGateUp ? (int64_t)p.E * 2 * p.f : (int64_t)p.E * p.d;
+    CUtensorMap map;
+    if (!encode_2d(&map, p.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, K, 16, 64,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(k_gemv<MODE, NCH>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           gemv_smem<MODE>());
+    if (err != cudaSuccess) return err;
+    k_gemv<MODE, NCH><<<gemv_grid<MODE, NCH>(num_sms), kWarpsPerBlock * 32, gemv_smem<MODE>(),
+                        stream>>>(map, p);
+    return cudaGetLastError();
 }
 
 template <int NCH>
 cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
-    cudaError_t err = set_gemv_smem<kGateUp, NCH>();
-    if (err == cudaSuccess) err = set_gemv_smem<kDown, NCH>();
-    if (err != cudaSuccess) return err;
-    const int grid = gemv_grid<kGateUp, NCH>(a.num_sms);
     GemvParams p{};
     p.E = a.E;
     p.top_k = a.top_k;
@@ -408,16 +540,21 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.A = a.A;
     p.offsets = a.offsets;
     p.perm = a.perm;
+    p.err = a.err;
     p.w = a.wgu;
     p.S = a.split_gu;
-    p.b_src = static_cast<const uint16_t*>(a.x);
+    p.b_src = static_cast<const uint16_t*>(a.x16);
     p.P = a.P_gu;
+    if (a.mark) a.mark(1, false, stream);
+    k_prep_x16<<<(unsigned)a.T, 256, 0, stream>>>(static_cast<const uint16_t*>(a.x), a.d,
+                                                  static_cast<uint16_t*>(a.x16), a.xexp);
+    if (a.mark) a.mark(1, true, stream);
     if (a.mark) a.mark(2, false, stream);
-    k_gemv<kGateUp, NCH><<<grid, kWarpsPerBlock * 32, gemv_smem<kGateUp, NCH>(), stream>>>(p);
-    err = cudaGetLastError();
+    cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
     if (err == cudaSuccess)
         k_swiglu<<<grid_for(a.A * a.f, a.num_sms, 8), 256, 0, stream>>>(
-            a.P_gu, a.split_gu, a.A, a.f, a.E, a.offsets, a.sgu, static_cast<uint16_t*>(a.H));
+            a.P_gu, a.split_gu, a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
+            static_cast<uint16_t*>(a.H));
     if (a.mark) a.mark(2, true, stream);
     if (err != cudaSuccess) return err;
     p.w = a.wd;
@@ -425,10 +562,9 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.b_src = static_cast<const uint16_t*>(a.H);
     p.P = a.P_d;
     if (a.mark) a.mark(3, false, stream);
-    k_gemv<kDown, NCH><<<gemv_grid<kDown, NCH>(a.num_sms), kWarpsPerBlock * 32,
-                         gemv_smem<kDown, NCH>(), stream>>>(p);
+    err = launch_gemv<kDown, NCH>(p, a.num_sms, stream);
     if (a.mark) a.mark(3, true, stream);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace

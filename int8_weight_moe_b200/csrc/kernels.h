@@ -1,10 +1,19 @@
 // Internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace jmoe {
+
+// TMA tensor map of a row-major 2-D tensor [rows][cols] with boxes of
+// box_rows x box_cols elements (false if the driver entry point is missing or
+// the encoder rejects the arguments).
+bool tensormap_available();
+bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
+               uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+               CUtensorMapSwizzle swizzle);
 
 // Bits of the sticky device error word (see jmoe_last_error).
 enum : unsigned {
@@ -47,6 +56,8 @@ struct DecodeArgs {
     const int32_t* offsets;  // [E+1]
     const int32_t* perm;     // [A]
     const int32_t* inv;      // [A]
+    void* x16;            // fp16 [T][d]: x * 2^-xexp[t] (workspace)
+    int32_t* xexp;        // [T] power-of-two shift of each token row (workspace)
     void* H;              // bf16 [A][f], expert-grouped slot order (workspace)
     float* P_gu;          // fp32 [split_gu][A][2f] partial sums (workspace)
     float* P_d;           // fp32 [split_d][A][d] partial sums (workspace)

@@ -406,39 +406,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ----------------------------------------------------------------------------- host side
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// Row-major 2-D tensor [rows][cols]; a box of box_rows x box_cols elements.
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
-              uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
-              CUtensorMapSwizzle swizzle) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
-    const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
                         int num_sms, cudaStream_t stream) {
@@ -451,7 +418,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmPa
 
 }  // namespace
 
-bool prefill_available() { return encode_fn() != nullptr; }
+bool prefill_available() { return tensormap_available(); }
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (a.T == 0) return cudaSuccess;
@@ -467,13 +434,13 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
 
     CUtensorMap mA1, mB1, mA2, mB2;
     const bool ok =
-        make_map(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BH, BK,
+        encode_2d(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-        make_map(&mB1, a.wgu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * 2 * a.f, a.d,
+        encode_2d(&mB1, a.wgu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * 2 * a.f, a.d,
                  BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        make_map(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BH, BK,
+        encode_2d(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-        make_map(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BN, BK,
+        encode_2d(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BN, BK,
                  CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
 

@@ -70,7 +70,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the size query and the forward calls.
 struct Workspace {
     size_t offsets, padded_offsets, perm, inv;  // routing tables
-    size_t H, Pgu, Pd, x16, xexp;               // decode path
+    size_t H, Hb, Pgu, Pd, x16, xexp, hmax;     // decode path
     int split_gu, split_d;
     size_t xperm, Hp, Yg;                       // tensor-core path
     size_t total;
@@ -102,8 +102,10 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
         w.split_d = jmoe::decode_split(f, units_d > 0 ? (target + units_d - 1) / units_d : 1,
                                        row_d > 0 ? (8LL << 20) / row_d : 1);
         w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
+        w.Hb = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
         w.x16 = take(sizeof(uint16_t) * (size_t)T * (size_t)d);
         w.xexp = take(sizeof(int32_t) * (size_t)T);
+        w.hmax = take(sizeof(int32_t) * (size_t)A);
         w.Pgu = take((size_t)w.split_gu * (size_t)row_gu);
         w.Pd = take((size_t)w.split_d * (size_t)row_d);
     } else {
@@ -171,6 +173,7 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         a.P_d = static_cast<float*>(at(w.Pd));
         a.split_gu = w.split_gu; a.split_d = w.split_d;
         a.x16 = at(w.x16); a.xexp = static_cast<int32_t*>(at(w.xexp));
+        a.Hb = at(w.Hb); a.hmax = static_cast<int32_t*>(at(w.hmax));
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;

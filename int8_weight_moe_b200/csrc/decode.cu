@@ -6,17 +6,16 @@
 // summary, section "ExpertsInt8 Quantization (Section 3.1)", steps 3-4): the
 // INT8 weights cross HBM once and are turned back into 16-bit floating point
 // on chip; the activations keep their BF16 values.  Every weight byte goes
-// HBM -> shared -> registers and is converted exactly (|q| <= 127).  In the
-// gate/up projection (two thirds of the bytes) the weights become fp16 values
-// -- the same numbers BF16 would hold, but the int8 -> fp16 conversion costs
-// half the ALU work -- and the token rows are staged as fp16 after a
-// power-of-two shift per token that brings the row maximum into [2^14, 2^15):
-// a bf16 value has 8 significant bits, so the staged values are exact and
-// every product equals the bf16 one; the shift is undone exactly after the dot
-// product.  The down projection uses bf16 weights against the bf16 hidden
-// activations.  The per-output-channel scale is applied once after the dot
-// product (an exact refactoring of sum_k x_k (q_k s)).  mma.sync m16n8k16
-// (16-bit in, fp32 accumulate), up to 8 tokens of the expert as the columns.
+// HBM -> shared (TMA) -> registers and is converted exactly (|q| <= 127) into
+// fp16 -- the same number BF16 would hold, at half the ALU cost of an
+// int8 -> bf16 conversion.  The activation operand (token rows for gate/up,
+// BF16-rounded hidden rows for down) is staged as fp16 after a power-of-two
+// shift per row that brings the row maximum into [2^14, 2^15): a bf16 value
+// has 8 significant bits, so the staged values are exact and every product
+// equals the bf16 one; the shifts are undone exactly after the dot products.
+// The per-output-channel scale is applied once after the dot product (an
+// exact refactoring of sum_k x_k (q_k s)).  mma.sync m16n8k16 (f16 in, fp32
+// accumulate), up to 8 tokens of the expert as the columns.
 
 // Fragment trick: the dot product does not care in which order k is summed,
 // so the 16 k-columns of an MMA step are a permutation of the 64-wide k-block
@@ -38,7 +37,8 @@
 // stores its raw fp32 partial sums; the small follow-up kernels add the S
 // pieces in a fixed order (deterministic) and apply scales, SwiGLU, gates:
 //   k_prep_x16 -> x16 (fp16, per-token shift)
-//   k_gemv<gate/up> -> P_gu[S][slot][2f] -> k_swiglu -> H (bf16, slot order)
+//   k_gemv<gate/up> -> P_gu[S][slot][2f] -> k_swiglu -> Hb (bf16) + row maxima
+//                                         -> k_h16 -> H (fp16, per-slot shift)
 //   k_gemv<down>    -> P_d [S][slot][d]  -> k_combine -> out (bf16)
 #include <cuda.h>
 
@@ -114,14 +114,19 @@ __device__ __forceinline__ int64_t q_drain_begin(int64_t total, int slots) {
     return total > slots ? total - slots : 0;
 }
 
-constexpr int kNB = 2;     // 64-byte k-blocks per ring slot
-constexpr int kSlots = 3;  // ring slots per warp: two slots (4 KB of gate/up weights) in flight
+constexpr int kSlots = 3;  // ring slots per warp: two 4 KB slots in flight
+
+// 64-byte k-blocks per ring slot: 4 KB of weights per slot in both modes.
+template <int MODE>
+constexpr int nb_of() {
+    return MODE == kGateUp ? 2 : 4;
+}
 
 // Shared memory of one warp: kSlots x [matrix][k-block][16 rows][64 B]; the
 // dense 64-byte row pitch makes the fragment reads of a warp conflict-free.
 template <int MODE>
 constexpr int slot_bytes() {
-    return (MODE == kGateUp ? 2 : 1) * kNB * 16 * 64;
+    return (MODE == kGateUp ? 2 : 1) * nb_of<MODE>() * 16 * 64;
 }
 
 template <int MODE>
@@ -133,6 +138,7 @@ template <int MODE, int NCH>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     k_gemv(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
     constexpr int NMAT = MODE == kGateUp ? 2 : 1;
+    constexpr int kNB = nb_of<MODE>();
     constexpr int kSlotBytes = slot_bytes<MODE>();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ uint64_t full[kWarpsPerBlock][kSlots];
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int n = 0; n < NCH; ++n) {
                     if (n * 8 < cur.cnt_pass) {
-                        mma_block<MODE == kGateUp>(acc[n][0], wq[0], wq[1], bc[b][n]);
+                        mma_block<true>(acc[n][0], wq[0], wq[1], bc[b][n]);
                         if (MODE == kGateUp) mma_block<true>(acc[n][NMAT - 1], wq[2], wq[3], bc[b][n]);
                     }
                 }
@@ -371,9 +377,10 @@ __device__ __forceinline__ int block_max_int(int v, int* red) {
 // fp16's normal range (2^-14, i.e. 2^28 times smaller than the row maximum).
 __global__ void __launch_bounds__(256)
     k_prep_x16(const uint16_t* __restrict__ x, int64_t d, uint16_t* __restrict__ x16,
-               int32_t* __restrict__ xexp) {
+               int32_t* __restrict__ xexp, int32_t* __restrict__ hmax, int top_k) {
     __shared__ int red[8];
     const int64_t t = blockIdx.x;
+    if (threadIdx.x < top_k) hmax[t * top_k + threadIdx.x] = 0;  // for k_swiglu's maxima
     const uint16_t* xr = x + t * d;
     int m = 0;
     for (int64_t k = threadIdx.x * 8; k < d; k += 256 * 8) {
@@ -399,42 +406,81 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// H[slot][n] = bf16( silu(s_g * u_g) * (s_u * u_u) ), u = 2^xexp[token] *
-// sum_z P (pieces in order; the power-of-two factor undoes the fp16 staging
-// of x exactly).
+// h = bf16( silu(s_g * u_g) * (s_u * u_u) ), u = 2^xexp[token] * sum_z P
+// (pieces in order; the power-of-two factor undoes the fp16 staging of x
+// exactly).  h goes to Hb (bf16) and the largest exponent field of each slot
+// to hmax[slot] (zeroed by k_prep_x16).
 __global__ void __launch_bounds__(256)
     k_swiglu(const float* __restrict__ P, int S, int64_t A, int64_t f, int E, int top_k,
              const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
              const int32_t* __restrict__ xexp, const float* __restrict__ sgu,
-             uint16_t* __restrict__ H) {
+             uint16_t* __restrict__ Hb, int32_t* __restrict__ hmax) {
     __shared__ int s_off[kMaxE + 1];
     if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
     __syncthreads();
     const int64_t total = (int64_t)s_off[E] * f;
-    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
-         v += (int64_t)gridDim.x * blockDim.x) {
-        const int slot = (int)(v / f);
-        const int64_t n = v % f;
-        const int e = expert_of_slot(s_off, E, slot);
-        const float sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
-        float vg = 0.f, vu = 0.f;
-        for (int z = 0; z < S; ++z) {
-            const float* row = P + ((int64_t)z * A + slot) * 2 * f;
-            vg += row[n];
-            vu += row[f + n];
+    const int lane = threadIdx.x & 31;
+    // warp-uniform loop (the warp-wide maximum below needs all 32 lanes)
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); v0 < total;
+         v0 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t v = v0 + lane;
+        const bool live = v < total;
+        const int slot = live ? (int)(v / f) : (int)(v0 / f);
+        int ex = 0;
+        if (live) {
+            const int64_t n = v % f;
+            const int e = expert_of_slot(s_off, E, slot);
+            const float sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
+            float vg = 0.f, vu = 0.f;
+            for (int z = 0; z < S; ++z) {
+                const float* row = P + ((int64_t)z * A + slot) * 2 * f;
+                vg += row[n];
+                vu += row[f + n];
+            }
+            const float* sg = sgu + (int64_t)e * 2 * f;
+            const uint16_t hb = __bfloat16_as_ushort(
+                __float2bfloat16_rn(silu_f32(sg[n] * (vg * sx)) * (sg[f + n] * (vu * sx))));
+            Hb[(int64_t)slot * f + n] = hb;
+            ex = (hb >> 7) & 0xff;
         }
-        const float* sg = sgu + (int64_t)e * 2 * f;
-        H[(int64_t)slot * f + n] = __bfloat16_as_ushort(
-            __float2bfloat16_rn(silu_f32(sg[n] * (vg * sx)) * (sg[f + n] * (vu * sx))));
+        // one atomic per warp when the warp covers a single slot
+        int m = ex;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const int slot0 = __shfl_sync(0xffffffffu, slot, 0);
+        if (__all_sync(0xffffffffu, slot == slot0)) {
+            if (lane == 0 && m > 0) atomicMax(&hmax[slot0], m);
+        } else if (ex > 0) {
+            atomicMax(&hmax[slot], ex);
+        }
     }
 }
 
-// out[t][m] = bf16( sum_j g_tj * (s_d[e_j][m] * sum_z P[z][inv[a]][m]) ), a = t*top_k + j.
+// H16[slot][n] = fp16( Hb[slot][n] * 2^-hexp ), hexp = row_shift(hmax[slot]):
+// the bf16 values are kept exactly (8 significant bits, row maximum brought
+// into [2^14, 2^15)).
+__global__ void __launch_bounds__(256)
+    k_h16(const uint16_t* __restrict__ Hb, int64_t f, const int32_t* __restrict__ offsets, int E,
+          const int32_t* __restrict__ hmax, uint16_t* __restrict__ H16) {
+    const int64_t total = (int64_t)offsets[E] * f / 2;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+         v += (int64_t)gridDim.x * blockDim.x) {
+        const int slot = (int)((2 * v) / f);
+        const float scale = ldexpf(1.0f, -row_shift(hmax[slot]));
+        const uint32_t u = reinterpret_cast<const uint32_t*>(Hb)[v];
+        const __half2 h = __floats2half2_rn(__uint_as_float(u << 16) * scale,
+                                            __uint_as_float(u & 0xffff0000u) * scale);
+        reinterpret_cast<uint32_t*>(H16)[v] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+}
+
+// out[t][m] = bf16( sum_j g_tj * (s_d[e_j][m] * (2^hexp * sum_z P[z][inv[a]][m])) ),
+// a = t*top_k + j, hexp = row_shift(hmax[inv[a]]).
 __global__ void __launch_bounds__(256)
     k_combine(const float* __restrict__ P, int S, int64_t A, int64_t T, int64_t d, int top_k,
               int E, const int32_t* __restrict__ ids, const float* __restrict__ gates,
-              const int32_t* __restrict__ inv, const float* __restrict__ sd,
-              uint16_t* __restrict__ out) {
+              const int32_t* __restrict__ inv, const int32_t* __restrict__ hmax,
+              const float* __restrict__ sd, uint16_t* __restrict__ out) {
     const int64_t nvec = d / 4;
     const int64_t total = T * nvec;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -451,12 +497,13 @@ __global__ void __launch_bounds__(256)
                 const float4 q = *reinterpret_cast<const float4*>(P + ((int64_t)z * A + slot) * d + m);
                 y[0] += q.x; y[1] += q.y; y[2] += q.z; y[3] += q.w;
             }
+            const float hs = ldexpf(1.0f, row_shift(hmax[slot]));
             const float4 s = *reinterpret_cast<const float4*>(sd + (int64_t)e * d + m);
             const float gw = gates[a];
-            o[0] += gw * (s.x * y[0]);
-            o[1] += gw * (s.y * y[1]);
-            o[2] += gw * (s.z * y[2]);
-            o[3] += gw * (s.w * y[3]);
+            o[0] += gw * (s.x * (y[0] * hs));
+            o[1] += gw * (s.y * (y[1] * hs));
+            o[2] += gw * (s.z * (y[2] * hs));
+            o[3] += gw * (s.w * (y[3] * hs));
         }
         uint2 r;
         r.x = pack_bf16x2(o[0], o[1]);
@@ -547,13 +594,18 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.P = a.P_gu;
     if (a.mark) a.mark(1, false, stream);
     k_prep_x16<<<(unsigned)a.T, 256, 0, stream>>>(static_cast<const uint16_t*>(a.x), a.d,
-                                                  static_cast<uint16_t*>(a.x16), a.xexp);
+                                                  static_cast<uint16_t*>(a.x16), a.xexp, a.hmax,
+                                                  a.top_k);
     if (a.mark) a.mark(1, true, stream);
     if (a.mark) a.mark(2, false, stream);
     cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
     if (err == cudaSuccess)
         k_swiglu<<<grid_for(a.A * a.f, a.num_sms, 8), 256, 0, stream>>>(
             a.P_gu, a.split_gu, a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
+            static_cast<uint16_t*>(a.Hb), a.hmax);
+    if (err == cudaSuccess)
+        k_h16<<<grid_for(a.A * a.f / 2, a.num_sms, 8), 256, 0, stream>>>(
+            static_cast<const uint16_t*>(a.Hb), a.f, a.offsets, a.E, a.hmax,
             static_cast<uint16_t*>(a.H));
     if (a.mark) a.mark(2, true, stream);
     if (err != cudaSuccess) return err;
@@ -595,7 +647,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (a.mark) a.mark(4, false, stream);
     k_combine<<<grid_for(a.T * (a.d / 4), a.num_sms, 8), 256, 0, stream>>>(
-        a.P_d, a.split_d, a.A, a.T, a.d, a.top_k, a.E, a.ids, a.gates, a.inv, a.sd,
+        a.P_d, a.split_d, a.A, a.T, a.d, a.top_k, a.E, a.ids, a.gates, a.inv, a.hmax, a.sd,
         static_cast<uint16_t*>(a.out));
     if (a.mark) a.mark(4, true, stream);
     return cudaGetLastError();

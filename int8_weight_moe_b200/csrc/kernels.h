@@ -58,7 +58,9 @@ struct DecodeArgs {
     const int32_t* inv;      // [A]
     void* x16;            // fp16 [T][d]: x * 2^-xexp[t] (workspace)
     int32_t* xexp;        // [T] power-of-two shift of each token row (workspace)
-    void* H;              // bf16 [A][f], expert-grouped slot order (workspace)
+    void* Hb;             // bf16 [A][f]: hidden activations, expert-grouped slot order
+    void* H;              // fp16 [A][f]: Hb * 2^-shift(hmax[slot]) (workspace)
+    int32_t* hmax;        // [A] largest exponent field of each hidden row (workspace)
     float* P_gu;          // fp32 [split_gu][A][2f] partial sums (workspace)
     float* P_d;           // fp32 [split_d][A][d] partial sums (workspace)
     int split_gu, split_d;   // K pieces of the two GEMVs

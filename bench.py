@@ -19,6 +19,7 @@ bounded sample of the same workload (the pages ship no code to run).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -150,7 +151,7 @@ class Layer:
                                   dtype=torch.uint8, device=device)
 
     def step(self, x=None, out=None, route_events=None):
-        """One pass of the hot path on the current stream; returns #kernel launches."""
+        """One pass of the hot path on the current stream."""
         import int8_weight_moe_b200 as jm
 
         x = self.x if x is None else x
@@ -158,9 +159,7 @@ class Layer:
         if self.wl.dense:
             jm.jmoe_mlp_forward(x, self.w_gu[0], self.s_gu[0], self.w_d[0], self.s_d[0], out=out,
                                 workspace=self.ws)
-            # fill (unit gates), grouping, gate/up, down, combine/finalize (+ gather on the
-            # tensor-core path)
-            return 6 if self.prefill_path() else 5
+            return
         if route_events:
             route_events[0].record()
         jm.jmoe_route(x, self.w_router, self.wl.top_k, self.bias, topk_ids=self.ids,
@@ -168,7 +167,6 @@ class Layer:
         if route_events:
             route_events[1].record()
         jm.jmoe_forward(self.desc, x, self.ids, self.gates, out=out, workspace=self.ws)
-        return 6 if self.prefill_path() else 5
 
     def prefill_path(self):
         """Whether the library's automatic choice is the tensor-core path here
@@ -187,20 +185,41 @@ class Layer:
 
 
 def kernel_work(layer: Layer):
-    """Algorithmic work of the dominant kernel (gate/up stage) per launch, and
-    of the whole step: bytes for the HBM-bound regime, FLOPs for prefill."""
+    """Algorithmic work of the dominant kernel (the gate/up GEMM) per launch
+    and of the whole step.  HBM regime: the gate/up GEMV must read the int8
+    gate/up rows of every touched expert (2*f*d bytes each) and each token's
+    activation row once (2*d bytes); the step must read all three matrices of
+    every touched expert, their fp32 scales, and the tokens in and out.
+    Tensor-core regime: 2 FLOPs per multiply-add, 2*f*d per assignment for
+    gate/up, 3*f*d for the whole step."""
     wl = layer.wl
     d, f, A, T = wl.d_model, wl.d_ff, wl.A, wl.T
     touched = layer.touched_experts()
-    gu_bytes = touched * 2 * f * (d + 4) + A * d * 2 + A * f * 2
+    gu_bytes = touched * 2 * f * d + T * d * 2
     step_bytes = touched * 3 * d * f + touched * (2 * f + d) * 4 + T * d * 2 * 2
     return {"touched": touched, "gate_up_bytes": gu_bytes, "step_bytes": step_bytes,
             "gate_up_flops": 4 * A * d * f, "step_flops": 6 * A * d * f}
 
 
-def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: bool = True):
-    """Warm-up, then exactly `steps` timed steps between barriers; per-stage
-    CUDA events recorded live on the launching stream."""
+def _primed_events(n: int):
+    """n timing events whose CUDA handles already exist (torch creates the
+    handle on the first record; the library re-records them later)."""
+    import torch
+
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for ev in evs:
+        ev.record()
+    return evs
+
+
+def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool,
+              stages=("gate_up",), route: bool = False):
+    """Warm-up, then exactly `steps` timed steps between barriers.  Inside the
+    timed region the library records a CUDA event pair on the launching
+    stream around each stage named in `stages` (and the bench around the
+    router if `route`); the other stages record nothing, so the step pays
+    only for the events it needs.  Returns (total ms, mean ms per recorded
+    stage that ran, kernel launches in the timed region)."""
     import torch
 
     import int8_weight_moe_b200 as jm
@@ -208,32 +227,31 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
     for _ in range(warmup):
         layer.step()
     torch.cuda.synchronize()
-    stage_events = []
     if dist_on:
         import torch.distributed as dist
 
         dist.barrier()
     torch.cuda.synchronize()
-    route_events = []
-    if profile:
-        # torch creates the CUDA event handle on the first record: record every
-        # event once now so the library can re-record them inside the steps
-        for _ in range(steps):
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
-            for ev in evs:
-                ev.record()
-            stage_events.append(evs)
-            route_events.append([torch.cuda.Event(enable_timing=True) for _ in range(2)])
-        torch.cuda.synchronize()
+    want = [i for i, name in enumerate(jm.STAGES) if name in stages]
+    stage_events, route_events = [], []
+    for _ in range(steps):
+        evs = [None] * (2 * len(jm.STAGES))
+        primed = _primed_events(2 * len(want))
+        for j, i in enumerate(want):
+            evs[2 * i], evs[2 * i + 1] = primed[2 * j], primed[2 * j + 1]
+        stage_events.append(evs)
+        route_events.append(_primed_events(2) if route else None)
+    torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
-    launches = 0
+    n0 = jm.jmoe_launch_count()
     start.record()
     for i in range(steps):
-        if profile:
+        if want:
             jm.jmoe_profile_events(stage_events[i])
-        launches += layer.step(route_events=route_events[i] if profile else None)
+        layer.step(route_events=route_events[i])
     stop.record()
+    launches = jm.jmoe_launch_count() - n0
     jm.jmoe_profile_events(None)
     torch.cuda.synchronize()
     if dist_on:
@@ -241,28 +259,79 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool, profile: boo
 
         dist.barrier()
     total_ms = start.elapsed_time(stop)
-    stages = {}
-    if profile and not layer.wl.dense:
-        stages["route"] = sum(a.elapsed_time(b) for a, b in route_events) / len(route_events)
-    for i, name in enumerate(jm.STAGES):
-        times = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for evs in stage_events]
-        # a stage that does not run on this path leaves its pre-recorded pair,
-        # which spans no step: report only stages whose events moved
-        if times and min(times) >= 0 and stage_ran(stage_events, i, start):
-            stages[name] = sum(times) / len(times)
-    return total_ms, stages, launches
+    out = {}
+    if route and not layer.wl.dense:
+        out["route"] = sum(a.elapsed_time(b) for a, b in route_events) / len(route_events)
+    for i in want:
+        pairs = [(evs[2 * i], evs[2 * i + 1]) for evs in stage_events]
+        # a stage that does not run on this path leaves its primed pair, which
+        # spans no step: report only stages whose events moved
+        if stage_ran(pairs, start):
+            out[jm.STAGES[i]] = sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
+    return total_ms, out, launches
 
 
-def stage_ran(stage_events, i, start):
-    """True when stage i's events were re-recorded inside the timed region."""
+def stage_breakdown(layer: Layer, steps: int, dist_on: bool):
+    """Mean ms of every stage (and the router), from a separate pass with an
+    event pair around each of them."""
+    import int8_weight_moe_b200 as jm
+
+    _, stages, _ = timed_run(layer, steps, 3, dist_on, stages=jm.STAGES, route=True)
+    return stages
+
+
+def stage_ran(pairs, start):
+    """True when the stage's events were re-recorded after `start`."""
     try:
-        return all(start.elapsed_time(evs[2 * i]) >= 0 for evs in stage_events)
+        return all(start.elapsed_time(a) >= 0 and a.elapsed_time(b) >= 0 for a, b in pairs)
     except RuntimeError:
         return False
 
 
-def roofline_entry(layer: Layer, stages: dict, peaks: dict, traffic=None):
+def sources_sha256(paths):
+    """sha256 over the listed source files (repo-relative), in order."""
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profile_traffic(workload: str, stage: str):
+    """DRAM bytes per launch (read + write) of the kernel behind `stage` on
+    `workload`, from an ncu summary under profiles/.  Each summary lists its
+    figures as "- key: value" lines: stage, workload, traffic_bytes_per_launch,
+    sources and sources_sha256.  None when no summary matches or when any of
+    the kernel's sources changed since the capture (the counters then describe
+    another kernel)."""
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for name in sorted(os.listdir(pdir)):
+        if not name.endswith(".md"):
+            continue
+        kv = {}
+        with open(os.path.join(pdir, name)) as fh:
+            for line in fh:
+                if line.startswith("- ") and ": " in line:
+                    k, v = line[2:].split(": ", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("stage") != stage or kv.get("workload") != workload:
+            continue
+        if "traffic_bytes_per_launch" not in kv or "sources" not in kv:
+            continue
+        try:
+            if sources_sha256(kv["sources"].split()) != kv.get("sources_sha256"):
+                return None
+        except OSError:
+            return None
+        return int(kv["traffic_bytes_per_launch"])
+    return None
+
+
+def roofline_entry(layer: Layer, stages: dict, peaks: dict):
     work = kernel_work(layer)
+    traffic = profile_traffic(layer.wl.name, "gate_up")
     ms = stages.get("gate_up")
     if ms is None or ms <= 0:
         return None
@@ -280,7 +349,7 @@ def roofline_entry(layer: Layer, stages: dict, peaks: dict, traffic=None):
             "ms": round(ms, 4), "peak_source": peaks["source"] + " hbm copy"}
 
 
-def e2e_run(layer: Layer, steps: int, warmup: int):
+def e2e_run(layer: Layer, steps: int, warmup: int, dist_on: bool = False):
     """Same metric through the public API with host buffers: per step a
     host->device copy of the tokens from pinned memory and a device->host read
     of the layer output, inside the timed region."""
@@ -295,6 +364,11 @@ def e2e_run(layer: Layer, steps: int, warmup: int):
         layer.step(x=xd)
         oh.copy_(layer.out, non_blocking=True)
     torch.cuda.synchronize()
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+        torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     start.record()
@@ -408,6 +482,29 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- ranks
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (every rank gets it); the value
+    itself without a process group.  Timings are combined this way: the job
+    takes as long as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank processes its own batch of `tokens_per_rank`
+    tokens per step, so the job processes world * tokens_per_rank per step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------------------- main
 
 
@@ -461,17 +558,16 @@ def main():
     sampler.start()
     total_ms, stages, launches = timed_run(layer, args.steps, args.warmup, dist_on)
     clocks = sampler.stop()
-    if dist_on:
-        import torch.distributed as dist
-
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    dev = torch.device("cuda", local)
+    total_ms = max_over_ranks(total_ms, dev)
     ms = total_ms / args.steps
-    value = world * wl.T / (ms * 1e-3)
+    value = whole_job_tokens_per_s(world, wl.T, ms)
     roof = roofline_entry(layer, stages, peaks)
-    e2e = e2e_run(layer, max(args.steps // 2, 10), 3)
-    e2e["value"] = round(e2e["value"] * world, 1)
+    breakdown = stage_breakdown(layer, min(args.steps, 50), dist_on)
+    e2e = e2e_run(layer, max(args.steps // 2, 10), 3, dist_on)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"], dev)
+    e2e["ms_per_step"] = round(e2e_ms, 4)
+    e2e["value"] = round(whole_job_tokens_per_s(world, wl.T, e2e_ms), 1)
     work = kernel_work(layer)
     step_gbs = work["step_bytes"] / (ms * 1e-3) / 1e9
     del layer
@@ -483,11 +579,12 @@ def main():
             lay = Layer(other, torch.device("cuda", local))
             steps = 20 if other.regime == "prefill" else 100
             tms, st, _ = timed_run(lay, steps, 3, dist_on)
-            oms = tms / steps
+            oms = max_over_ranks(tms, dev) / steps
+            bd = stage_breakdown(lay, steps, dist_on)
             w2 = kernel_work(lay)
-            entry = {"workload": other.name, "tokens_per_s": round(other.T / (oms * 1e-3), 1),
+            entry = {"workload": other.name, "tokens_per_s": round(whole_job_tokens_per_s(world, other.T, oms), 1),
                      "ms_per_step": round(oms, 4), "path": "prefill" if lay.prefill_path() else "decode",
-                     "stages_ms": {k: round(v, 4) for k, v in st.items()},
+                     "stages_ms": {k: round(v, 4) for k, v in bd.items()},
                      "roofline": roofline_entry(lay, st, peaks),
                      "step_hbm_gbs": round(w2["step_bytes"] / (oms * 1e-3) / 1e9, 1),
                      "step_tflops": round(w2["step_flops"] / (oms * 1e-3) / 1e12, 2)}
@@ -512,7 +609,10 @@ def main():
                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches, "clocks": clocks,
-                "stages_ms": {k: round(v, 4) for k, v in stages.items()},
+                "stages_ms": {k: round(v, 4) for k, v in breakdown.items()},
+                "stages_ms_source": "separate pass after the timed one, with an event pair "
+                                    "around every stage (the timed pass records only the "
+                                    "gate/up pair)",
                 "step_hbm_gbs": round(step_gbs, 1),
                 "touched_experts": work["touched"], "also": also}
         print(json.dumps(line), flush=True)

@@ -194,12 +194,22 @@ jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, 
  * handles passed as void*) that the following jmoe_forward / jmoe_mlp_forward
  * calls record on their stream around their kernels: events[2*i] before and
  * events[2*i+1] after stage i, where the stages are 0 = grouping by expert,
- * 1 = row gather (tensor-core path only), 2 = gate/up GEMM + SwiGLU,
- * 3 = down GEMM, 4 = combine.  Stages that do not run record nothing.
- * n = 0 or events = NULL switches recording off.  The registration is
- * process-wide and not thread-safe; the caller keeps the events alive.
- * n must be 0 or 10. */
+ * 1 = row gather (tensor-core path) or activation preparation (decode path),
+ * 2 = gate/up GEMM (with SwiGLU in its epilogue on the tensor-core path),
+ * 3 = down GEMM, 4 = combine, 5 = SwiGLU and down-operand rows (decode path).
+ * Stages that do not run record nothing, and neither do stages whose two
+ * entries are NULL (so a caller can time one stage without the cost of the
+ * other records); one NULL entry of a pair is JMOE_EINVAL.  n = 0 or
+ * events = NULL switches recording off.  The registration is process-wide and
+ * not thread-safe; the caller keeps the events alive.  n must be 0 or 12. */
 jmoe_status jmoe_profile_events(void* const* events, int32_t n);
+
+/* Launch counter (diagnostics; the pages have no counterpart).  Stores in
+ * *count the number of kernels this library has launched in this process
+ * since it was loaded, over all devices and host threads; a caller takes the
+ * difference around a region to count the launches inside it.  Never
+ * synchronises.  Returns JMOE_EINVAL when count is NULL. */
+jmoe_status jmoe_launch_count(uint64_t* count);
 
 /* Reads and clears the device error word of the current device.  Unlike the
  * other calls it synchronises the device.  Returns JMOE_OK when no kernel

@@ -26,9 +26,10 @@ JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 # Every C entry point the header declares.
 EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_permute", "jmoe_forward_workspace_size",
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
-            "jmoe_profile_events", "jmoe_last_error", "jmoe_status_string")
+            "jmoe_profile_events", "jmoe_launch_count", "jmoe_last_error",
+            "jmoe_status_string")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
-STAGES = ("permute", "gather", "gate_up", "down", "combine")
+STAGES = ("permute", "gather", "gate_up", "down", "combine", "act")
 
 
 class JmoeError(RuntimeError):
@@ -72,6 +73,7 @@ def load() -> ctypes.CDLL:
     lib.jmoe_mlp_workspace_size.argtypes = [i64, i64, i64, i32, ctypes.POINTER(sz)]
     lib.jmoe_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i32, vp]
     lib.jmoe_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    lib.jmoe_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
     lib.jmoe_last_error.argtypes = []
     for name in EXPORTED[:-1]:
         getattr(lib, name).restype = st
@@ -267,12 +269,21 @@ def jmoe_mlp_forward(x, w_gu, s_gu, w_d, s_d, out=None, workspace=None, path=JMO
 
 
 def jmoe_profile_events(events) -> None:
-    """Register torch.cuda.Event objects (2 per stage, see jmoe.h) or None to stop."""
+    """Register torch.cuda.Event objects (2 per stage, see jmoe.h; None skips a
+    stage) or None to stop."""
     if not events:
         _check("jmoe_profile_events", load().jmoe_profile_events(None, 0))
         return
-    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event if ev is not None else None
+                                            for ev in events])
     _check("jmoe_profile_events", load().jmoe_profile_events(arr, len(events)))
+
+
+def jmoe_launch_count() -> int:
+    """Kernels launched by the library so far in this process (all devices)."""
+    n = ctypes.c_uint64(0)
+    _check("jmoe_launch_count", load().jmoe_launch_count(ctypes.byref(n)))
+    return int(n.value)
 
 
 def jmoe_last_error() -> int:

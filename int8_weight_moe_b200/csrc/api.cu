@@ -15,11 +15,12 @@ namespace {
 __device__ unsigned g_jmoe_err_word;
 
 constexpr int kMaxDevices = 64;
-constexpr int kStages = 5;
+constexpr int kStages = 6;
 cudaEvent_t g_stage_events[2 * kStages];
 std::atomic<bool> g_profile_on{false};
 std::atomic<unsigned*> g_err_ptr[kMaxDevices];
 std::atomic<int> g_num_sms[kMaxDevices];
+std::atomic<uint64_t> g_launches{0};
 
 // Below this many token->expert assignments the decode (GEMV-like) kernels
 // run; at and above it the tcgen05 grouped GEMM.
@@ -57,8 +58,10 @@ int num_sms() {
 }
 
 void stage_mark(int stage, bool after, cudaStream_t s) {
-    if (g_profile_on.load(std::memory_order_relaxed))
-        cudaEventRecord(g_stage_events[2 * stage + (after ? 1 : 0)], s);
+    if (g_profile_on.load(std::memory_order_relaxed)) {
+        cudaEvent_t ev = g_stage_events[2 * stage + (after ? 1 : 0)];
+        if (ev) cudaEventRecord(ev, s);
+    }
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -213,7 +216,15 @@ void* noalloc_scratch() {
 
 }  // namespace
 
+void jmoe::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 extern "C" {
+
+jmoe_status jmoe_launch_count(uint64_t* count) {
+    if (!count) return JMOE_EINVAL;
+    *count = g_launches.load(std::memory_order_relaxed);
+    return JMOE_OK;
+}
 
 const char* jmoe_status_string(jmoe_status s) {
     switch (s) {
@@ -383,10 +394,9 @@ jmoe_status jmoe_profile_events(void* const* events, int32_t n) {
         return JMOE_OK;
     }
     if (n != 2 * kStages) return JMOE_EINVAL;
-    for (int i = 0; i < n; ++i) {
-        if (!events[i]) return JMOE_EINVAL;
-        g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
-    }
+    for (int i = 0; i < n; i += 2)
+        if ((events[i] == nullptr) != (events[i + 1] == nullptr)) return JMOE_EINVAL;
+    for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_profile_on.store(true);
     return JMOE_OK;
 }

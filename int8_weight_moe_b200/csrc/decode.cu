@@ -574,6 +574,7 @@ cudaError_t launch_gemv(const GemvParams& p, int num_sms, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     k_gemv<MODE, NCH><<<gemv_grid<MODE, NCH>(num_sms), kWarpsPerBlock * 32, gemv_smem<MODE>(),
                         stream>>>(map, p);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -596,18 +597,23 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     k_prep_x16<<<(unsigned)a.T, 256, 0, stream>>>(static_cast<const uint16_t*>(a.x), a.d,
                                                   static_cast<uint16_t*>(a.x16), a.xexp, a.hmax,
                                                   a.top_k);
+    note_launch();
     if (a.mark) a.mark(1, true, stream);
     if (a.mark) a.mark(2, false, stream);
     cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
-    if (err == cudaSuccess)
+    if (a.mark) a.mark(2, true, stream);
+    if (a.mark) a.mark(5, false, stream);
+    if (err == cudaSuccess) {
         k_swiglu<<<grid_for(a.A * a.f, a.num_sms, 8), 256, 0, stream>>>(
             a.P_gu, a.split_gu, a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
             static_cast<uint16_t*>(a.Hb), a.hmax);
-    if (err == cudaSuccess)
+        note_launch();
         k_h16<<<grid_for(a.A * a.f / 2, a.num_sms, 8), 256, 0, stream>>>(
             static_cast<const uint16_t*>(a.Hb), a.f, a.offsets, a.E, a.hmax,
             static_cast<uint16_t*>(a.H));
-    if (a.mark) a.mark(2, true, stream);
+        note_launch();
+    }
+    if (a.mark) a.mark(5, true, stream);
     if (err != cudaSuccess) return err;
     p.w = a.wd;
     p.S = a.split_d;
@@ -637,6 +643,7 @@ cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int
                             const int32_t* ids, void* out, int num_sms, cudaStream_t stream) {
     k_finalize<<<grid_for(T * (d / 4), num_sms, 8), 256, 0, stream>>>(
         Y, T, d, top_k, E, ids, static_cast<uint16_t*>(out));
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -649,6 +656,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     k_combine<<<grid_for(a.T * (a.d / 4), a.num_sms, 8), 256, 0, stream>>>(
         a.P_d, a.split_d, a.A, a.T, a.d, a.top_k, a.E, a.ids, a.gates, a.inv, a.hmax, a.sd,
         static_cast<uint16_t*>(a.out));
+    note_launch();
     if (a.mark) a.mark(4, true, stream);
     return cudaGetLastError();
 }

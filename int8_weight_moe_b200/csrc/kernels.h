@@ -11,6 +11,10 @@ namespace jmoe {
 // box_rows x box_cols elements (false if the driver entry point is missing or
 // the encoder rejects the arguments).
 bool tensormap_available();
+
+// Counts one kernel launch (process-wide, all devices); every launch site in
+// the library calls it right after the launch.
+void note_launch();
 bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
                uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
                CUtensorMapSwizzle swizzle);

@@ -137,6 +137,7 @@ cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream) {
     int64_t blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
     k_fill_f32<<<(unsigned)blocks, 256, 0, stream>>>(p, v, n);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -144,6 +145,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_
                            int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,
                            cudaStream_t stream) {
     k_permute<<<1, kThreads, 0, stream>>>(ids, A, E, pad, offsets, padded_offsets, perm, inv, err);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -158,6 +160,7 @@ cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
     k_gather_rows<<<(unsigned)blocks, 256, 0, stream>>>((const uint16_t*)x_bf16, d, top_k, E,
                                                         offsets, padded_offsets, perm, max_rows,
                                                         (uint16_t*)x_perm);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -413,6 +413,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmPa
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     k_grouped_gemm<MODE><<<num_sms, kThreads, kSmemBytes, stream>>>(a, b, p);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -90,6 +90,7 @@ cudaError_t launch_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8
     if (rows == 0) return cudaSuccess;
     k_quantize_rows<<<(unsigned)rows, kThreads, 0, stream>>>((const uint16_t*)w_bf16, cols, q,
                                                              scales);
+    note_launch();
     return cudaGetLastError();
 }
 

@@ -154,12 +154,14 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
     if (T < (int64_t)num_sms * 8) {
         k_route_wide<<<(unsigned)T, kMaxE * 32, 0, stream>>>((const uint16_t*)x_bf16, d, w_router,
                                                              bias, E, top_k, ids, gates, logits);
+        note_launch();
     } else {
         int64_t blocks = (T + 3) / 4;
         const int64_t cap = (int64_t)num_sms * 16;
         if (blocks > cap) blocks = cap;
         k_route<4><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
             (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, ids, gates, logits);
+        note_launch();
     }
     return cudaGetLastError();
 }

@@ -108,3 +108,13 @@ def test_mlp_validation():
     assert lib.jmoe_mlp_forward(*no_x) == jm.JMOE_EINVAL
     small = list(args); small[10] = 8
     assert lib.jmoe_mlp_forward(*small) == jm.JMOE_EWORKSPACE
+
+
+def test_launch_counter_counts_nothing_for_rejected_calls():
+    lib = jm.load()
+    assert lib.jmoe_launch_count(None) == jm.JMOE_EINVAL
+    n0 = jm.jmoe_launch_count()
+    assert n0 >= 0
+    assert lib.jmoe_quantize(None, 4, 16, GOOD, GOOD, None) == jm.JMOE_EINVAL
+    assert lib.jmoe_permute(GOOD, 4, 2, 16, None, GOOD, GOOD, None) == jm.JMOE_EINVAL
+    assert jm.jmoe_launch_count() == n0

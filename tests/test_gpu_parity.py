@@ -305,3 +305,19 @@ def test_invalid_expert_id_sets_device_error_word():
     assert jm.jmoe_last_error() == jm.JMOE_EDEVICE
     assert jm.jmoe_last_error() == jm.JMOE_OK  # cleared by the read
     assert bool(torch.isfinite(out.float()).all())
+
+
+@pytest.mark.parametrize("path,expected", [(jm.JMOE_PATH_DECODE, 7), (jm.JMOE_PATH_PREFILL, 5)])
+def test_launch_counter_per_path(path, expected):
+    # decode: grouping, activation prep, gate/up GEMV, SwiGLU, fp16 rows,
+    # down GEMV, combine; tensor-core: grouping, row gather, two grouped GEMMs,
+    # finalize.  The router is one more launch.
+    dev = DeviceLayer(TINY)
+    ids, g = jm.jmoe_route(dev.x, dev.w_router, TINY.top_k, dev.bias)
+    n0 = jm.jmoe_launch_count()
+    jm.jmoe_route(dev.x, dev.w_router, TINY.top_k, dev.bias, topk_ids=ids, topk_w=g)
+    n1 = jm.jmoe_launch_count()
+    jm.jmoe_forward(dev.desc(path), dev.x, ids, g)
+    n2 = jm.jmoe_launch_count()
+    torch.cuda.synchronize()
+    assert (n1 - n0, n2 - n1) == (1, expected)

@@ -172,9 +172,9 @@ jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int
  *  - Size limit: if the scratch jmoe_forward_workspace_size would report for
  *    the decode kernels exceeds JMOE_NOALLOC_SCRATCH_BYTES, the call returns
  *    JMOE_EWORKSPACE before launching anything.  Roughly: the hidden
- *    activations take T*top_k * d_ff * 2 bytes and the split-K partial sums
- *    of the two projections up to 24 MB, or at least T*top_k * (2*d_ff +
- *    d_model) * 4 bytes (for example, 32 tokens at d_model 8192, d_ff 24576
+ *    activations take T*top_k * d_ff * 4 bytes (bf16 and fp16 copies) and
+ *    the split-K partial sums of the two projections, which share one
+ *    buffer, up to 16 MB (for example, 32 tokens at d_model 8192, d_ff 24576
  *    and top-2 fit; 64 tokens at those sizes do not).
  *  - The first call on a device looks up the array's device address for that
  *    device (with that device current) and caches it; make that first call
@@ -193,10 +193,11 @@ jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, 
 /* Stage timing hook (diagnostics).  Registers `n` CUDA events (cudaEvent_t
  * handles passed as void*) that the following jmoe_forward / jmoe_mlp_forward
  * calls record on their stream around their kernels: events[2*i] before and
- * events[2*i+1] after stage i, where the stages are 0 = grouping by expert,
- * 1 = row gather (tensor-core path) or activation preparation (decode path),
- * 2 = gate/up GEMM (with SwiGLU in its epilogue on the tensor-core path),
- * 3 = down GEMM, 4 = combine, 5 = SwiGLU and down-operand rows (decode path).
+ * events[2*i+1] after stage i, where the stages are 0 = grouping by expert
+ * (on the decode path together with the fp16 token rows), 1 = row gather
+ * (tensor-core path), 2 = gate/up GEMM (on the tensor-core path with SwiGLU
+ * in its epilogue), 3 = down GEMM, 4 = combine, 5 = SwiGLU and the fp16
+ * hidden rows (decode path).
  * Stages that do not run record nothing, and neither do stages whose two
  * entries are NULL (so a caller can time one stage without the cost of the
  * other records); one NULL entry of a pair is JMOE_EINVAL.  n = 0 or

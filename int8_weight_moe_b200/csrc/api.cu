@@ -73,7 +73,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the size query and the forward calls.
 struct Workspace {
     size_t offsets, padded_offsets, perm, inv;  // routing tables
-    size_t H, Hb, Pgu, Pd, x16, xexp, hmax;     // decode path
+    size_t H, Hb, P, x16, xexp, hmax;           // decode path
     int split_gu, split_d;
     size_t xperm, Hp, Yg;                       // tensor-core path
     size_t total;
@@ -94,7 +94,9 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     w.inv = take(sizeof(int32_t) * (size_t)A);
     if (!prefill) {
         // K pieces: about 16 work items per warp on a 148-SM GPU, with the
-        // partial-sum buffers capped at 16 MB (gate/up) and 8 MB (down).
+        // partial sums capped at 16 MB for gate/up and 8 MB for down.  The
+        // two GEMVs share one partial-sum buffer: the gate/up sums are used
+        // up (SwiGLU) before the down GEMV writes its own.
         const int64_t target = 148LL * 16 * 16;
         const int64_t touched = A < E ? A : E;
         const int64_t units_gu = touched * (f / 16), units_d = touched * (d / 16);
@@ -104,13 +106,14 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
                                         row_gu > 0 ? (16LL << 20) / row_gu : 1);
         w.split_d = jmoe::decode_split(f, units_d > 0 ? (target + units_d - 1) / units_d : 1,
                                        row_d > 0 ? (8LL << 20) / row_d : 1);
+        const size_t pgu = (size_t)w.split_gu * (size_t)row_gu;
+        const size_t pd = (size_t)w.split_d * (size_t)row_d;
         w.H = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
         w.Hb = take(sizeof(uint16_t) * (size_t)A * (size_t)f);
         w.x16 = take(sizeof(uint16_t) * (size_t)T * (size_t)d);
         w.xexp = take(sizeof(int32_t) * (size_t)T);
         w.hmax = take(sizeof(int32_t) * (size_t)A);
-        w.Pgu = take((size_t)w.split_gu * (size_t)row_gu);
-        w.Pd = take((size_t)w.split_d * (size_t)row_d);
+        w.P = take(pgu > pd ? pgu : pd);
     } else {
         const int64_t tm = jmoe::kPrefillTileM;
         w.rows_padded = (A + (int64_t)E * (tm - 1) + tm - 1) / tm * tm;
@@ -162,27 +165,28 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
     unsigned* err = err_word();
     const int sms = num_sms();
 
-    stage_mark(0, false, stream);
-    cudaError_t e = jmoe::launch_permute(ids, A, E, jmoe::kPrefillTileM, offsets, poff, perm, inv,
-                                         err, stream);
-    stage_mark(0, true, stream);
-    if (e != cudaSuccess) return JMOE_ECUDA;
     if (!prefill) {
+        // grouping happens inside the decode path's first kernel
         jmoe::DecodeArgs a{};
         a.x = x; a.T = T; a.A = A; a.d = d; a.f = f; a.E = E; a.top_k = k;
         a.wgu = desc->w_gu; a.sgu = desc->s_gu; a.wd = desc->w_d; a.sd = desc->s_d;
         a.ids = ids; a.gates = gates; a.offsets = offsets; a.perm = perm; a.inv = inv;
-        a.H = at(w.H); a.P_gu = static_cast<float*>(at(w.Pgu));
-        a.P_d = static_cast<float*>(at(w.Pd));
+        a.H = at(w.H); a.Hb = at(w.Hb);
+        a.P_gu = static_cast<float*>(at(w.P)); a.P_d = a.P_gu;
         a.split_gu = w.split_gu; a.split_d = w.split_d;
         a.x16 = at(w.x16); a.xexp = static_cast<int32_t*>(at(w.xexp));
-        a.Hb = at(w.Hb); a.hmax = static_cast<int32_t*>(at(w.hmax));
+        a.hmax = static_cast<int32_t*>(at(w.hmax));
         a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;
         a.err = err;
         return from_cuda(jmoe::launch_decode(a, stream));
     }
+    stage_mark(0, false, stream);
+    cudaError_t e = jmoe::launch_permute(ids, A, E, jmoe::kPrefillTileM, offsets, poff, perm, inv,
+                                         err, stream);
+    stage_mark(0, true, stream);
+    if (e != cudaSuccess) return JMOE_ECUDA;
     jmoe::PrefillArgs p{};
     p.x = x; p.T = T; p.A = A; p.d = d; p.f = f; p.E = E; p.top_k = k;
     p.wgu = desc->w_gu; p.sgu = desc->s_gu; p.wd = desc->w_d; p.sd = desc->s_d;

@@ -29,14 +29,18 @@
 // item is (touched expert, 16 output channels, one pass of up to 8*NCH
 // tokens, one K piece of S): a slab of 16 rows (gate/up: 16 gate + the same
 // 16 up rows) x K/S bytes.  Items are small (16-32 KB) and dealt round-robin
-// to all warps of the GPU, so the warps finish together; each warp keeps a
-// ring of kDepth 64-byte steps of weights -- and of the matching activation
-// fragments -- in shared memory, filled by cp.async three steps ahead of use
-// and across item boundaries (the bytes in flight live in shared memory, not
-// in registers), so there are no bubbles and no barriers at all.  An item
-// stores its raw fp32 partial sums; the small follow-up kernels add the S
-// pieces in a fixed order (deterministic) and apply scales, SwiGLU, gates:
-//   k_prep_x16 -> x16 (fp16, per-token shift)
+// to all warps of the GPU, the K pieces of a unit to neighbouring warps, so
+// the warps finish together and the rows being read at any moment are few
+// and shared by several warps (DRAM rows stay open for more of their bytes).
+// Each warp keeps a ring of 4 KB slots in its own shared memory, filled by
+// TMA two slots ahead of use and across item boundaries, with the matching
+// activation fragments loaded one slot ahead; there are no barriers.  An
+// item stores its raw fp32 partial sums; the small follow-up kernels add the
+// S pieces in a fixed order (deterministic) and apply scales, SwiGLU, gates.
+// (Finishing units inside the streaming warps instead -- a counter per unit,
+// the last piece's warp adding them -- measured much slower: every fence,
+// atomic and dependent read at an item's end stalls that warp's short ring.)
+//   k_dprep -> grouping by expert (one CTA) + x16 (fp16, per-token shift)
 //   k_gemv<gate/up> -> P_gu[S][slot][2f] -> k_swiglu -> Hb (bf16) + row maxima
 //                                         -> k_h16 -> H (fp16, per-slot shift)
 //   k_gemv<down>    -> P_d [S][slot][d]  -> k_combine -> out (bf16)
@@ -44,6 +48,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "permute.cuh"
 #include "sm100.cuh"
 
 namespace jmoe {
@@ -372,18 +377,26 @@ __device__ __forceinline__ int block_max_int(int v, int* red) {
     return m;
 }
 
+// Block T: the stable grouping of the assignments by expert (offsets, perm,
+// inv; invalid expert ids are left out and flagged).  Blocks t < T:
 // x16[t] = fp16(x[t] * 2^-xexp[t]).  A bf16 value has 8 significant bits, so
 // the scaled value is exactly representable in fp16 unless it falls below
 // fp16's normal range (2^-14, i.e. 2^28 times smaller than the row maximum).
-__global__ void __launch_bounds__(256)
-    k_prep_x16(const uint16_t* __restrict__ x, int64_t d, uint16_t* __restrict__ x16,
-               int32_t* __restrict__ xexp, int32_t* __restrict__ hmax, int top_k) {
-    __shared__ int red[8];
+__global__ void __launch_bounds__(kPermuteThreads)
+    k_dprep(const uint16_t* __restrict__ x, int64_t T, int64_t d, uint16_t* __restrict__ x16,
+            int32_t* __restrict__ xexp, int32_t* __restrict__ hmax, const int32_t* __restrict__ ids,
+            int E, int top_k, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+            int32_t* __restrict__ inv, unsigned* err) {
+    if (blockIdx.x == T) {
+        block_permute(ids, T * top_k, E, 1, offsets, nullptr, perm, inv, err);
+        return;
+    }
+    __shared__ int red[kPermuteThreads / 32];
     const int64_t t = blockIdx.x;
     if (threadIdx.x < top_k) hmax[t * top_k + threadIdx.x] = 0;  // for k_swiglu's maxima
     const uint16_t* xr = x + t * d;
     int m = 0;
-    for (int64_t k = threadIdx.x * 8; k < d; k += 256 * 8) {
+    for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8) {
         const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -392,7 +405,7 @@ __global__ void __launch_bounds__(256)
     const int sh = row_shift(block_max_int(m, red));
     if (threadIdx.x == 0) xexp[t] = sh;
     const float scale = ldexpf(1.0f, -sh);
-    for (int64_t k = threadIdx.x * 8; k < d; k += 256 * 8) {
+    for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8) {
         const uint4 v = *reinterpret_cast<const uint4*>(xr + k);
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
@@ -409,7 +422,7 @@ __global__ void __launch_bounds__(256)
 // h = bf16( silu(s_g * u_g) * (s_u * u_u) ), u = 2^xexp[token] * sum_z P
 // (pieces in order; the power-of-two factor undoes the fp16 staging of x
 // exactly).  h goes to Hb (bf16) and the largest exponent field of each slot
-// to hmax[slot] (zeroed by k_prep_x16).
+// to hmax[slot] (zeroed by k_dprep).
 __global__ void __launch_bounds__(256)
     k_swiglu(const float* __restrict__ P, int S, int64_t A, int64_t f, int E, int top_k,
              const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
@@ -593,12 +606,14 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.S = a.split_gu;
     p.b_src = static_cast<const uint16_t*>(a.x16);
     p.P = a.P_gu;
-    if (a.mark) a.mark(1, false, stream);
-    k_prep_x16<<<(unsigned)a.T, 256, 0, stream>>>(static_cast<const uint16_t*>(a.x), a.d,
-                                                  static_cast<uint16_t*>(a.x16), a.xexp, a.hmax,
-                                                  a.top_k);
+    if (a.mark) a.mark(0, false, stream);
+    k_dprep<<<(unsigned)(a.T + 1), kPermuteThreads, 0, stream>>>(
+        static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<uint16_t*>(a.x16), a.xexp,
+        a.hmax, a.ids, a.E, a.top_k, a.offsets, a.perm, a.inv, a.err);
     note_launch();
-    if (a.mark) a.mark(1, true, stream);
+    if (a.mark) a.mark(0, true, stream);
+    const cudaError_t prep = cudaGetLastError();
+    if (prep != cudaSuccess) return prep;
     if (a.mark) a.mark(2, false, stream);
     cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
     if (a.mark) a.mark(2, true, stream);

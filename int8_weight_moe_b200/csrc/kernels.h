@@ -57,16 +57,16 @@ struct DecodeArgs {
     const float* sd;      // [E][d]
     const int32_t* ids;   // [T][top_k]
     const float* gates;   // [T][top_k]
-    const int32_t* offsets;  // [E+1]
-    const int32_t* perm;     // [A]
-    const int32_t* inv;      // [A]
+    int32_t* offsets;     // [E+1] (workspace, written by the path)
+    int32_t* perm;        // [A]   (workspace)
+    int32_t* inv;         // [A]   (workspace)
     void* x16;            // fp16 [T][d]: x * 2^-xexp[t] (workspace)
     int32_t* xexp;        // [T] power-of-two shift of each token row (workspace)
     void* Hb;             // bf16 [A][f]: hidden activations, expert-grouped slot order
     void* H;              // fp16 [A][f]: Hb * 2^-shift(hmax[slot]) (workspace)
     int32_t* hmax;        // [A] largest exponent field of each hidden row (workspace)
     float* P_gu;          // fp32 [split_gu][A][2f] partial sums (workspace)
-    float* P_d;           // fp32 [split_d][A][d] partial sums (workspace)
+    float* P_d;           // fp32 [split_d][A][d] partial sums (workspace; may alias P_gu)
     int split_gu, split_d;   // K pieces of the two GEMVs
     int64_t max_per_expert;  // host-side bound used to size register tiles
     void* out;            // bf16 [T][d]

@@ -6,91 +6,22 @@
 // the expert computation; here routing is split into this bit-exact
 // counting sort and the expert GEMMs that consume its output.
 //
-// k_permute: one CTA of 1024 threads.
-//   pass 1: per-expert counts (shared-memory atomics; order-independent);
-//   scan:   offsets[e] = exclusive prefix; padded offsets (each count rounded
-//           up to the tensor-core path's row tile) for the gather;
-//   pass 2: the assignments are visited in ascending order, 1024 at a time;
-//           inside a warp, __match_any_sync groups lanes with the same expert
-//           and a popcount of the lower lanes gives the stable rank; per-warp
-//           counts are prefix-summed across the 32 warps.  perm and inv come
-//           out identical to a stable counting sort.
+// k_permute: one CTA of 1024 threads running the stable counting sort of
+// permute.cuh.
 #include "common.cuh"
 #include "kernels.h"
+#include "permute.cuh"
 
 namespace jmoe {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 16;
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPermuteThreads)
     k_permute(const int32_t* __restrict__ ids, int64_t A, int E, int pad, int32_t* __restrict__ offsets,
               int32_t* __restrict__ padded_offsets, int32_t* __restrict__ perm,
               int32_t* __restrict__ inv, unsigned* err) {
-    __shared__ int s_count[kMaxE];
-    __shared__ int s_cursor[kMaxE];
-    __shared__ int s_warp_count[kWarps][kMaxE];
-    __shared__ int s_warp_base[kWarps][kMaxE];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-
-    if (tid < kMaxE) s_count[tid] = 0;
-    __syncthreads();
-    bool bad = false;
-    for (int64_t a = tid; a < A; a += kThreads) {
-        const int e = ids[a];
-        if (e >= 0 && e < E)
-            atomicAdd(&s_count[e], 1);
-        else
-            bad = true;
-    }
-    if (bad) flag_error(err, kErrBadExpert);
-    __syncthreads();
-    if (tid == 0) {
-        int run = 0, prun = 0;
-        for (int e = 0; e < E; ++e) {
-            offsets[e] = run;
-            if (padded_offsets) padded_offsets[e] = prun;
-            s_cursor[e] = run;
-            run += s_count[e];
-            prun += (s_count[e] + pad - 1) / pad * pad;
-        }
-        offsets[E] = run;
-        if (padded_offsets) padded_offsets[E] = prun;
-    }
-    for (int i = tid; i < kWarps * kMaxE; i += kThreads) (&s_warp_count[0][0])[i] = 0;
-    __syncthreads();
-
-    for (int64_t base = 0; base < A; base += kThreads) {
-        const int64_t a = base + tid;
-        int e = a < A ? ids[a] : -1;
-        if (e < 0 || e >= E) e = -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        if (e >= 0 && rank == 0) s_warp_count[warp][e] = __popc(peers);
-        __syncthreads();
-        if (tid < E) {
-            int run = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                s_warp_base[w][tid] = run;
-                run += s_warp_count[w][tid];
-                s_warp_count[w][tid] = 0;
-            }
-            s_count[tid] = run;  // this chunk's total for expert tid
-        }
-        __syncthreads();
-        if (e >= 0) {
-            const int pos = s_cursor[e] + s_warp_base[warp][e] + rank;
-            perm[pos] = (int32_t)a;
-            if (inv) inv[a] = pos;
-        } else if (a < A && inv) {
-            inv[a] = -1;
-        }
-        __syncthreads();
-        if (tid < E) s_cursor[tid] += s_count[tid];
-        __syncthreads();
-    }
+    block_permute(ids, A, E, pad, offsets, padded_offsets, perm, inv, err);
 }
 
 // x_perm[padded_offsets[e] + r] = x[perm[offsets[e] + r] / top_k] for
@@ -144,7 +75,7 @@ cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream) {
 cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_t* offsets,
                            int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,
                            cudaStream_t stream) {
-    k_permute<<<1, kThreads, 0, stream>>>(ids, A, E, pad, offsets, padded_offsets, perm, inv, err);
+    k_permute<<<1, kPermuteThreads, 0, stream>>>(ids, A, E, pad, offsets, padded_offsets, perm, inv, err);
     note_launch();
     return cudaGetLastError();
 }

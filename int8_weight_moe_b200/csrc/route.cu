@@ -64,21 +64,58 @@ __device__ void select_topk(const float* l, int64_t t, int E, int top_k, int32_t
 }
 
 // Few tokens: one CTA of 16 warps per token, warp e computes expert e's
-// logit (same per-lane order and halving tree), loads deeply unrolled.
+// logit (same per-lane order and halving tree).  The token row is staged in
+// shared memory once; each warp streams its expert's router row through two
+// 4 KB shared-memory buffers with 16-byte cp.async copies (all copies of a
+// chunk in flight at once, the next chunk landing while this one is summed),
+// and lane j then reads its own k = j (mod 32) entries, conflict-free.
+constexpr int kChunk = 1024;  // router-row floats per chunk
+constexpr int kChunkSmem = 2 * kChunk * 4;  // per warp: two chunks
+constexpr size_t kWideMaxSmem = 200 * 1024;  // 128 KB of chunks + token rows up to d = 36864
+
+__device__ __forceinline__ void route_chunk_copy(float* dst, const float* src, int n, int lane) {
+    // n floats (a multiple of 64): n/4 copies of 16 bytes, spread over the lanes
+    for (int i = lane; i < n / 4; i += 32) cp_async_16(dst + 4 * i, src + 4 * i, 16);
+    cp_async_commit();
+}
+
 __global__ void __launch_bounds__(kMaxE * 32)
     k_route_wide(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
                  const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
                  float* __restrict__ gates, float* __restrict__ logits) {
+    extern __shared__ __align__(16) uint8_t route_smem[];
+    float* s_w = reinterpret_cast<float*>(route_smem);  // [16 warps][2][kChunk]
+    uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + kMaxE * kChunkSmem);  // [d]
     __shared__ float s_logit[kMaxE];
     const int lane = threadIdx.x & 31, e = threadIdx.x >> 5;
     const int64_t t = blockIdx.x;
+    const int nchunks = (int)((d + kChunk - 1) / kChunk);
+    float* buf = s_w + e * 2 * kChunk;
+    const float* w = wr + (int64_t)e * d;
+    if (e < E) route_chunk_copy(buf, w, (int)(d < kChunk ? d : (int64_t)kChunk), lane);
+    const uint16_t* xr = x + t * d;
+    for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
+        *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
+    __syncthreads();
     if (e < E) {
-        const uint16_t* xr = x + t * d;
-        const float* w = wr + (int64_t)e * d;
         double acc = 0.0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int64_t base = (int64_t)c * kChunk;
+            if (c + 1 < nchunks) {
+                route_chunk_copy(buf + ((c + 1) & 1) * kChunk, w + base + kChunk,
+                                 (int)(d - base - kChunk < kChunk ? d - base - kChunk : (int64_t)kChunk), lane);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncwarp();
+            const float* cw = buf + (c & 1) * kChunk;
+            const int n = (int)(d - base < kChunk ? d - base : (int64_t)kChunk);
 #pragma unroll 8
-        for (int64_t k = lane; k < d; k += 32)
-            acc = fma((double)bf16_bits_to_f32(__ldg(xr + k)), (double)__ldg(w + k), acc);
+            for (int k = lane; k < n; k += 32)
+                acc = fma((double)bf16_bits_to_f32(s_x[base + k]), (double)cw[k], acc);
+            __syncwarp();  // the buffer is refilled two chunks later
+        }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o);
         if (lane == 0) s_logit[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
@@ -151,9 +188,13 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
     if (T == 0) return cudaSuccess;
     // Few tokens: a 16-warp CTA per token (latency); many tokens: 4 tokens per
     // 4-warp CTA, which cuts the router-weight traffic fourfold.
-    if (T < (int64_t)num_sms * 8) {
-        k_route_wide<<<(unsigned)T, kMaxE * 32, 0, stream>>>((const uint16_t*)x_bf16, d, w_router,
-                                                             bias, E, top_k, ids, gates, logits);
+    const size_t smem = (size_t)kMaxE * kChunkSmem + (size_t)d * sizeof(uint16_t);
+    if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);
+        if (e != cudaSuccess) return e;
+        k_route_wide<<<(unsigned)T, kMaxE * 32, smem, stream>>>(
+            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, ids, gates, logits);
         note_launch();
     } else {
         int64_t blocks = (T + 3) / 4;

@@ -307,11 +307,11 @@ def test_invalid_expert_id_sets_device_error_word():
     assert bool(torch.isfinite(out.float()).all())
 
 
-@pytest.mark.parametrize("path,expected", [(jm.JMOE_PATH_DECODE, 7), (jm.JMOE_PATH_PREFILL, 5)])
+@pytest.mark.parametrize("path,expected", [(jm.JMOE_PATH_DECODE, 6), (jm.JMOE_PATH_PREFILL, 5)])
 def test_launch_counter_per_path(path, expected):
-    # decode: grouping, activation prep, gate/up GEMV, SwiGLU, fp16 rows,
-    # down GEMV, combine; tensor-core: grouping, row gather, two grouped GEMMs,
-    # finalize.  The router is one more launch.
+    # decode: grouping with fp16 token rows, gate/up GEMV, SwiGLU, fp16 hidden
+    # rows, down GEMV, combine; tensor-core: grouping, row gather, two grouped
+    # GEMMs, finalize.  The router is one more launch.
     dev = DeviceLayer(TINY)
     ids, g = jm.jmoe_route(dev.x, dev.w_router, TINY.top_k, dev.bias)
     n0 = jm.jmoe_launch_count()

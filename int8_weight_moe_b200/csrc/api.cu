@@ -93,18 +93,20 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     w.perm = take(sizeof(int32_t) * (size_t)A);
     w.inv = take(sizeof(int32_t) * (size_t)A);
     if (!prefill) {
-        // K pieces: about 16 work items per warp on a 148-SM GPU, with the
-        // partial sums capped at 16 MB for gate/up and 8 MB for down.  The
-        // two GEMVs share one partial-sum buffer: the gate/up sums are used
-        // up (SwiGLU) before the down GEMV writes its own.
-        const int64_t target = 148LL * 16 * 16;
+        // K pieces: about 16 work items per warp on a 148-SM GPU for gate/up
+        // and 2 for down (measured best: larger down items halve the per-item
+        // overhead and the partial sums the combine reads), with the partial
+        // sums capped at 16 MB for gate/up and 8 MB for down.  The two GEMVs
+        // share one partial-sum buffer: the gate/up sums are used up (SwiGLU)
+        // before the down GEMV writes its own.
+        const int64_t target_gu = 148LL * 16 * 16, target_d = 148LL * 16 * 2;
         const int64_t touched = A < E ? A : E;
         const int64_t units_gu = touched * (f / 16), units_d = touched * (d / 16);
         const int64_t row_gu = A * 2 * f * (int64_t)sizeof(float);
         const int64_t row_d = A * d * (int64_t)sizeof(float);
-        w.split_gu = jmoe::decode_split(d, units_gu > 0 ? (target + units_gu - 1) / units_gu : 1,
+        w.split_gu = jmoe::decode_split(d, units_gu > 0 ? (target_gu + units_gu - 1) / units_gu : 1,
                                         row_gu > 0 ? (16LL << 20) / row_gu : 1);
-        w.split_d = jmoe::decode_split(f, units_d > 0 ? (target + units_d - 1) / units_d : 1,
+        w.split_d = jmoe::decode_split(f, units_d > 0 ? (target_d + units_d - 1) / units_d : 1,
                                        row_d > 0 ? (8LL << 20) / row_d : 1);
         const size_t pgu = (size_t)w.split_gu * (size_t)row_gu;
         const size_t pd = (size_t)w.split_d * (size_t)row_d;

@@ -352,13 +352,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     }
 }
 
-// Expert of a grouped slot (offsets[e] <= slot < offsets[e+1]).
-__device__ __forceinline__ int expert_of_slot(const int* off, int E, int slot) {
-    int e = 0;
-    while (e + 1 < E && off[e + 1] <= slot) ++e;
-    return e;
-}
-
 // Power-of-two shift that puts the largest |value| of a row (biased fp32 /
 // bf16 exponent field emax) into [2^14, 2^15), inside fp16's normal range.
 __device__ __forceinline__ int row_shift(int emax) {
@@ -422,50 +415,58 @@ __global__ void __launch_bounds__(kPermuteThreads)
 // h = bf16( silu(s_g * u_g) * (s_u * u_u) ), u = 2^xexp[token] * sum_z P
 // (pieces in order; the power-of-two factor undoes the fp16 staging of x
 // exactly).  h goes to Hb (bf16) and the largest exponent field of each slot
-// to hmax[slot] (zeroed by k_dprep).
+// to hmax[slot] (zeroed by k_dprep).  Block (chunk, slot): the slot's expert
+// and shift are looked up once, each thread takes 4 consecutive channels
+// (16-byte loads of every piece), and one atomic per block publishes the
+// block's maximum.
+constexpr int kSwigluChunk = 1024;  // channels per block (256 threads x 4)
+
 __global__ void __launch_bounds__(256)
     k_swiglu(const float* __restrict__ P, int S, int64_t A, int64_t f, int E, int top_k,
              const int32_t* __restrict__ offsets, const int32_t* __restrict__ perm,
              const int32_t* __restrict__ xexp, const float* __restrict__ sgu,
              uint16_t* __restrict__ Hb, int32_t* __restrict__ hmax) {
-    __shared__ int s_off[kMaxE + 1];
-    if (threadIdx.x <= E) s_off[threadIdx.x] = offsets[threadIdx.x];
-    __syncthreads();
-    const int64_t total = (int64_t)s_off[E] * f;
-    const int lane = threadIdx.x & 31;
-    // warp-uniform loop (the warp-wide maximum below needs all 32 lanes)
-    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); v0 < total;
-         v0 += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t v = v0 + lane;
-        const bool live = v < total;
-        const int slot = live ? (int)(v / f) : (int)(v0 / f);
+    __shared__ int s_e;
+    __shared__ float s_sx;
+    __shared__ int red[8];
+    const int used = offsets[E];  // dropped assignments leave trailing slots unused
+    const int64_t n = (int64_t)blockIdx.x * kSwigluChunk + threadIdx.x * 4;
+    for (int slot = blockIdx.y; slot < used; slot += gridDim.y) {
+        if (threadIdx.x == 0) {
+            int e = 0;
+            while (e + 1 < E && offsets[e + 1] <= slot) ++e;
+            s_e = e;
+            s_sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
+        }
+        __syncthreads();
         int ex = 0;
-        if (live) {
-            const int64_t n = v % f;
-            const int e = expert_of_slot(s_off, E, slot);
-            const float sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
-            float vg = 0.f, vu = 0.f;
+        if (n < f) {
+            const float sx = s_sx;
+            float vg[4] = {0.f, 0.f, 0.f, 0.f}, vu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
             for (int z = 0; z < S; ++z) {
                 const float* row = P + ((int64_t)z * A + slot) * 2 * f;
-                vg += row[n];
-                vu += row[f + n];
+                const float4 g = __ldg(reinterpret_cast<const float4*>(row + n));
+                const float4 u = __ldg(reinterpret_cast<const float4*>(row + f + n));
+                vg[0] += g.x; vg[1] += g.y; vg[2] += g.z; vg[3] += g.w;
+                vu[0] += u.x; vu[1] += u.y; vu[2] += u.z; vu[3] += u.w;
             }
-            const float* sg = sgu + (int64_t)e * 2 * f;
-            const uint16_t hb = __bfloat16_as_ushort(
-                __float2bfloat16_rn(silu_f32(sg[n] * (vg * sx)) * (sg[f + n] * (vu * sx))));
-            Hb[(int64_t)slot * f + n] = hb;
-            ex = (hb >> 7) & 0xff;
-        }
-        // one atomic per warp when the warp covers a single slot
-        int m = ex;
+            const float* sg = sgu + (int64_t)s_e * 2 * f;
+            const float4 s0 = __ldg(reinterpret_cast<const float4*>(sg + n));
+            const float4 s1 = __ldg(reinterpret_cast<const float4*>(sg + f + n));
+            const float sgv[4] = {s0.x, s0.y, s0.z, s0.w}, suv[4] = {s1.x, s1.y, s1.z, s1.w};
+            uint16_t hb[4];
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const int slot0 = __shfl_sync(0xffffffffu, slot, 0);
-        if (__all_sync(0xffffffffu, slot == slot0)) {
-            if (lane == 0 && m > 0) atomicMax(&hmax[slot0], m);
-        } else if (ex > 0) {
-            atomicMax(&hmax[slot], ex);
+            for (int i = 0; i < 4; ++i) {
+                hb[i] = __bfloat16_as_ushort(__float2bfloat16_rn(
+                    silu_f32(sgv[i] * (vg[i] * sx)) * (suv[i] * (vu[i] * sx))));
+                ex = max(ex, (int)((hb[i] >> 7) & 0xff));
+            }
+            *reinterpret_cast<uint2*>(Hb + (int64_t)slot * f + n) =
+                make_uint2(hb[0] | ((uint32_t)hb[1] << 16), hb[2] | ((uint32_t)hb[3] << 16));
         }
+        const int m = block_max_int(ex, red);  // ends with a barrier: s_e, s_sx reusable
+        if (threadIdx.x == 0 && m > 0) atomicMax(&hmax[slot], m);
     }
 }
 
@@ -488,40 +489,59 @@ __global__ void __launch_bounds__(256)
 }
 
 // out[t][m] = bf16( sum_j g_tj * (s_d[e_j][m] * (2^hexp * sum_z P[z][inv[a]][m])) ),
-// a = t*top_k + j, hexp = row_shift(hmax[inv[a]]).
+// a = t*top_k + j, hexp = row_shift(hmax[inv[a]]).  Block (chunk, token): the
+// token's slots, experts, gates and shifts are looked up once; each thread
+// takes 4 consecutive channels (16-byte loads).
+constexpr int kCombineChunk = 1024;  // channels per block (256 threads x 4)
+constexpr int kMaxTopK = 2;
+
 __global__ void __launch_bounds__(256)
     k_combine(const float* __restrict__ P, int S, int64_t A, int64_t T, int64_t d, int top_k,
               int E, const int32_t* __restrict__ ids, const float* __restrict__ gates,
               const int32_t* __restrict__ inv, const int32_t* __restrict__ hmax,
               const float* __restrict__ sd, uint16_t* __restrict__ out) {
-    const int64_t nvec = d / 4;
-    const int64_t total = T * nvec;
-    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
-         v += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = v / nvec, m = (v % nvec) * 4;
-        float o[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < top_k; ++j) {
-            const int64_t a = t * top_k + j;
+    __shared__ int s_slot[kMaxTopK], s_e[kMaxTopK];
+    __shared__ float s_gw[kMaxTopK], s_hs[kMaxTopK];
+    const int64_t m = (int64_t)blockIdx.x * kCombineChunk + threadIdx.x * 4;
+    for (int64_t t = blockIdx.y; t < T; t += gridDim.y) {
+        if (threadIdx.x < top_k) {
+            const int64_t a = t * top_k + threadIdx.x;
             const int e = ids[a];
             const int slot = inv[a];
-            if (e < 0 || e >= E || slot < 0) continue;
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int z = 0; z < S; ++z) {
-                const float4 q = *reinterpret_cast<const float4*>(P + ((int64_t)z * A + slot) * d + m);
-                y[0] += q.x; y[1] += q.y; y[2] += q.z; y[3] += q.w;
-            }
-            const float hs = ldexpf(1.0f, row_shift(hmax[slot]));
-            const float4 s = *reinterpret_cast<const float4*>(sd + (int64_t)e * d + m);
-            const float gw = gates[a];
-            o[0] += gw * (s.x * (y[0] * hs));
-            o[1] += gw * (s.y * (y[1] * hs));
-            o[2] += gw * (s.z * (y[2] * hs));
-            o[3] += gw * (s.w * (y[3] * hs));
+            const bool ok = e >= 0 && e < E && slot >= 0;
+            s_slot[threadIdx.x] = ok ? slot : -1;
+            s_e[threadIdx.x] = ok ? e : 0;
+            s_gw[threadIdx.x] = gates[a];
+            s_hs[threadIdx.x] = ok ? ldexpf(1.0f, row_shift(hmax[slot])) : 0.0f;
         }
-        uint2 r;
-        r.x = pack_bf16x2(o[0], o[1]);
-        r.y = pack_bf16x2(o[2], o[3]);
-        *reinterpret_cast<uint2*>(out + t * d + m) = r;
+        __syncthreads();
+        if (m < d) {
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < top_k; ++j) {
+                const int slot = s_slot[j];
+                if (slot < 0) continue;
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int z = 0; z < S; ++z) {
+                    const float4 q = __ldg(
+                        reinterpret_cast<const float4*>(P + ((int64_t)z * A + slot) * d + m));
+                    y[0] += q.x; y[1] += q.y; y[2] += q.z; y[3] += q.w;
+                }
+                const float hs = s_hs[j];
+                const float4 sv =
+                    __ldg(reinterpret_cast<const float4*>(sd + (int64_t)s_e[j] * d + m));
+                const float gw = s_gw[j];
+                o[0] += gw * (sv.x * (y[0] * hs));
+                o[1] += gw * (sv.y * (y[1] * hs));
+                o[2] += gw * (sv.z * (y[2] * hs));
+                o[3] += gw * (sv.w * (y[3] * hs));
+            }
+            uint2 r;
+            r.x = pack_bf16x2(o[0], o[1]);
+            r.y = pack_bf16x2(o[2], o[3]);
+            *reinterpret_cast<uint2*>(out + t * d + m) = r;
+        }
+        __syncthreads();  // the next token's lookups overwrite the shared values
     }
 }
 
@@ -619,7 +639,9 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     if (a.mark) a.mark(2, true, stream);
     if (a.mark) a.mark(5, false, stream);
     if (err == cudaSuccess) {
-        k_swiglu<<<grid_for(a.A * a.f, a.num_sms, 8), 256, 0, stream>>>(
+        k_swiglu<<<dim3((unsigned)((a.f + kSwigluChunk - 1) / kSwigluChunk),
+                        (unsigned)(a.A < 65535 ? a.A : 65535)),
+                   256, 0, stream>>>(
             a.P_gu, a.split_gu, a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
             static_cast<uint16_t*>(a.Hb), a.hmax);
         note_launch();
@@ -668,7 +690,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
                                             : launch_decode_nch<2>(a, stream);
     if (err != cudaSuccess) return err;
     if (a.mark) a.mark(4, false, stream);
-    k_combine<<<grid_for(a.T * (a.d / 4), a.num_sms, 8), 256, 0, stream>>>(
+    k_combine<<<dim3((unsigned)((a.d + kCombineChunk - 1) / kCombineChunk),
+                     (unsigned)(a.T < 65535 ? a.T : 65535)),
+                256, 0, stream>>>(
         a.P_d, a.split_d, a.A, a.T, a.d, a.top_k, a.E, a.ids, a.gates, a.inv, a.hmax, a.sd,
         static_cast<uint16_t*>(a.out));
     note_launch();

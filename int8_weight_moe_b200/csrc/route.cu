@@ -17,9 +17,13 @@
 // Work split: for many tokens a CTA of 4 warps handles kTok tokens; warp w
 // owns experts w, w+4, w+8, w+12, so each lane keeps 4 x kTok independent
 // fp64 accumulators and every router weight it loads serves kTok tokens.
-// For few tokens (decode) a 16-warp CTA takes one token, one expert per warp.
-// The k loops are unrolled so the loads of several steps are in flight
-// together.  Softmax (fp32) and top-k run in one thread per token afterwards.
+// For few tokens (decode) one warp per expert: a cluster of 4 CTAs per token
+// (each warp's router row copied to shared memory in one round trip, logits
+// gathered in the first CTA through distributed shared memory), or for rows
+// too wide for that a 16-warp CTA per token streaming the rows in chunks.
+// Softmax (fp32) and top-k run in one thread per token afterwards.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -124,6 +128,57 @@ __global__ void __launch_bounds__(kMaxE * 32)
     if (threadIdx.x == 0) select_topk(s_logit, t, E, top_k, ids, gates, logits);
 }
 
+// Few tokens, d_model up to about 11k: a cluster of 4 CTAs per token, 4
+// warps per CTA, warp w of CTA r computing expert 4r + w.  Each warp pulls its
+// whole router row into shared memory with 16-byte cp.async copies at once
+// (one memory round trip), sums in the canonical order, and writes its logit
+// into the first CTA's shared memory (distributed shared memory); after the
+// cluster barrier the first CTA selects the top-k.
+constexpr int kRouteCluster = 4;
+constexpr int kExpertsPerCta = kMaxE / kRouteCluster;
+constexpr size_t kClusterMaxSmem = 200 * 1024;
+
+__global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExpertsPerCta * 32)
+    k_route_cluster(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
+                    const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
+                    float* __restrict__ gates, float* __restrict__ logits) {
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(16) uint8_t route_smem[];
+    float* s_w = reinterpret_cast<float*>(route_smem);  // [kExpertsPerCta][d]
+    uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + (size_t)kExpertsPerCta * d * 4);
+    __shared__ float s_logit[kMaxE];  // filled in the cluster's first CTA
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = (int)rank * kExpertsPerCta + warp;
+    const int64_t t = blockIdx.x / kRouteCluster;
+    float* row = s_w + (size_t)warp * d;
+    if (e < E) {
+        const float* w = wr + (int64_t)e * d;
+        for (int64_t i = lane; i < d / 4; i += 32) cp_async_16(row + 4 * i, w + 4 * i, 16);
+    }
+    cp_async_commit();
+    const uint16_t* xr = x + t * d;
+    for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
+        *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
+    cp_async_wait<0>();
+    __syncthreads();
+    if (e < E) {
+        double acc = 0.0;
+#pragma unroll 8
+        for (int64_t k = lane; k < d; k += 32)
+            acc = fma((double)bf16_bits_to_f32(s_x[k]), (double)row[k], acc);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            float* dst = cluster.map_shared_rank(s_logit, 0);
+            dst[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
+        }
+    }
+    cluster.sync();
+    if (rank == 0 && threadIdx.x == 0) select_topk(s_logit, t, E, top_k, ids, gates, logits);
+}
+
 template <int kTok>
 __global__ void __launch_bounds__(kWarps * 32)
     k_route(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
@@ -186,10 +241,19 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
                          const float* bias, int E, int top_k, int32_t* ids, float* gates,
                          float* logits, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    // Few tokens: a 16-warp CTA per token (latency); many tokens: 4 tokens per
-    // 4-warp CTA, which cuts the router-weight traffic fourfold.
+    // Few tokens: a cluster of 4 CTAs per token (or, for very wide rows, a
+    // 16-warp CTA streaming the router rows in chunks); many tokens: 4 tokens
+    // per 4-warp CTA, which cuts the router-weight traffic fourfold.
+    const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
     const size_t smem = (size_t)kMaxE * kChunkSmem + (size_t)d * sizeof(uint16_t);
-    if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
+    if (T < (int64_t)num_sms * 8 && csmem <= kClusterMaxSmem && T * kRouteCluster < (1LL << 31)) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
+        if (e != cudaSuccess) return e;
+        k_route_cluster<<<(unsigned)(T * kRouteCluster), kExpertsPerCta * 32, csmem, stream>>>(
+            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, ids, gates, logits);
+        note_launch();
+    } else if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);
         if (e != cudaSuccess) return e;

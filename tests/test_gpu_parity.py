@@ -104,6 +104,19 @@ def test_route_bitexact(wl):
         assert 0.33 <= frac <= 0.47, frac
 
 
+@pytest.mark.parametrize("T,d,E", [(3, 12288, 16), (5, 16384, 12)])
+def test_route_wide_rows_bitexact(T, d, E):
+    # rows too wide for the per-token cluster kernel take the chunked one
+    wl = Workload("route_wide", 13, T, d, 64, E=E)
+    dev = DeviceLayer(wl)
+    ora = OracleLayer(wl)
+    ids, g, logits = jm.jmoe_route(dev.x, dev.w_router, wl.top_k, dev.bias, want_logits=True)
+    lo, io, go = ora.route()
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert np.abs(g.cpu().numpy().astype(np.float64) - go).max() <= 1e-6
+
+
 def test_route_top1_and_ties():
     d, E = 256, 16
     x = synth.normal_bf16_gpu(3, synth.X, 1.0, (40, d))

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "kernels.h"
 
 namespace jmoe {
@@ -130,5 +132,51 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&r);
 }
+
+// Programmatic dependent launch.  pdl_wait: block until the preceding kernel
+// on the stream (launched before this one with the programmatic-serialisation
+// attribute set on this launch) has completed and its writes are visible; a
+// no-op when this kernel was launched without that attribute.
+// pdl_launch_dependents: let the next such kernel start launching once every
+// CTA of this grid has executed it (or exited), so its launch overlaps this
+// kernel's tail; it grants no access to this kernel's results.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel on the stream is still finishing; every kernel
+// launched this way calls pdl_wait() before it reads anything the previous
+// kernels wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    note_launch();
+    return e;
+}
+
+struct GemvParams {
+    int E, top_k, S;           // experts, experts per token, K pieces
+    int64_t d, f;
+    const int8_t* w;           // gate/up [E][2f][d] or down [E][d][f]
+    const int32_t* offsets;    // [E+1]
+    const int32_t* perm;       // [A]
+    const uint16_t* b_src;     // x [T][d] (gate/up) or H [A][f] (down)
+    float* P;                  // partial sums [S][A][cols]
+    int64_t A;
+    unsigned* err;
+};
 
 }  // namespace jmoe

@@ -59,18 +59,6 @@ constexpr int kMaxE = 16;
 
 enum { kGateUp = 0, kDown = 1 };
 
-struct GemvParams {
-    int E, top_k, S;           // experts, experts per token, K pieces
-    int64_t d, f;
-    const int8_t* w;           // gate/up [E][2f][d] or down [E][d][f]
-    const int32_t* offsets;    // [E+1]
-    const int32_t* perm;       // [A]
-    const uint16_t* b_src;     // x [T][d] (gate/up) or H [A][f] (down)
-    float* P;                  // partial sums [S][A][cols]
-    int64_t A;
-    unsigned* err;
-};
-
 // x (or h) fragment for one token row: 16 consecutive bf16 starting at p.
 __device__ __forceinline__ void load_b(const uint16_t* p, uint32_t (&b)[8]) {
     if (p) {
@@ -150,6 +138,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     __shared__ int s_start[kMaxE + 1];  // first item of expert e
     __shared__ int s_off[kMaxE + 1];
     __shared__ int s_abort;
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, c = lane & 3;
     uint8_t* ring = smem_raw + warp * kSlots * kSlotBytes;
     const int E = p.E, S = p.S;
@@ -380,6 +370,8 @@ __global__ void __launch_bounds__(kPermuteThreads)
             int32_t* __restrict__ xexp, int32_t* __restrict__ hmax, const int32_t* __restrict__ ids,
             int E, int top_k, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
             int32_t* __restrict__ inv, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     if (blockIdx.x == T) {
         block_permute(ids, T * top_k, E, 1, offsets, nullptr, perm, inv, err);
         return;
@@ -429,6 +421,8 @@ __global__ void __launch_bounds__(256)
     __shared__ int s_e;
     __shared__ float s_sx;
     __shared__ int red[8];
+    pdl_wait();
+    pdl_launch_dependents();
     const int used = offsets[E];  // dropped assignments leave trailing slots unused
     const int64_t n = (int64_t)blockIdx.x * kSwigluChunk + threadIdx.x * 4;
     for (int slot = blockIdx.y; slot < used; slot += gridDim.y) {
@@ -476,6 +470,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     k_h16(const uint16_t* __restrict__ Hb, int64_t f, const int32_t* __restrict__ offsets, int E,
           const int32_t* __restrict__ hmax, uint16_t* __restrict__ H16) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t total = (int64_t)offsets[E] * f / 2;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
          v += (int64_t)gridDim.x * blockDim.x) {
@@ -502,6 +498,8 @@ __global__ void __launch_bounds__(256)
               const float* __restrict__ sd, uint16_t* __restrict__ out) {
     __shared__ int s_slot[kMaxTopK], s_e[kMaxTopK];
     __shared__ float s_gw[kMaxTopK], s_hs[kMaxTopK];
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t m = (int64_t)blockIdx.x * kCombineChunk + threadIdx.x * 4;
     for (int64_t t = blockIdx.y; t < T; t += gridDim.y) {
         if (threadIdx.x < top_k) {
@@ -605,10 +603,8 @@ cudaError_t launch_gemv(const GemvParams& p, int num_sms, cudaStream_t stream) {
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            gemv_smem<MODE>());
     if (err != cudaSuccess) return err;
-    k_gemv<MODE, NCH><<<gemv_grid<MODE, NCH>(num_sms), kWarpsPerBlock * 32, gemv_smem<MODE>(),
-                        stream>>>(map, p);
-    note_launch();
-    return cudaGetLastError();
+    return launch_pdl(k_gemv<MODE, NCH>, dim3(gemv_grid<MODE, NCH>(num_sms)),
+                      dim3(kWarpsPerBlock * 32), gemv_smem<MODE>(), stream, map, p);
 }
 
 template <int NCH>
@@ -627,28 +623,27 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.b_src = static_cast<const uint16_t*>(a.x16);
     p.P = a.P_gu;
     if (a.mark) a.mark(0, false, stream);
-    k_dprep<<<(unsigned)(a.T + 1), kPermuteThreads, 0, stream>>>(
+    const cudaError_t prep = launch_pdl(
+        k_dprep, dim3((unsigned)(a.T + 1)), dim3(kPermuteThreads), 0, stream,
         static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<uint16_t*>(a.x16), a.xexp,
         a.hmax, a.ids, a.E, a.top_k, a.offsets, a.perm, a.inv, a.err);
-    note_launch();
     if (a.mark) a.mark(0, true, stream);
-    const cudaError_t prep = cudaGetLastError();
     if (prep != cudaSuccess) return prep;
     if (a.mark) a.mark(2, false, stream);
     cudaError_t err = launch_gemv<kGateUp, NCH>(p, a.num_sms, stream);
     if (a.mark) a.mark(2, true, stream);
     if (a.mark) a.mark(5, false, stream);
     if (err == cudaSuccess) {
-        k_swiglu<<<dim3((unsigned)((a.f + kSwigluChunk - 1) / kSwigluChunk),
-                        (unsigned)(a.A < 65535 ? a.A : 65535)),
-                   256, 0, stream>>>(
-            a.P_gu, a.split_gu, a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
-            static_cast<uint16_t*>(a.Hb), a.hmax);
-        note_launch();
-        k_h16<<<grid_for(a.A * a.f / 2, a.num_sms, 8), 256, 0, stream>>>(
-            static_cast<const uint16_t*>(a.Hb), a.f, a.offsets, a.E, a.hmax,
-            static_cast<uint16_t*>(a.H));
-        note_launch();
+        err = launch_pdl(k_swiglu,
+                         dim3((unsigned)((a.f + kSwigluChunk - 1) / kSwigluChunk),
+                              (unsigned)(a.A < 65535 ? a.A : 65535)),
+                         dim3(256), 0, stream, static_cast<const float*>(a.P_gu), a.split_gu,
+                         a.A, a.f, a.E, a.top_k, a.offsets, a.perm, a.xexp, a.sgu,
+                         static_cast<uint16_t*>(a.Hb), a.hmax);
+        if (err == cudaSuccess)
+            err = launch_pdl(k_h16, dim3(grid_for(a.A * a.f / 2, a.num_sms, 8)), dim3(256), 0,
+                             stream, static_cast<const uint16_t*>(a.Hb), a.f, a.offsets, a.E,
+                             a.hmax, static_cast<uint16_t*>(a.H));
     }
     if (a.mark) a.mark(5, true, stream);
     if (err != cudaSuccess) return err;
@@ -690,14 +685,14 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
                                             : launch_decode_nch<2>(a, stream);
     if (err != cudaSuccess) return err;
     if (a.mark) a.mark(4, false, stream);
-    k_combine<<<dim3((unsigned)((a.d + kCombineChunk - 1) / kCombineChunk),
-                     (unsigned)(a.T < 65535 ? a.T : 65535)),
-                256, 0, stream>>>(
-        a.P_d, a.split_d, a.A, a.T, a.d, a.top_k, a.E, a.ids, a.gates, a.inv, a.hmax, a.sd,
-        static_cast<uint16_t*>(a.out));
-    note_launch();
+    err = launch_pdl(k_combine,
+                     dim3((unsigned)((a.d + kCombineChunk - 1) / kCombineChunk),
+                          (unsigned)(a.T < 65535 ? a.T : 65535)),
+                     dim3(256), 0, stream, static_cast<const float*>(a.P_d), a.split_d, a.A, a.T,
+                     a.d, a.top_k, a.E, a.ids, a.gates, static_cast<const int32_t*>(a.inv),
+                     static_cast<const int32_t*>(a.hmax), a.sd, static_cast<uint16_t*>(a.out));
     if (a.mark) a.mark(4, true, stream);
-    return cudaGetLastError();
+    return err;
 }
 
 }  // namespace jmoe

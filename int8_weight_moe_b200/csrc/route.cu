@@ -148,6 +148,8 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
     uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + (size_t)kExpertsPerCta * d * 4);
     __shared__ float s_logit[kMaxE];  // filled in the cluster's first CTA
     cg::cluster_group cluster = cg::this_cluster();
+    pdl_wait();  // the previous step may still read ids and gates
+    pdl_launch_dependents();
     const unsigned rank = cluster.block_rank();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = (int)rank * kExpertsPerCta + warp;
@@ -250,9 +252,9 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
         if (e != cudaSuccess) return e;
-        k_route_cluster<<<(unsigned)(T * kRouteCluster), kExpertsPerCta * 32, csmem, stream>>>(
-            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, ids, gates, logits);
-        note_launch();
+        return launch_pdl(k_route_cluster, dim3((unsigned)(T * kRouteCluster)),
+                          dim3(kExpertsPerCta * 32), csmem, stream, (const uint16_t*)x_bf16, d,
+                          w_router, bias, E, top_k, ids, gates, logits);
     } else if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);

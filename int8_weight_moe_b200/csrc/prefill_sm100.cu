@@ -12,13 +12,19 @@
 // (sum_k x_k (q_k s) = s sum_k x_k q_k).  Activations stay BF16 (step 4);
 // accumulation is fp32 in TMEM.
 //
-// One CTA per SM, 15 warps:
+// One CTA per SM, 16 warps:
 //   warp 0      TMA producer of the activation tile A [256 rows x 64 k] bf16
 //               (two 128-row boxes; the second is skipped when the expert ends)
-//   warp 1      TMEM allocator and MMA issuer (one thread)
+//   warp 1      TMEM allocator and MMA issuer of the first 128-row half
 //   warp 2      TMA producer of the INT8 weight tile [128 rows x 64 k]
 //   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled)
 //   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
+//   warp 15     MMA issuer of the second 128-row half
+// Two issuing threads, one per half (each with its own accumulator, so the
+// order of every accumulation stays fixed): a thread that waits on an
+// mbarrier stops issuing until the MMAs it already queued have been
+// dispatched, and the tensor pipe would idle through every such wait if one
+// thread issued everything; with two, the other thread's MMAs fill it.
 // Rings: A + converted B share 3 stages (48 KB each); the INT8 tiles, which
 // come from HBM, have 8 stages (8 KB each) to cover its latency.  Each weight tile, once converted, feeds two M = 128
 // MMAs (256 token rows), which halves the conversion work per multiply-add
@@ -63,7 +69,9 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(BH, BN);
 constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
 constexpr int kConvWarp0 = 3, kConvWarps = 8;
 constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps, kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+constexpr int kWarpMMA2 = kEpiWarp0 + kEpiWarps;
+constexpr int kThreads = (kWarpMMA2 + 1) * 32;
+constexpr int kIssuers = 2;  // MMA-issuing threads (one per 128-row half)
 constexpr int kMaxE = 16;
 
 enum Mode { kGateUp = 0, kDown = 1 };
@@ -86,7 +94,7 @@ struct GemmParams {
 };
 
 struct Shared {
-    uint64_t ab_full_a[kStagesAB], ab_full_b[kStagesAB], ab_empty[kStagesAB];
+    uint64_t ab_full[kStagesAB], ab_empty[kStagesAB];
     uint64_t b8_full[kStages8], b8_empty[kStages8];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t drain;
@@ -149,19 +157,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesAB; ++i) {
-            mbar_init(&S.ab_full_a[i], 1);
-            mbar_init(&S.ab_full_b[i], kConvWarps);
-            mbar_init(&S.ab_empty[i], 1);
+            // the A producer's expect-tx arrival (plus the TMA bytes) and the
+            // converter warps' arrivals
+            mbar_init(&S.ab_full[i], 1 + kConvWarps);
+            mbar_init(&S.ab_empty[i], kIssuers);
         }
         for (int i = 0; i < kStages8; ++i) {
             mbar_init(&S.b8_full[i], 1);
             mbar_init(&S.b8_empty[i], kConvWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_full[i], kIssuers);
             mbar_init(&S.acc_empty[i], kEpiWarps);
         }
-        mbar_init(&S.drain, 1);
+        mbar_init(&S.drain, kIssuers);
         S.abort = 0;
         fence_mbar_init();
     }
@@ -202,16 +211,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int s = g % kStagesAB;
                     const uint32_t ph = (g / kStagesAB) & 1;
                     if (!mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) break;
-                    mbar_arrive_expect_tx(&S.ab_full_a[s], t.halves * kHalfBytes);
-                    tma_load_2d(tileA(s), &tmA, &S.ab_full_a[s], kb * BK, t.row0);
+                    mbar_arrive_expect_tx(&S.ab_full[s], t.halves * kHalfBytes);
+                    tma_load_2d(tileA(s), &tmA, &S.ab_full[s], kb * BK, t.row0);
                     if (t.halves == 2)
-                        tma_load_2d(tileA(s) + kHalfBytes, &tmA, &S.ab_full_a[s], kb * BK,
+                        tma_load_2d(tileA(s) + kHalfBytes, &tmA, &S.ab_full[s], kb * BK,
                                     t.row0 + BH);
                 }
             }
             // make sure no copy is still landing in shared memory when the CTA exits
             for (uint32_t h = (g > (uint32_t)kStagesAB ? g - kStagesAB : 0); h < g; ++h)
-                wait_drain(&S.ab_full_a[h % kStagesAB], (h / kStagesAB) & 1);
+                wait_drain(&S.ab_full[h % kStagesAB], (h / kStagesAB) & 1);
         }
     } else if (warp == kWarpProdB) {
         if (lane == 0) {
@@ -237,32 +246,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (uint32_t h = (g > (uint32_t)kStages8 ? g - kStages8 : 0); h < g; ++h)
                 wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1);
         }
-    } else if (warp == kWarpMMA) {
+    } else if (warp == kWarpMMA || warp == kWarpMMA2) {
         if (lane == 0) {
+            const int h = warp == kWarpMMA ? 0 : 1;  // the 128-row half this thread issues
             uint32_t g = 0;
             int it = 0;
             for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
-                const int t_halves = decode_tile(S, E, p.n_tiles, tile).halves;
+                const bool active = h < decode_tile(S, E, p.n_tiles, tile).halves;
                 const int buf = it & 1;
                 if (!mbar_wait(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * 2 * BN;
+                const uint32_t d_tmem = tmem + buf * 2 * BN + h * BN;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStagesAB;
                     const uint32_t ph = (g / kStagesAB) & 1;
-                    if (!mbar_wait(&S.ab_full_a[s], ph, abort) ||
-                        !mbar_wait(&S.ab_full_b[s], ph, abort)) {
+                    if (!mbar_wait(&S.ab_full[s], ph, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(tileA(s)), b0 = smem_u32(tileBbf(s));
-                    for (int h = 0; h < t_halves; ++h) {
+                    if (active) {
+                        const uint32_t a0 = smem_u32(tileA(s)) + h * kHalfBytes;
+                        const uint32_t b0 = smem_u32(tileBbf(s));
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_bf16_ss(d_tmem + h * BN, desc_sw128(a0 + h * kHalfBytes + kk * 32),
-                                        desc_sw128(b0 + kk * 32), kIdesc, (kb | kk) != 0);
+                            mma_bf16_ss(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
+                                        kIdesc, (kb | kk) != 0);
                     }
                     mma_commit(&S.ab_empty[s]);
                 }
@@ -305,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&S.ab_full_b[s]);
+                    mbar_arrive(&S.ab_full[s]);
                     mbar_arrive(&S.b8_empty[s8]);
                 }
             }

@@ -283,8 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             wait_drain(&S.drain, 0);
         }
     } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
+        // Thread ct converts the 16-byte int8 chunks q = ct and ct + 256 of the
+        // tile (row q / 4, bytes 16 (q % 4) .. +16): both loads are issued
+        // before any conversion, and each chunk becomes two 16-byte bf16 units
+        // 2 (q % 4) and 2 (q % 4) + 1 of the row's 128-byte swizzled line.
         const int ct = threadIdx.x - kConvWarp0 * 32;  // 0..255
-        const int chunk = ct & 7;
         uint32_t g = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok && !*abort; tile += gridDim.x) {
@@ -300,17 +303,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint8_t* src = tileB8(s8);
                 uint8_t* dst = tileBbf(s);
+                uint4 v[2];
 #pragma unroll
-                for (int j = 0; j < BN / 32; ++j) {
-                    const int row = (ct >> 3) + 32 * j;
-                    const uint2 v = *reinterpret_cast<const uint2*>(src + row * BK + chunk * 8);
-                    uint4 o;
-                    o.x = i8x2_to_bf16x2<0>(v.x);
-                    o.y = i8x2_to_bf16x2<1>(v.x);
-                    o.z = i8x2_to_bf16x2<0>(v.y);
-                    o.w = i8x2_to_bf16x2<1>(v.y);
-                    *reinterpret_cast<uint4*>(dst + (row >> 3) * 1024 + (row & 7) * 128 +
-                                              ((chunk ^ (row & 7)) << 4)) = o;
+                for (int j = 0; j < 2; ++j)
+                    v[j] = *reinterpret_cast<const uint4*>(src + (ct + 256 * j) * 16);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int q = ct + 256 * j, row = q >> 2, u0 = 2 * (q & 3);
+                    uint8_t* line = dst + (row >> 3) * 1024 + (row & 7) * 128;
+                    const uint4 o0 = make_uint4(i8x2_to_bf16x2<0>(v[j].x), i8x2_to_bf16x2<1>(v[j].x),
+                                                i8x2_to_bf16x2<0>(v[j].y), i8x2_to_bf16x2<1>(v[j].y));
+                    const uint4 o1 = make_uint4(i8x2_to_bf16x2<0>(v[j].z), i8x2_to_bf16x2<1>(v[j].z),
+                                                i8x2_to_bf16x2<0>(v[j].w), i8x2_to_bf16x2<1>(v[j].w));
+                    *reinterpret_cast<uint4*>(line + ((u0 ^ (row & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4*>(line + (((u0 + 1) ^ (row & 7)) << 4)) = o1;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();

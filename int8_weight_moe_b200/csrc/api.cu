@@ -101,7 +101,7 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
         // before the down GEMV writes its own.
         const int64_t target_gu = 148LL * 16 * 16, target_d = 148LL * 16 * 2;
         const int64_t touched = A < E ? A : E;
-        const int64_t units_gu = touched * (f / 16), units_d = touched * (d / 16);
+        const int64_t units_gu = touched * (f / 16), units_d = touched * (d / 32);
         const int64_t row_gu = A * 2 * f * (int64_t)sizeof(float);
         const int64_t row_d = A * d * (int64_t)sizeof(float);
         w.split_gu = jmoe::decode_split(d, units_gu > 0 ? (target_gu + units_gu - 1) / units_gu : 1,

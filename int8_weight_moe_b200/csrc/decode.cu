@@ -109,17 +109,26 @@ __device__ __forceinline__ int64_t q_drain_begin(int64_t total, int slots) {
 
 constexpr int kSlots = 3;  // ring slots per warp: two 4 KB slots in flight
 
-// 64-byte k-blocks per ring slot: 4 KB of weights per slot in both modes.
+// Every item reads two 16-row weight matrices that share the activation
+// fragments: gate/up, the 16 gate rows and the same 16 up rows of a unit of 16
+// channels; down, the two 16-row halves of a unit of 32 output channels.  A
+// ring slot holds 2 k-blocks of 64 bytes of both: 4 KB.
 template <int MODE>
 constexpr int nb_of() {
-    return MODE == kGateUp ? 2 : 4;
+    return 2;
+}
+
+// Output channels of one unit.
+template <int MODE>
+constexpr int unit_rows() {
+    return MODE == kGateUp ? 16 : 32;
 }
 
 // Shared memory of one warp: kSlots x [matrix][k-block][16 rows][64 B]; the
 // dense 64-byte row pitch makes the fragment reads of a warp conflict-free.
 template <int MODE>
 constexpr int slot_bytes() {
-    return (MODE == kGateUp ? 2 : 1) * nb_of<MODE>() * 16 * 64;
+    return 2 * nb_of<MODE>() * 16 * 64;
 }
 
 template <int MODE>
@@ -130,7 +139,7 @@ constexpr int gemv_smem() {
 template <int MODE, int NCH>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     k_gemv(const __grid_constant__ CUtensorMap tmW, const GemvParams p) {
-    constexpr int NMAT = MODE == kGateUp ? 2 : 1;
+    constexpr int NMAT = 2;
     constexpr int kNB = nb_of<MODE>();
     constexpr int kSlotBytes = slot_bytes<MODE>();
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -145,7 +154,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int E = p.E, S = p.S;
     const int64_t K = MODE == kGateUp ? p.d : p.f;
     const int64_t rows_out = MODE == kGateUp ? p.f : p.d;
-    const int groups = (int)(rows_out / 16);
+    const int groups = (int)(rows_out / unit_rows<MODE>());
+    // row offset of the second matrix: the up rows (f below the gate rows) or
+    // the second 16-row half of the down unit
+    const int moff = MODE == kGateUp ? (int)p.f : 16;
     if (threadIdx.x <= E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
     if (lane == 0)
         for (int i = 0; i < kSlots; ++i) sm100::mbar_init(&full[warp][i], 1);
@@ -192,7 +204,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
     auto set_prefetch_item = [&](int it) {
         const Item u = item_of(it);
-        prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16 : u.e * (int)p.d + u.group * 16;
+        prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16
+                               : u.e * (int)p.d + u.group * unit_rows<MODE>();
         pk = u.z * kb_item * 64;
     };
     auto issue = [&](int slot) {
@@ -204,7 +217,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int b = 0; b < kNB; ++b)
                     sm100::tma_load_2d(dst + (m * kNB + b) * 1024, &tmW, &full[warp][slot],
-                                       pk + (pj * kNB + b) * 64, prow + m * (int)p.f);
+                                       pk + (pj * kNB + b) * 64, prow + m * moff);
         }
         if (++pj == nsl) {
             pj = 0;
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                 for (int n = 0; n < NCH; ++n) {
                     if (n * 8 < cur.cnt_pass) {
                         mma_block<true>(acc[n][0], wq[0], wq[1], bc[b][n]);
-                        if (MODE == kGateUp) mma_block<true>(acc[n][NMAT - 1], wq[2], wq[3], bc[b][n]);
+                        mma_block<true>(acc[n][1], wq[2], wq[3], bc[b][n]);
                     }
                 }
             }
@@ -322,7 +335,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int slot = n * 8 + 2 * c + (i & 1);
-                        const int64_t col = (int64_t)m * p.f + cur.u.group * 16 + g8 + (i >> 1) * 8;
+                        const int64_t col =
+                            MODE == kGateUp
+                                ? (int64_t)m * p.f + cur.u.group * 16 + g8 + (i >> 1) * 8
+                                : (int64_t)cur.u.group * 32 + m * 16 + g8 + (i >> 1) * 8;
                         if (slot < cur.cnt_pass)
                             P[(int64_t)(cur.base + slot) * cols + col] = acc[n][m][0][i] + acc[n][m][1][i];
                         acc[n][m][0][i] = acc[n][m][1][i] = 0.0f;

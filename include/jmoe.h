@@ -14,7 +14,7 @@
  *    HBM to on-chip memory; step 4, activations stay BF16.
  *  - same page, section "The Jamba Hybrid Block Structure": the MoE layer
  *    output MoE(x) = sum over the top-2 experts of g_i(x) * Expert_i(x),
- *    16 experts.
+ *    16 experts.  (The library takes 1..64 experts and top-k 1..4.)
  *  - "Jamba: A Hybrid Transformer-Mamba Language Model" (paper summary,
  *    arXiv 2403.19887), section "Mixture-of-Experts (MoE) in Jamba: Router,
  *    Top-K, and Load Balancing": g = softmax(W_r h), top-K selection, and
@@ -72,8 +72,8 @@ typedef enum {
  *   s_d  : fp32  [E][d_model]          one scale per row of w_d
  * A row's dequantised weights are q * s (ExpertsInt8 step 3). */
 typedef struct {
-    int32_t E;       /* number of experts, 1..16 */
-    int32_t top_k;   /* experts per token, 1 or 2, <= E */
+    int32_t E;       /* number of experts, 1..64 */
+    int32_t top_k;   /* experts per token, 1..4, <= E */
     int64_t d_model; /* hidden size, multiple of 64 */
     int64_t d_ff;    /* expert intermediate size, multiple of 64 */
     const int8_t* w_gu;
@@ -107,11 +107,23 @@ jmoe_status jmoe_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t
  * Logits are fp64 dot products summed in a fixed order (lane j of 32 sums
  * the elements k = j mod 32 in ascending k, then a halving tree over the 32
  * lanes), plus the bias, rounded once to fp32; selection uses these fp32
- * logits, so ids are reproducible bit for bit.  E in 1..16, top_k in {1,2},
- * d a multiple of 64, T >= 0. */
+ * logits, so ids are reproducible bit for bit.  E in 1..64, top_k in 1..4
+ * (<= E), d a multiple of 64, T >= 0. */
 jmoe_status jmoe_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
                        const float* bias, int32_t E, int32_t top_k, int32_t* topk_ids,
                        float* topk_w, float* logits, void* stream);
+
+/* jmoe_route with a choice of gates.  The two pages differ here: the Jamba
+ * summary ("Top-K selection") renormalises the selected probabilities over
+ * the selected set, the Jamba-1.5 summary ("The Jamba Hybrid Block
+ * Structure") calls the gates softmax-normalised.  flags = 0 gives the
+ * renormalised gates of jmoe_route; JMOE_ROUTE_SOFTMAX_GATES gives the plain
+ * softmax probability (over all E experts) of each selected expert.  Other
+ * bits are JMOE_EINVAL.  Everything else is as jmoe_route. */
+#define JMOE_ROUTE_SOFTMAX_GATES 1u
+jmoe_status jmoe_route_ex(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
+                          const float* bias, int32_t E, int32_t top_k, uint32_t flags,
+                          int32_t* topk_ids, float* topk_w, float* logits, void* stream);
 
 /* Grouping of the T*top_k token->expert assignments by expert (the dispatch
  * step the fused MoE kernel performs; Jamba-1.5 summary, "Innovation 2").
@@ -121,7 +133,8 @@ jmoe_status jmoe_route(const void* x_bf16, int64_t T, int64_t d, const float* w_
  * ascending a, then expert 1, ...; inv: device int32 [T*top_k] (written),
  * inv[perm[i]] = i.  Deterministic and bit-exact.  An id outside [0, E)
  * sets JMOE_EDEVICE in the device error word and the assignment is dropped.
- * A single thread block does the work (T*top_k up to 2^24). */
+ * A single thread block does the work (T*top_k up to 2^24).  E in 1..64,
+ * top_k in 1..4. */
 jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int32_t E,
                          int32_t* offsets, int32_t* perm, int32_t* inv, void* stream);
 

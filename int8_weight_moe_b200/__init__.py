@@ -24,11 +24,12 @@ JMOE_EWORKSPACE, JMOE_ECUDA, JMOE_ETIMEOUT, JMOE_EDEVICE = 4, 5, 6, 7
 JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 
 # Every C entry point the header declares.
-EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_permute", "jmoe_forward_workspace_size",
+EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_permute", "jmoe_forward_workspace_size",
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
             "jmoe_profile_events", "jmoe_launch_count", "jmoe_last_error",
             "jmoe_status_string")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
+JMOE_ROUTE_SOFTMAX_GATES = 1
 STAGES = ("permute", "gather", "gate_up", "down", "combine", "act")
 
 
@@ -66,6 +67,8 @@ def load() -> ctypes.CDLL:
     st = ctypes.c_int
     lib.jmoe_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
     lib.jmoe_route.argtypes = [vp, i64, i64, vp, vp, i32, i32, vp, vp, vp, vp]
+    lib.jmoe_route_ex.argtypes = [vp, i64, i64, vp, vp, i32, i32, ctypes.c_uint32, vp, vp, vp,
+                                  vp]
     lib.jmoe_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
     lib.jmoe_forward_workspace_size.argtypes = [ctypes.POINTER(MoeDesc), i64, ctypes.POINTER(sz)]
     lib.jmoe_forward.argtypes = [ctypes.POINTER(MoeDesc), vp, i64, vp, vp, vp, vp, sz, vp]
@@ -134,8 +137,12 @@ def jmoe_quantize(w, q=None, scales=None):
 
 
 def jmoe_route(x, w_router, top_k: int = 2, bias=None, topk_ids=None, topk_w=None,
-               logits=None, want_logits: bool = False):
-    """Router logits -> (topk_ids int32 [T, k], topk_w fp32 [T, k][, logits])."""
+               logits=None, want_logits: bool = False, softmax_gates: bool = False):
+    """Router logits -> (topk_ids int32 [T, k], topk_w fp32 [T, k][, logits]).
+
+    Gates are the selected softmax probabilities renormalised over the
+    selection, or with softmax_gates=True the plain softmax probabilities
+    (jmoe_route_ex with JMOE_ROUTE_SOFTMAX_GATES)."""
     import torch
 
     _need(x, torch.bfloat16, "x")
@@ -150,9 +157,10 @@ def jmoe_route(x, w_router, top_k: int = 2, bias=None, topk_ids=None, topk_w=Non
         topk_w = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
     if want_logits and logits is None:
         logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
-    _check("jmoe_route", load().jmoe_route(_ptr(x), T, d, _ptr(w_router), _ptr(bias), E, top_k,
-                                           _ptr(topk_ids), _ptr(topk_w), _ptr(logits),
-                                           _stream(x)))
+    flags = JMOE_ROUTE_SOFTMAX_GATES if softmax_gates else 0
+    _check("jmoe_route_ex", load().jmoe_route_ex(_ptr(x), T, d, _ptr(w_router), _ptr(bias), E,
+                                                 top_k, flags, _ptr(topk_ids), _ptr(topk_w),
+                                                 _ptr(logits), _stream(x)))
     return (topk_ids, topk_w, logits) if want_logits else (topk_ids, topk_w)
 
 

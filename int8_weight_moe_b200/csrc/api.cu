@@ -135,8 +135,8 @@ bool use_prefill(int32_t path, int64_t A) {
 
 jmoe_status check_desc(const jmoe_moe_desc* desc) {
     if (!desc) return JMOE_EINVAL;
-    if (desc->E < 1 || desc->E > 16) return JMOE_EUNSUPPORTED;
-    if (desc->top_k < 1 || desc->top_k > 2 || desc->top_k > desc->E) return JMOE_EUNSUPPORTED;
+    if (desc->E < 1 || desc->E > 64) return JMOE_EUNSUPPORTED;
+    if (desc->top_k < 1 || desc->top_k > 4 || desc->top_k > desc->E) return JMOE_EUNSUPPORTED;
     if (desc->d_model <= 0 || desc->d_ff <= 0) return JMOE_EINVAL;
     if (desc->d_model % 64 || desc->d_ff % 64) return JMOE_EUNSUPPORTED;
     if (desc->path < JMOE_PATH_AUTO || desc->path > JMOE_PATH_PREFILL) return JMOE_EINVAL;
@@ -260,22 +260,31 @@ jmoe_status jmoe_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t
 jmoe_status jmoe_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
                        const float* bias, int32_t E, int32_t top_k, int32_t* topk_ids,
                        float* topk_w, float* logits, void* stream) {
+    return jmoe_route_ex(x_bf16, T, d, w_router, bias, E, top_k, 0u, topk_ids, topk_w, logits,
+                         stream);
+}
+
+jmoe_status jmoe_route_ex(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
+                          const float* bias, int32_t E, int32_t top_k, uint32_t flags,
+                          int32_t* topk_ids, float* topk_w, float* logits, void* stream) {
     if (T < 0 || d <= 0) return JMOE_EINVAL;
-    if (E < 1 || E > 16 || top_k < 1 || top_k > 2 || top_k > E) return JMOE_EUNSUPPORTED;
+    if (flags & ~JMOE_ROUTE_SOFTMAX_GATES) return JMOE_EINVAL;
+    if (E < 1 || E > 64 || top_k < 1 || top_k > 4 || top_k > E) return JMOE_EUNSUPPORTED;
     if (d % 64) return JMOE_EUNSUPPORTED;
     if (T == 0) return JMOE_OK;
     if (!x_bf16 || !w_router || !topk_ids || !topk_w) return JMOE_EINVAL;
     if (!aligned16(x_bf16) || !aligned16(w_router) || !aligned16(topk_ids) || !aligned16(topk_w) ||
         (bias && !aligned16(bias)) || (logits && !aligned16(logits)))
         return JMOE_EALIGN;
-    return from_cuda(jmoe::launch_route(x_bf16, T, d, w_router, bias, E, top_k, topk_ids, topk_w,
+    const int renorm = (flags & JMOE_ROUTE_SOFTMAX_GATES) ? 0 : 1;
+    return from_cuda(jmoe::launch_route(x_bf16, T, d, w_router, bias, E, top_k, renorm, topk_ids, topk_w,
                                         logits, num_sms(), (cudaStream_t)stream));
 }
 
 jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int32_t E,
                          int32_t* offsets, int32_t* perm, int32_t* inv, void* stream) {
     if (T < 0) return JMOE_EINVAL;
-    if (E < 1 || E > 16 || top_k < 1 || top_k > 2) return JMOE_EUNSUPPORTED;
+    if (E < 1 || E > 64 || top_k < 1 || top_k > 4) return JMOE_EUNSUPPORTED;
     if (T * top_k > (1LL << 24)) return JMOE_EUNSUPPORTED;
     if (!offsets) return JMOE_EINVAL;
     if (T > 0 && (!topk_ids || !perm || !inv)) return JMOE_EINVAL;
@@ -289,7 +298,7 @@ jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int3
 jmoe_status jmoe_forward_workspace_size(const jmoe_moe_desc* desc, int64_t T, size_t* bytes) {
     if (!bytes || !desc) return JMOE_EINVAL;
     if (T < 0) return JMOE_EINVAL;
-    if (desc->E < 1 || desc->E > 16 || desc->top_k < 1 || desc->top_k > 2 ||
+    if (desc->E < 1 || desc->E > 64 || desc->top_k < 1 || desc->top_k > 4 ||
         desc->top_k > desc->E)
         return JMOE_EUNSUPPORTED;
     if (desc->d_model <= 0 || desc->d_ff <= 0) return JMOE_EINVAL;

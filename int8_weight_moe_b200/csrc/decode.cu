@@ -55,7 +55,7 @@ namespace jmoe {
 namespace {
 
 constexpr int kWarpsPerBlock = 4;
-constexpr int kMaxE = 16;
+constexpr int kMaxE = 64;
 
 enum { kGateUp = 0, kDown = 1 };
 
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(256)
 // token's slots, experts, gates and shifts are looked up once; each thread
 // takes 4 consecutive channels (16-byte loads).
 constexpr int kCombineChunk = 1024;  // channels per block (256 threads x 4)
-constexpr int kMaxTopK = 2;
+constexpr int kMaxTopK = 4;
 
 __global__ void __launch_bounds__(256)
     k_combine(const float* __restrict__ P, int S, int64_t A, int64_t T, int64_t d, int top_k,

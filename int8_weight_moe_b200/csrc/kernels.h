@@ -31,9 +31,11 @@ constexpr int kPrefillTileM = 128;
 cudaError_t launch_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t* q,
                             float* scales, cudaStream_t stream);
 
+// renorm != 0: the chosen softmax probabilities renormalised over the
+// selection; 0: the plain softmax probabilities.
 cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
-                         const float* bias, int E, int top_k, int32_t* ids, float* gates,
-                         float* logits, int num_sms, cudaStream_t stream);
+                         const float* bias, int E, int top_k, int renorm, int32_t* ids,
+                         float* gates, float* logits, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_t* offsets,
                            int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,

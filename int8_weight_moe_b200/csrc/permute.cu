@@ -15,7 +15,7 @@
 namespace jmoe {
 namespace {
 
-constexpr int kMaxE = 16;
+constexpr int kMaxE = 64;
 
 __global__ void __launch_bounds__(kPermuteThreads)
     k_permute(const int32_t* __restrict__ ids, int64_t A, int E, int pad, int32_t* __restrict__ offsets,

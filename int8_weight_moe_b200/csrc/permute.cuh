@@ -21,7 +21,7 @@
 namespace jmoe {
 
 constexpr int kPermuteThreads = 1024;
-constexpr int kPermuteMaxE = 16;
+constexpr int kPermuteMaxE = 64;
 
 __device__ __forceinline__ void block_permute(const int32_t* __restrict__ ids, int64_t A, int E,
                                               int pad, int32_t* __restrict__ offsets,

@@ -72,7 +72,7 @@ constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps, kEpiWarps = 4;
 constexpr int kWarpMMA2 = kEpiWarp0 + kEpiWarps;
 constexpr int kThreads = (kWarpMMA2 + 1) * 32;
 constexpr int kIssuers = 2;  // MMA-issuing threads (one per 128-row half)
-constexpr int kMaxE = 16;
+constexpr int kMaxE = 64;
 
 enum Mode { kGateUp = 0, kDown = 1 };
 

@@ -31,48 +31,52 @@ namespace jmoe {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kMaxE = 16;
-constexpr int kPerWarp = kMaxE / kWarps;
+constexpr int kMaxE = 64;      // experts
+constexpr int kMaxTopK = 4;
+constexpr int kGroupE = 16;    // experts computed together (one warp each, or 4 per warp)
+constexpr int kPerWarp = kGroupE / kWarps;
 
-// Top-k on one token's fp32 logits (strict '>' keeps the lower index on
-// ties), fp32 softmax over all E experts, renormalised over the selection.
-__device__ void select_topk(const float* l, int64_t t, int E, int top_k, int32_t* ids,
-                            float* gates, float* logits) {
+// Top-k on one token's fp32 logits: k passes of a strict '>' argmax over the
+// experts not yet chosen (the lower index wins ties), fp32 softmax over all E
+// experts, then the chosen probabilities -- renormalised over the selection
+// (in selection order) when `renorm`, as they are otherwise.
+__device__ void select_topk(const float* l, int64_t t, int E, int top_k, int renorm,
+                            int32_t* ids, float* gates, float* logits) {
     if (logits)
         for (int e = 0; e < E; ++e) logits[t * E + e] = l[e];
-    int e1 = 0;
-    for (int e = 1; e < E; ++e)
-        if (l[e] > l[e1]) e1 = e;
-    int e2 = -1;
-    if (top_k == 2)
-        for (int e = 0; e < E; ++e)
-            if (e != e1 && (e2 < 0 || l[e] > l[e2])) e2 = e;
+    int chosen[kMaxTopK];
+    for (int j = 0; j < top_k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            bool taken = false;
+            for (int i = 0; i < j; ++i) taken |= chosen[i] == e;
+            if (!taken && (best < 0 || l[e] > l[best])) best = e;
+        }
+        chosen[j] = best;
+    }
     float p[kMaxE];
-    const float m = l[e1];
+    const float m = l[chosen[0]];
     float z = 0.0f;
     for (int e = 0; e < E; ++e) {
         p[e] = expf(l[e] - m);
         z += p[e];
     }
     for (int e = 0; e < E; ++e) p[e] = p[e] / z;
-    if (top_k == 1) {
-        ids[t] = e1;
-        gates[t] = 1.0f;
-    } else {
-        const float sel = p[e1] + p[e2];
-        ids[2 * t] = e1;
-        ids[2 * t + 1] = e2;
-        gates[2 * t] = p[e1] / sel;
-        gates[2 * t + 1] = p[e2] / sel;
+    float sel = 0.0f;
+    for (int j = 0; j < top_k; ++j) sel += p[chosen[j]];
+    for (int j = 0; j < top_k; ++j) {
+        ids[t * top_k + j] = chosen[j];
+        gates[t * top_k + j] = renorm ? p[chosen[j]] / sel : p[chosen[j]];
     }
 }
 
-// Few tokens: one CTA of 16 warps per token, warp e computes expert e's
-// logit (same per-lane order and halving tree).  The token row is staged in
-// shared memory once; each warp streams its expert's router row through two
-// 4 KB shared-memory buffers with 16-byte cp.async copies (all copies of a
-// chunk in flight at once, the next chunk landing while this one is summed),
-// and lane j then reads its own k = j (mod 32) entries, conflict-free.
+// Few tokens, very wide rows: one CTA of 16 warps per token, warp w computing
+// experts w, w + 16, ... (same per-lane order and halving tree).  The token
+// row is staged in shared memory once; each warp streams its expert's router
+// row through two 4 KB shared-memory buffers with 16-byte cp.async copies
+// (all copies of a chunk in flight at once, the next chunk landing while this
+// one is summed), and lane j then reads its own k = j (mod 32) entries,
+// conflict-free.
 constexpr int kChunk = 1024;  // router-row floats per chunk
 constexpr int kChunkSmem = 2 * kChunk * 4;  // per warp: two chunks
 constexpr size_t kWideMaxSmem = 200 * 1024;  // 128 KB of chunks + token rows up to d = 36864
@@ -83,25 +87,25 @@ __device__ __forceinline__ void route_chunk_copy(float* dst, const float* src, i
     cp_async_commit();
 }
 
-__global__ void __launch_bounds__(kMaxE * 32)
+__global__ void __launch_bounds__(kGroupE * 32)
     k_route_wide(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
-                 const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
-                 float* __restrict__ gates, float* __restrict__ logits) {
+                 const float* __restrict__ bias, int E, int top_k, int renorm,
+                 int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits) {
     extern __shared__ __align__(16) uint8_t route_smem[];
     float* s_w = reinterpret_cast<float*>(route_smem);  // [16 warps][2][kChunk]
-    uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + kMaxE * kChunkSmem);  // [d]
+    uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + kGroupE * kChunkSmem);  // [d]
     __shared__ float s_logit[kMaxE];
-    const int lane = threadIdx.x & 31, e = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = blockIdx.x;
     const int nchunks = (int)((d + kChunk - 1) / kChunk);
-    float* buf = s_w + e * 2 * kChunk;
-    const float* w = wr + (int64_t)e * d;
-    if (e < E) route_chunk_copy(buf, w, (int)(d < kChunk ? d : (int64_t)kChunk), lane);
+    float* buf = s_w + warp * 2 * kChunk;
     const uint16_t* xr = x + t * d;
     for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
         *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
     __syncthreads();
-    if (e < E) {
+    for (int e = warp; e < E; e += kGroupE) {
+        const float* w = wr + (int64_t)e * d;
+        route_chunk_copy(buf, w, (int)(d < kChunk ? d : (int64_t)kChunk), lane);
         double acc = 0.0;
         for (int c = 0; c < nchunks; ++c) {
             const int64_t base = (int64_t)c * kChunk;
@@ -125,114 +129,141 @@ __global__ void __launch_bounds__(kMaxE * 32)
         if (lane == 0) s_logit[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
     }
     __syncthreads();
-    if (threadIdx.x == 0) select_topk(s_logit, t, E, top_k, ids, gates, logits);
+    if (threadIdx.x == 0) select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
 }
 
 // Few tokens, d_model up to about 11k: a cluster of 4 CTAs per token, 4
-// warps per CTA, warp w of CTA r computing expert 4r + w.  Each warp pulls its
-// whole router row into shared memory with 16-byte cp.async copies at once
-// (one memory round trip), sums in the canonical order, and writes its logit
-// into the first CTA's shared memory (distributed shared memory); after the
-// cluster barrier the first CTA selects the top-k.
+// warps per CTA, warp w of CTA r computing experts 4r + w, 4r + w + 16, ....
+// Each warp pulls one whole router row into shared memory with 16-byte
+// cp.async copies at once (one memory round trip per expert), sums in the
+// canonical order, and writes its logit into the first CTA's shared memory
+// (distributed shared memory); after the cluster barrier the first CTA
+// selects the top-k.
 constexpr int kRouteCluster = 4;
-constexpr int kExpertsPerCta = kMaxE / kRouteCluster;
+constexpr int kExpertsPerCta = kGroupE / kRouteCluster;
 constexpr size_t kClusterMaxSmem = 200 * 1024;
 
 __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExpertsPerCta * 32)
     k_route_cluster(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
-                    const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
-                    float* __restrict__ gates, float* __restrict__ logits) {
+                    const float* __restrict__ bias, int E, int top_k, int renorm,
+                    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits) {
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) uint8_t route_smem[];
     float* s_w = reinterpret_cast<float*>(route_smem);  // [kExpertsPerCta][d]
     uint16_t* s_x = reinterpret_cast<uint16_t*>(route_smem + (size_t)kExpertsPerCta * d * 4);
     __shared__ float s_logit[kMaxE];  // filled in the cluster's first CTA
     cg::cluster_group cluster = cg::this_cluster();
+    // first half of a cluster barrier: no CTA writes into another CTA's shared
+    // memory before every CTA of the cluster has started (the wait is below)
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     pdl_wait();  // the previous step may still read ids and gates
     pdl_launch_dependents();
     const unsigned rank = cluster.block_rank();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = (int)rank * kExpertsPerCta + warp;
     const int64_t t = blockIdx.x / kRouteCluster;
     float* row = s_w + (size_t)warp * d;
-    if (e < E) {
+    auto copy_row = [&](int e) {
         const float* w = wr + (int64_t)e * d;
         for (int64_t i = lane; i < d / 4; i += 32) cp_async_16(row + 4 * i, w + 4 * i, 16);
-    }
-    cp_async_commit();
+        cp_async_commit();
+    };
+    const int e0 = (int)rank * kExpertsPerCta + warp;
+    if (e0 < E) copy_row(e0);
     const uint16_t* xr = x + t * d;
     for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
         *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
-    cp_async_wait<0>();
     __syncthreads();
-    if (e < E) {
+    float* dst = cluster.map_shared_rank(s_logit, 0);
+    auto logit_of_row = [&](int e) {
+        cp_async_wait<0>();
+        __syncwarp();
         double acc = 0.0;
 #pragma unroll 8
         for (int64_t k = lane; k < d; k += 32)
             acc = fma((double)bf16_bits_to_f32(s_x[k]), (double)row[k], acc);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o);
-        if (lane == 0) {
-            float* dst = cluster.map_shared_rank(s_logit, 0);
-            dst[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
-        }
+        return __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
+    };
+    float l0 = 0.0f;
+    if (e0 < E) l0 = logit_of_row(e0);
+    // second half of the start barrier, after the first row's sum: every CTA
+    // of the cluster is running before the first remote write
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (e0 < E && lane == 0) dst[e0] = l0;
+    for (int e = e0 + kGroupE; e < E; e += kGroupE) {
+        __syncwarp();  // every lane is done with the row before it is refilled
+        copy_row(e);
+        const float l = logit_of_row(e);
+        if (lane == 0) dst[e] = l;
     }
     cluster.sync();
-    if (rank == 0 && threadIdx.x == 0) select_topk(s_logit, t, E, top_k, ids, gates, logits);
+    if (rank == 0 && threadIdx.x == 0) select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
 }
 
-template <int kTok>
+// Many tokens: a CTA of 4 warps handles kTok tokens; for each group of 16
+// experts, warp w owns experts w, w+4, w+8, w+12 of the group, so each lane
+// keeps 4 x kTok independent fp64 accumulators and every router weight it
+// loads serves kTok tokens.
+template <int kTok, bool kMultiGroup>
 __global__ void __launch_bounds__(kWarps * 32)
     k_route(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
-            const float* __restrict__ bias, int E, int top_k, int32_t* __restrict__ ids,
+            const float* __restrict__ bias, int E, int top_k, int renorm, int32_t* __restrict__ ids,
             float* __restrict__ gates, float* __restrict__ logits) {
     __shared__ float s_logit[kTok][kMaxE];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int64_t t0 = (int64_t)blockIdx.x * kTok; t0 < T; t0 += (int64_t)gridDim.x * kTok) {
-        double acc[kTok][kPerWarp];
-#pragma unroll
-        for (int t = 0; t < kTok; ++t)
-#pragma unroll
-            for (int i = 0; i < kPerWarp; ++i) acc[t][i] = 0.0;
         const uint16_t* xr[kTok];
 #pragma unroll
         for (int t = 0; t < kTok; ++t) xr[t] = x + min(t0 + t, T - 1) * d;  // clamp: tail tokens
-#pragma unroll 4
-        for (int64_t k = lane; k < d; k += 32) {
-            double xk[kTok];
-#pragma unroll
-            for (int t = 0; t < kTok; ++t) xk[t] = (double)bf16_bits_to_f32(__ldg(xr[t] + k));
-#pragma unroll
-            for (int i = 0; i < kPerWarp; ++i) {
-                const int e = warp + kWarps * i;
-                if (e < E) {
-                    const double w = (double)__ldg(wr + (int64_t)e * d + k);
-#pragma unroll
-                    for (int t = 0; t < kTok; ++t) acc[t][i] = fma(xk[t], w, acc[t][i]);
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1)
+        // one group of 16 experts unless kMultiGroup (a compile-time bound
+        // keeps the single-group loop as tight as a straight body)
+        const int groups_end = kMultiGroup ? E : 1;
+        for (int eg = 0; eg < groups_end; eg += kGroupE) {
+            double acc[kTok][kPerWarp];
 #pragma unroll
             for (int t = 0; t < kTok; ++t)
 #pragma unroll
-                for (int i = 0; i < kPerWarp; ++i)
-                    acc[t][i] += __shfl_down_sync(0xffffffffu, acc[t][i], o);
-        if (lane == 0) {
+                for (int i = 0; i < kPerWarp; ++i) acc[t][i] = 0.0;
+#pragma unroll 4
+            for (int64_t k = lane; k < d; k += 32) {
+                double xk[kTok];
 #pragma unroll
-            for (int i = 0; i < kPerWarp; ++i) {
-                const int e = warp + kWarps * i;
-                if (e < E) {
-                    const double b = bias ? (double)bias[e] : 0.0;
+                for (int t = 0; t < kTok; ++t) xk[t] = (double)bf16_bits_to_f32(__ldg(xr[t] + k));
 #pragma unroll
-                    for (int t = 0; t < kTok; ++t) s_logit[t][e] = __double2float_rn(acc[t][i] + b);
+                for (int i = 0; i < kPerWarp; ++i) {
+                    const int e = eg + warp + kWarps * i;
+                    if (e < E) {
+                        const double w = (double)__ldg(wr + (int64_t)e * d + k);
+#pragma unroll
+                        for (int t = 0; t < kTok; ++t) acc[t][i] = fma(xk[t], w, acc[t][i]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+                for (int t = 0; t < kTok; ++t)
+#pragma unroll
+                    for (int i = 0; i < kPerWarp; ++i)
+                        acc[t][i] += __shfl_down_sync(0xffffffffu, acc[t][i], o);
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < kPerWarp; ++i) {
+                    const int e = eg + warp + kWarps * i;
+                    if (e < E) {
+                        const double b = bias ? (double)bias[e] : 0.0;
+#pragma unroll
+                        for (int t = 0; t < kTok; ++t)
+                            s_logit[t][e] = __double2float_rn(acc[t][i] + b);
+                    }
                 }
             }
         }
         __syncthreads();
         if (threadIdx.x < kTok && t0 + threadIdx.x < T)
-            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, ids, gates, logits);
+            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, renorm, ids, gates,
+                        logits);
         __syncthreads();
     }
 }
@@ -240,34 +271,40 @@ __global__ void __launch_bounds__(kWarps * 32)
 }  // namespace
 
 cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
-                         const float* bias, int E, int top_k, int32_t* ids, float* gates,
-                         float* logits, int num_sms, cudaStream_t stream) {
+                         const float* bias, int E, int top_k, int renorm, int32_t* ids,
+                         float* gates, float* logits, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
     // Few tokens: a cluster of 4 CTAs per token (or, for very wide rows, a
     // 16-warp CTA streaming the router rows in chunks); many tokens: 4 tokens
     // per 4-warp CTA, which cuts the router-weight traffic fourfold.
     const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
-    const size_t smem = (size_t)kMaxE * kChunkSmem + (size_t)d * sizeof(uint16_t);
+    const size_t smem = (size_t)kGroupE * kChunkSmem + (size_t)d * sizeof(uint16_t);
     if (T < (int64_t)num_sms * 8 && csmem <= kClusterMaxSmem && T * kRouteCluster < (1LL << 31)) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
         if (e != cudaSuccess) return e;
         return launch_pdl(k_route_cluster, dim3((unsigned)(T * kRouteCluster)),
                           dim3(kExpertsPerCta * 32), csmem, stream, (const uint16_t*)x_bf16, d,
-                          w_router, bias, E, top_k, ids, gates, logits);
+                          w_router, bias, E, top_k, renorm, ids, gates, logits);
     } else if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);
         if (e != cudaSuccess) return e;
-        k_route_wide<<<(unsigned)T, kMaxE * 32, smem, stream>>>(
-            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, ids, gates, logits);
+        k_route_wide<<<(unsigned)T, kGroupE * 32, smem, stream>>>(
+            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         note_launch();
     } else {
         int64_t blocks = (T + 3) / 4;
         const int64_t cap = (int64_t)num_sms * 16;
         if (blocks > cap) blocks = cap;
-        k_route<4><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-            (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, ids, gates, logits);
+        if (E <= kGroupE)
+            k_route<4, false><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+                (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, renorm, ids, gates,
+                logits);
+        else
+            k_route<4, true><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+                (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, renorm, ids, gates,
+                logits);
         note_launch();
     }
     return cudaGetLastError();

@@ -63,6 +63,8 @@ class Oracle:
         lib.oracle_router_logits.restype = None
         lib.oracle_topk_gates.argtypes = [vp, i64, i32, i32, vp, vp]
         lib.oracle_topk_gates.restype = ctypes.c_int
+        lib.oracle_topk_gates_mode.argtypes = [vp, i64, i32, i32, i32, vp, vp]
+        lib.oracle_topk_gates_mode.restype = ctypes.c_int
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp]
         lib.oracle_permute.restype = None
         lib.oracle_moe_forward.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp,
@@ -98,22 +100,24 @@ class Oracle:
                                       None if b is None else b.ctypes.data, out.ctypes.data)
         return out
 
-    def topk_gates(self, logits: np.ndarray, top_k: int):
-        """Top-k expert ids (ties to the lower index) and renormalised fp64 gates."""
+    def topk_gates(self, logits: np.ndarray, top_k: int, renorm: bool = True):
+        """Top-k expert ids (ties to the lower index) and fp64 gates: the
+        selected softmax probabilities renormalised over the selection, or
+        (renorm=False) the plain softmax probabilities."""
         l = _c(logits, np.float32)
         T, E = l.shape
         ids = np.empty((T, top_k), dtype=np.int32)
         g = np.empty((T, top_k), dtype=np.float64)
-        rc = self.lib.oracle_topk_gates(l.ctypes.data, T, E, top_k, ids.ctypes.data,
-                                        g.ctypes.data)
+        rc = self.lib.oracle_topk_gates_mode(l.ctypes.data, T, E, top_k, 1 if renorm else 0,
+                                             ids.ctypes.data, g.ctypes.data)
         if rc != 0:
             raise ValueError("oracle_topk_gates: unsupported E/top_k")
         return ids, g
 
-    def route(self, x_bits, w_router, top_k: int, bias=None):
+    def route(self, x_bits, w_router, top_k: int, bias=None, renorm: bool = True):
         """Router logits, top-k ids and gates for every token."""
         logits = self.router_logits(x_bits, w_router, bias)
-        ids, g = self.topk_gates(logits, top_k)
+        ids, g = self.topk_gates(logits, top_k, renorm)
         return logits, ids, g
 
     def permute(self, ids: np.ndarray, E: int):
@@ -206,12 +210,12 @@ def router_logits(x_bits, w_router, bias=None):
     return default().router_logits(x_bits, w_router, bias)
 
 
-def topk_gates(logits, top_k):
-    return default().topk_gates(logits, top_k)
+def topk_gates(logits, top_k, renorm=True):
+    return default().topk_gates(logits, top_k, renorm)
 
 
-def route(x_bits, w_router, top_k, bias=None):
-    return default().route(x_bits, w_router, top_k, bias)
+def route(x_bits, w_router, top_k, bias=None, renorm=True):
+    return default().route(x_bits, w_router, top_k, bias, renorm)
 
 
 def permute(ids, E):

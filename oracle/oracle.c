@@ -120,12 +120,15 @@ void oracle_router_logits(const uint16_t* x_bf16, int64_t T, int64_t d, const fl
 }
 
 /* ------------------------------------------------------------------------ */
-/* Top-k selection of [J1] with renormalised softmax gates.                 */
+/* Top-k selection of [J1] and its gates.                                   */
 /* ids[t][j] is the j-th selected expert (largest logit first; among equal  */
-/* logits the smaller index first).  gates[t][j] = p_{ids[t][j]} / sum over  */
-/* the selected set of p, where p = softmax over all E logits (fp64).       */
-int oracle_topk_gates(const float* logits, int64_t T, int E, int top_k, int32_t* ids,
-                      double* gates) {
+/* logits the smaller index first).  With renorm != 0 ([J1]: renormalised   */
+/* over the selected set) gates[t][j] = p_{ids[t][j]} / sum over the        */
+/* selected set of p; with renorm == 0 (the plain reading of [J15]'s        */
+/* "softmax-normalized" gates) gates[t][j] = p_{ids[t][j]}; p = softmax over */
+/* all E logits (fp64).                                                      */
+int oracle_topk_gates_mode(const float* logits, int64_t T, int E, int top_k, int renorm,
+                           int32_t* ids, double* gates) {
     if (E < 1 || E > 64 || top_k < 1 || top_k > E) return 1;
     for (int64_t t = 0; t < T; ++t) {
         const float* l = logits + t * E;
@@ -154,9 +157,15 @@ int oracle_topk_gates(const float* logits, int64_t T, int E, int top_k, int32_t*
         for (int e = 0; e < E; ++e) p[e] /= z;
         double sel = 0.0;
         for (int j = 0; j < top_k; ++j) sel += p[chosen[j]];
-        for (int j = 0; j < top_k; ++j) gates[t * top_k + j] = p[chosen[j]] / sel;
+        for (int j = 0; j < top_k; ++j)
+            gates[t * top_k + j] = renorm ? p[chosen[j]] / sel : p[chosen[j]];
     }
     return 0;
+}
+
+int oracle_topk_gates(const float* logits, int64_t T, int E, int top_k, int32_t* ids,
+                      double* gates) {
+    return oracle_topk_gates_mode(logits, T, E, top_k, 1, ids, gates);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -191,15 +191,51 @@ def _topk_bruteforce(l, k):
 
 
 def pin_topk_bruteforce(o):
-    """Top-2 (and top-1, top-3) ids equal brute force over all ordered tuples."""
+    """Top-2 (and top-1, top-3; top-4 of 8) ids equal brute force over all
+    ordered tuples."""
     rng = np.random.default_rng(7)
-    for k in (1, 2, 3):
-        l = rng.standard_normal((40, 16)).astype(np.float32)
-        l[:5, 4] = l[:5, 11] = 3.0  # exact ties at the top
-        l[5:10, 2] = l[5:10, 9] = l[5:10, 13] = 2.5  # three-way ties
+    for k, E in ((1, 16), (2, 16), (3, 16), (4, 8)):
+        l = rng.standard_normal((40, E)).astype(np.float32)
+        l[:5, 4] = l[:5, E - 5] = 3.0  # exact ties at the top
+        l[5:10, 2] = l[5:10, E - 7] = l[5:10, E - 3] = 2.5  # three-way ties
         ids, _ = o.topk_gates(l, k)
         for t in range(l.shape[0]):
             assert list(ids[t]) == _topk_bruteforce(l[t], k), (k, t)
+
+
+def pin_topk_wide_stable_sort(o):
+    """64 experts, top-4: the ids are the first four of a stable descending
+    sort of the logits (equal logits keep ascending index order)."""
+    rng = np.random.default_rng(17)
+    l = rng.integers(-6, 7, size=(200, 64)).astype(np.float32) / 2  # many exact ties
+    ids, _ = o.topk_gates(l, 4)
+    ref = np.argsort(-l, axis=1, kind="stable")[:, :4]
+    assert np.array_equal(ids, ref)
+
+
+def pin_softmax_gates(o):
+    """Plain softmax gates (no renormalisation).  Closed forms: with two
+    experts and top-1 the gate is the logistic function of the logit gap;
+    with every expert selected the gates sum to 1 and g_i / g_j =
+    exp(l_i - l_j); and plain = renormalised x (sum of the plain gates)."""
+    rng = np.random.default_rng(18)
+    l2 = (rng.standard_normal((64, 2)) * 3).astype(np.float32)
+    ids, g = o.topk_gates(l2, 1, renorm=False)
+    lo = l2[np.arange(64), 1 - ids[:, 0]].astype(np.float64)
+    ls = l2[np.arange(64), ids[:, 0]].astype(np.float64)
+    assert np.allclose(g[:, 0], 1.0 / (1.0 + np.exp(lo - ls)), rtol=0, atol=1e-15)
+    l4 = (rng.standard_normal((64, 4)) * 2).astype(np.float32)
+    ids4, g4 = o.topk_gates(l4, 4, renorm=False)
+    assert np.allclose(g4.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    li = np.take_along_axis(l4, ids4, axis=1).astype(np.float64)
+    assert np.allclose(g4[:, 1:] / g4[:, :1], np.exp(li[:, 1:] - li[:, :1]), rtol=1e-14, atol=0)
+    l16 = (rng.standard_normal((64, 16)) * 2).astype(np.float32)
+    for k in (1, 2, 4):
+        idp, gp = o.topk_gates(l16, k, renorm=False)
+        idr, gr = o.topk_gates(l16, k, renorm=True)
+        assert np.array_equal(idp, idr)
+        assert np.allclose(gp, gr * gp.sum(axis=1, keepdims=True), rtol=1e-15, atol=0)
+        assert np.all(gp.sum(axis=1) <= 1.0 + 1e-15)
 
 
 def pin_topk_tie_identical_rows(o):

@@ -45,8 +45,9 @@ def call_forward(dsc, x=GOOD, T=8, ids=GOOD, w=GOOD, out=GOOD, ws=GOOD, ws_bytes
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(E=0), jm.JMOE_EUNSUPPORTED), (dict(E=17), jm.JMOE_EUNSUPPORTED),
-    (dict(top_k=3), jm.JMOE_EUNSUPPORTED), (dict(E=1, top_k=2), jm.JMOE_EUNSUPPORTED),
+    (dict(E=0), jm.JMOE_EUNSUPPORTED), (dict(E=65), jm.JMOE_EUNSUPPORTED),
+    (dict(top_k=5), jm.JMOE_EUNSUPPORTED), (dict(E=1, top_k=2), jm.JMOE_EUNSUPPORTED),
+    (dict(E=3, top_k=4), jm.JMOE_EUNSUPPORTED),
     (dict(d_model=100), jm.JMOE_EUNSUPPORTED), (dict(d_ff=96), jm.JMOE_EUNSUPPORTED),
     (dict(d_model=0), jm.JMOE_EINVAL), (dict(path=7), jm.JMOE_EINVAL),
     (dict(w_gu=None), jm.JMOE_EINVAL), (dict(s_d=None), jm.JMOE_EINVAL),
@@ -85,8 +86,14 @@ def test_quantize_route_permute_validation():
     assert lib.jmoe_quantize(None, 4, 16, GOOD, GOOD, None) == jm.JMOE_EINVAL
     assert lib.jmoe_quantize(BAD, 4, 16, GOOD, GOOD, None) == jm.JMOE_EALIGN
     assert lib.jmoe_quantize(None, 0, 16, None, None, None) == jm.JMOE_OK
-    assert lib.jmoe_route(GOOD, 4, 256, GOOD, None, 17, 2, GOOD, GOOD, None, None) == \
+    assert lib.jmoe_route(GOOD, 4, 256, GOOD, None, 65, 2, GOOD, GOOD, None, None) == \
         jm.JMOE_EUNSUPPORTED
+    assert lib.jmoe_route(GOOD, 4, 256, GOOD, None, 64, 5, GOOD, GOOD, None, None) == \
+        jm.JMOE_EUNSUPPORTED
+    assert lib.jmoe_route_ex(GOOD, 4, 256, GOOD, None, 16, 2, 2, GOOD, GOOD, None, None) == \
+        jm.JMOE_EINVAL
+    assert lib.jmoe_route_ex(None, 0, 256, None, None, 64, 4, jm.JMOE_ROUTE_SOFTMAX_GATES, None,
+                             None, None, None) == jm.JMOE_OK
     assert lib.jmoe_route(GOOD, 4, 100, GOOD, None, 16, 2, GOOD, GOOD, None, None) == \
         jm.JMOE_EUNSUPPORTED
     assert lib.jmoe_route(GOOD, 4, 256, GOOD, BAD, 16, 2, GOOD, GOOD, None, None) == \
@@ -94,7 +101,8 @@ def test_quantize_route_permute_validation():
     assert lib.jmoe_route(None, 4, 256, GOOD, None, 16, 2, GOOD, GOOD, None, None) == \
         jm.JMOE_EINVAL
     assert lib.jmoe_route(None, 0, 256, None, None, 16, 2, None, None, None, None) == jm.JMOE_OK
-    assert lib.jmoe_permute(GOOD, 4, 3, 16, GOOD, GOOD, GOOD, None) == jm.JMOE_EUNSUPPORTED
+    assert lib.jmoe_permute(GOOD, 4, 5, 16, GOOD, GOOD, GOOD, None) == jm.JMOE_EUNSUPPORTED
+    assert lib.jmoe_permute(GOOD, 4, 2, 65, GOOD, GOOD, GOOD, None) == jm.JMOE_EUNSUPPORTED
     assert lib.jmoe_permute(GOOD, 4, 2, 16, None, GOOD, GOOD, None) == jm.JMOE_EINVAL
     assert lib.jmoe_permute(GOOD, 4, 2, 16, GOOD, BAD, GOOD, None) == jm.JMOE_EALIGN
 

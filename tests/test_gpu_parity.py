@@ -334,3 +334,44 @@ def test_launch_counter_per_path(path, expected):
     n2 = jm.jmoe_launch_count()
     torch.cuda.synchronize()
     assert (n1 - n0, n2 - n1) == (1, expected)
+
+
+# ----------------------------------------------------------------------------- generalised routing
+
+ROUTE_SHAPES = [(64, 4), (8, 2), (32, 3), (64, 1)]
+
+
+@pytest.mark.parametrize("E,top_k", ROUTE_SHAPES, ids=lambda v: str(v))
+@pytest.mark.parametrize("softmax_gates", [False, True], ids=["renorm", "softmax"])
+@pytest.mark.parametrize("T,d", [(37, 256), (5, 12288), (1300, 256)],
+                         ids=["cluster", "wide_rows", "many_tokens"])
+def test_route_generalised_bitexact(E, top_k, softmax_gates, T, d):
+    wl = Workload("route_gen", 14, T, d, 64, E=E, top_k=top_k)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g, logits = jm.jmoe_route(dev.x, dev.w_router, top_k, want_logits=True,
+                                   softmax_gates=softmax_gates)
+    lo, io, go = oracle.route(ora.x_bits, ora.w_router, top_k, renorm=not softmax_gates)
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    gg = g.cpu().numpy().astype(np.float64)
+    # fp32 softmax: the denominator sums up to 64 terms, so up to ~64 ulp
+    assert np.abs(gg - go).max() <= 4e-6
+    if not softmax_gates:
+        assert np.abs(gg.sum(axis=1) - 1.0).max() <= 2.0 ** -20
+
+
+@pytest.mark.parametrize("E,top_k,T", [(64, 4, 37), (8, 2, 300), (32, 3, 129), (48, 4, 2)],
+                         ids=lambda v: str(v))
+@pytest.mark.parametrize("path", PATHS)
+def test_forward_generalised_routing(E, top_k, T, path):
+    wl = Workload("fwd_gen", 15, T, 256, 576, E=E, top_k=top_k)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g = jm.jmoe_route(dev.x, dev.w_router, top_k, softmax_gates=(E == 32))
+    out = jm.jmoe_forward(dev.desc(path), dev.x, ids, g)
+    torch.cuda.synchronize()
+    _, io, go = oracle.route(ora.x_bits, ora.w_router, top_k, renorm=(E != 32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    tokens = np.arange(T) if T <= 64 else np.r_[0:8, T - 8:T]
+    ref = ora.forward_tokens(tokens, io, go)
+    assert_close(bf16_to_f64(out)[tokens], ref, f"E={E} top_k={top_k}")
+    assert jm.jmoe_last_error() == jm.JMOE_OK

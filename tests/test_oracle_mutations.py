@@ -27,8 +27,14 @@ MUTATIONS = [
     # top-k and gates
     ("ties_to_higher_index", "if (best < 0 || l[e] > l[best]) best = e;",
      "if (best < 0 || l[e] >= l[best]) best = e;"),
-    ("gates_not_renormalised", "gates[t * top_k + j] = p[chosen[j]] / sel;",
+    ("gates_not_renormalised", "gates[t * top_k + j] = renorm ? p[chosen[j]] / sel : p[chosen[j]];",
      "gates[t * top_k + j] = p[chosen[j]];"),
+    ("softmax_gates_renormalised",
+     "gates[t * top_k + j] = renorm ? p[chosen[j]] / sel : p[chosen[j]];",
+     "gates[t * top_k + j] = p[chosen[j]] / sel;"),
+    ("softmax_gates_over_selection_only", "for (int e = 0; e < E; ++e) p[e] /= z;",
+     "for (int e = 0; e < E; ++e) p[e] /= z;\n        if (!renorm) { double zs = 0.0; for (int j = 0; j < top_k; ++j) zs += p[chosen[j]]; for (int e = 0; e < E; ++e) p[e] /= zs; }"),
+    ("topk_allows_repeats", "if (taken) continue;", "(void)taken;"),
     ("softmax_missing_max_shift", "p[e] = exp((double)l[e] - m);", "p[e] = exp((double)l[e]);"),
     # permutation
     ("permute_reverse_order", "for (int64_t a = 0; a < A; ++a) {\n        int32_t pos",

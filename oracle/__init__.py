@@ -65,6 +65,8 @@ class Oracle:
         lib.oracle_topk_gates.restype = ctypes.c_int
         lib.oracle_topk_gates_mode.argtypes = [vp, i64, i32, i32, i32, vp, vp]
         lib.oracle_topk_gates_mode.restype = ctypes.c_int
+        lib.oracle_rmsnorm.argtypes = [vp, i64, i64, vp, ctypes.c_float, vp]
+        lib.oracle_rmsnorm.restype = None
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp]
         lib.oracle_permute.restype = None
         lib.oracle_moe_forward.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp,
@@ -113,6 +115,16 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle_topk_gates: unsupported E/top_k")
         return ids, g
+
+    def rmsnorm(self, x_bits: np.ndarray, gamma_bits: np.ndarray, eps: float) -> np.ndarray:
+        """RMSNorm of bf16 rows: bf16 bits of (x * r) * gamma, r = 1/sqrt(mean(x^2) + eps)."""
+        x = _c(x_bits, np.uint16)
+        gm = _c(gamma_bits, np.uint16)
+        T, d = x.shape
+        assert gm.shape == (d,)
+        out = np.empty((T, d), dtype=np.uint16)
+        self.lib.oracle_rmsnorm(x.ctypes.data, T, d, gm.ctypes.data, float(eps), out.ctypes.data)
+        return out
 
     def route(self, x_bits, w_router, top_k: int, bias=None, renorm: bool = True):
         """Router logits, top-k ids and gates for every token."""
@@ -212,6 +224,10 @@ def router_logits(x_bits, w_router, bias=None):
 
 def topk_gates(logits, top_k, renorm=True):
     return default().topk_gates(logits, top_k, renorm)
+
+
+def rmsnorm(x_bits, gamma_bits, eps):
+    return default().rmsnorm(x_bits, gamma_bits, eps)
 
 
 def route(x_bits, w_router, top_k, bias=None, renorm=True):

@@ -64,6 +64,60 @@ static double round_to_bf16(double v) {
     return (double)f;
 }
 
+/* Round an fp64 value once, to nearest with ties to even, to the nearest     */
+/* bfloat16 (8 significant bits; fp32's exponent range, subnormals down to    */
+/* 2^-133); returns the bf16 bit pattern.  Scaling by powers of two and rint  */
+/* (ties to even in the default mode) are exact, so there is one rounding.    */
+static uint16_t f64_to_bf16_bits(double v) {
+    if (v != v) return 0x7fc0u;
+    const uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    double r;
+    if (a < ldexp(1.0, -126)) {
+        r = rint(a * ldexp(1.0, 133)) * ldexp(1.0, -133);
+    } else {
+        int e;
+        frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+        const double q = ldexp(1.0, e - 8);
+        r = rint(a / q) * q;
+    }
+    if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7f80u);
+    float f = (float)r; /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(sign | (uint16_t)((u >> 16) & 0x7fffu));
+}
+
+/* ------------------------------------------------------------------------ */
+/* RMSNorm ahead of the router (the pages: RMSNorm precedes the modules of   */
+/* a Jamba block).  Plain reading, with every rounding fixed so the routing   */
+/* that follows is reproducible bit for bit:                                  */
+/*   ss = sum of x_k^2 in fp64 in the canonical order of the router (lane j   */
+/*        of 32 sums k = j mod 32 ascending, then the halving tree; squares   */
+/*        of bf16 values are exact in fp64),                                  */
+/*   r  = 1 / sqrt(ss / d + eps)  (fp64, correctly rounded sqrt and divides), */
+/*   y_k = bf16( (x_k * r) * gamma_k )  (fp64 products, one rounding).        */
+void oracle_rmsnorm(const uint16_t* x_bf16, int64_t T, int64_t d, const uint16_t* gamma_bf16,
+                    float eps, uint16_t* y_bf16) {
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t* x = x_bf16 + t * d;
+        double p[32];
+        for (int j = 0; j < 32; ++j) {
+            p[j] = 0.0;
+            for (int64_t k = j; k < d; k += 32) {
+                const double v = (double)bf16_to_f32(x[k]);
+                p[j] += v * v;
+            }
+        }
+        for (int o = 16; o >= 1; o /= 2)
+            for (int j = 0; j < o; ++j) p[j] = p[j] + p[j + o];
+        const double r = 1.0 / sqrt(p[0] / (double)d + (double)eps);
+        for (int64_t k = 0; k < d; ++k)
+            y_bf16[t * d + k] = f64_to_bf16_bits(((double)bf16_to_f32(x[k]) * r) *
+                                                 (double)bf16_to_f32(gamma_bf16[k]));
+    }
+}
+
 /* ------------------------------------------------------------------------ */
 /* Step 1 of [J15]: BF16 weights -> INT8 + one fp32 scale per output row.    */
 /* w_bf16 is row-major [rows][cols]; a row is one output channel.           */

@@ -65,3 +65,25 @@ def round_f32_to_bf16_bits(f: np.ndarray) -> np.ndarray:
     u = np.asarray(f, dtype=np.float32).view(np.uint32).astype(np.uint64)
     u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
     return u.astype(np.uint16)
+
+
+def exact_to_bf16_bits(v: Fraction) -> int:
+    """Round an exact rational once, to nearest with ties to even, to bfloat16
+    (8 significant bits, fp32's exponent range); returns the bit pattern."""
+    if v == 0:
+        return 0
+    sign = 0x8000 if v < 0 else 0
+    a = -v if v < 0 else v
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    if e < -126:
+        q = Fraction(1, 2 ** 133)
+    else:
+        q = Fraction(2) ** (e - 7)
+    n = round_half_even(a / q)
+    r = n * q
+    if r >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    f = np.float32(float(r))  # exact: at most 8 significant bits
+    return sign | int((f.view(np.uint32) >> 16) & 0x7FFF)

@@ -24,7 +24,8 @@ from fractions import Fraction
 import numpy as np
 
 import synth
-from exact import bf16_bits, bf16_value, fr, round_half_even, to_fp32
+from exact import (bf16_bits, bf16_value, exact_to_bf16_bits, fr, round_f32_to_bf16_bits,
+                   round_half_even, to_fp32)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -463,6 +464,54 @@ def pin_bf16_h_variant(o):
     b = o.mlp_forward(x, qg[0], sg[0], qd[0], sd[0], round_h_bf16=True)
     rel = np.abs(a - b).sum() / np.abs(a).sum()
     assert 0 < rel < 5e-3, rel
+
+
+def _rmsnorm_exact(x_bits, g_bits, eps):
+    """RMSNorm to ~60 digits (Fractions, Decimal square root), rounded once to
+    bf16: the value the oracle must hit unless it lies within a few fp64 ulps
+    of a bf16 rounding boundary."""
+    import decimal
+    from fractions import Fraction
+
+    ctx = decimal.Context(prec=60)
+    x = [fr(v) for v in bf16_value(x_bits)]
+    g = [fr(v) for v in bf16_value(g_bits)]
+    mean = sum(v * v for v in x) / len(x) + fr(np.float32(eps))
+    rs = ctx.divide(decimal.Decimal(1), ctx.sqrt(ctx.divide(decimal.Decimal(mean.numerator),
+                                                            decimal.Decimal(mean.denominator))))
+    r = Fraction(rs)
+    return np.array([exact_to_bf16_bits(xv * r * gv) for xv, gv in zip(x, g)], dtype=np.uint16)
+
+
+def pin_rmsnorm_exact(o):
+    """RMSNorm equals the exact value rounded once to bf16, for a typical eps
+    and for a large eps on small activations (where dropping eps shows)."""
+    rng = np.random.default_rng(21)
+    for sigma, eps in ((1.0, 1e-6), (0.4, 0.5)):
+        x = round_f32_to_bf16_bits((rng.standard_normal((6, 96)) * sigma).astype(np.float32))
+        g = round_f32_to_bf16_bits((1.0 + 0.25 * rng.standard_normal(96)).astype(np.float32))
+        y = o.rmsnorm(x, g, eps)
+        for t in range(x.shape[0]):
+            assert np.array_equal(y[t], _rmsnorm_exact(x[t], g, eps)), (sigma, eps, t)
+
+
+def pin_rmsnorm_invariants(o):
+    """Bitwise: y(-x) = -y(x); with eps = 0, y(2^m x) = y(x); doubling gamma
+    doubles y; a constant row with gamma = 1 and eps = 0 normalises to +-1."""
+    rng = np.random.default_rng(22)
+    x = round_f32_to_bf16_bits(rng.standard_normal((8, 128)).astype(np.float32))
+    g = round_f32_to_bf16_bits((0.5 + rng.random(128)).astype(np.float32))
+    y = o.rmsnorm(x, g, 0.0)
+    assert np.array_equal(o.rmsnorm(x ^ np.uint16(0x8000), g, 0.0), y ^ np.uint16(0x8000))
+    x32 = bf16_bits(bf16_value(x) * 32.0)
+    assert np.array_equal(o.rmsnorm(x32, g, 0.0), y)
+    g2 = bf16_bits(bf16_value(g) * 2.0)
+    assert np.array_equal(bf16_value(o.rmsnorm(x, g2, 0.0)), bf16_value(y) * 2.0)
+    c = np.full((3, 64), 0, dtype=np.uint16)
+    c[0], c[1], c[2] = bf16_bits([3.0])[0], bf16_bits([-0.125])[0], bf16_bits([1.5])[0]
+    ones = bf16_bits(np.ones(64))
+    yc = bf16_value(o.rmsnorm(c, ones, 0.0))
+    assert np.all(yc[0] == 1.0) and np.all(yc[1] == -1.0) and np.all(yc[2] == 1.0)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -36,6 +36,14 @@ MUTATIONS = [
      "for (int e = 0; e < E; ++e) p[e] /= z;\n        if (!renorm) { double zs = 0.0; for (int j = 0; j < top_k; ++j) zs += p[chosen[j]]; for (int e = 0; e < E; ++e) p[e] /= zs; }"),
     ("topk_allows_repeats", "if (taken) continue;", "(void)taken;"),
     ("softmax_missing_max_shift", "p[e] = exp((double)l[e] - m);", "p[e] = exp((double)l[e]);"),
+    # RMSNorm ahead of the router
+    ("rmsnorm_eps_dropped", "1.0 / sqrt(p[0] / (double)d + (double)eps)", "1.0 / sqrt(p[0] / (double)d)"),
+    ("rmsnorm_sum_not_mean", "1.0 / sqrt(p[0] / (double)d + (double)eps)",
+     "1.0 / sqrt(p[0] + (double)eps)"),
+    ("rmsnorm_no_sqrt", "1.0 / sqrt(p[0] / (double)d + (double)eps)",
+     "1.0 / (p[0] / (double)d + (double)eps)"),
+    ("rmsnorm_gamma_ignored", "((double)bf16_to_f32(x[k]) * r) *\n                                                 (double)bf16_to_f32(gamma_bf16[k])",
+     "((double)bf16_to_f32(x[k]) * r)"),
     # permutation
     ("permute_reverse_order", "for (int64_t a = 0; a < A; ++a) {\n        int32_t pos",
      "for (int64_t a = A - 1; a >= 0; --a) {\n        int32_t pos"),

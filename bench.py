@@ -33,8 +33,9 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 import synth  # noqa: E402
-from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DENSE,  # noqa: E402
-                             MINI_PREFILL, SIGMA_R, SIGMA_W, SIGMA_X, TINY, Workload)
+from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE,  # noqa: E402
+                             MINI_DECODE_E64, MINI_DENSE, MINI_PREFILL, SIGMA_R, SIGMA_W, SIGMA_X,
+                             TINY, Workload)
 
 HEADLINE = MINI_DECODE
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 roofline"
@@ -349,6 +350,35 @@ def roofline_entry(layer: Layer, stages: dict, peaks: dict):
             "ms": round(ms, 4), "peak_source": peaks["source"] + " hbm copy"}
 
 
+def graph_run(layer: Layer, steps: int, warmup: int = 3):
+    """The whole layer with its RMSNorm prologue -- RMSNorm + router + experts
+    -- captured once in a CUDA graph (int8_weight_moe_b200.MoeLayerGraph) and
+    replayed; ms per replay from CUDA events on the replay stream."""
+    import torch
+
+    import int8_weight_moe_b200 as jm
+
+    wl = layer.wl
+    gamma = (synth.normal_bf16_gpu(wl.seed + 7, synth.X, 0.25, (wl.d_model,),
+                                   device=layer.device).float() + 1.0).to(torch.bfloat16)
+    g = jm.MoeLayerGraph(layer.desc, layer.w_router, wl.T, gamma=gamma, eps=1e-6,
+                         bias=layer.bias)
+    g.x.copy_(layer.x)
+    for _ in range(warmup):
+        g.run()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        g.run()
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / steps
+    return {"workload": wl.name + " + RMSNorm prologue, CUDA graph", "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(wl.T / (ms * 1e-3), 1)}
+
+
 def e2e_run(layer: Layer, steps: int, warmup: int, dist_on: bool = False):
     """Same metric through the public API with host buffers: per step a
     host->device copy of the tokens from pinned memory and a device->host read
@@ -568,6 +598,7 @@ def main():
     e2e_ms = max_over_ranks(e2e["ms_per_step"], dev)
     e2e["ms_per_step"] = round(e2e_ms, 4)
     e2e["value"] = round(whole_job_tokens_per_s(world, wl.T, e2e_ms), 1)
+    graph_line = graph_run(layer, max(args.steps // 2, 10)) if not wl.dense else None
     work = kernel_work(layer)
     step_gbs = work["step_bytes"] / (ms * 1e-3) / 1e9
     del layer
@@ -575,7 +606,8 @@ def main():
 
     also = []
     if not args.no_also and not args.only:
-        for other in (TINY, MINI_PREFILL, MINI_DENSE, LARGE_DECODE, LARGE_PREFILL_SKEW):
+        for other in (TINY, MINI_PREFILL, MINI_DENSE, LARGE_DECODE, LARGE_PREFILL_SKEW,
+                      MINI_DECODE_E64):
             lay = Layer(other, torch.device("cuda", local))
             steps = 20 if other.regime == "prefill" else 100
             tms, st, _ = timed_run(lay, steps, 3, dist_on)
@@ -614,7 +646,7 @@ def main():
                                     "around every stage (the timed pass records only the "
                                     "gate/up pair)",
                 "step_hbm_gbs": round(step_gbs, 1),
-                "touched_experts": work["touched"], "also": also}
+                "touched_experts": work["touched"], "graph": graph_line, "also": also}
         print(json.dumps(line), flush=True)
     if dist_on:
         import torch.distributed as dist

@@ -125,6 +125,32 @@ jmoe_status jmoe_route_ex(const void* x_bf16, int64_t T, int64_t d, const float*
                           const float* bias, int32_t E, int32_t top_k, uint32_t flags,
                           int32_t* topk_ids, float* topk_w, float* logits, void* stream);
 
+/* RMSNorm ("Jamba: A Hybrid Transformer-Mamba Language Model", paper
+ * summary: section "The major components and their responsibilities" places
+ * an RMSNorm at the input of the block's modules; section "Training
+ * Infrastructure and Stabilization Techniques" defines RMSNorm(x) =
+ * x / sqrt(mean(x^2) + eps) * gamma).  Every rounding is fixed, so the
+ * routing that follows is reproducible bit for bit:
+ *   ss = sum of x_k^2 in fp64 in the router's order (lane j of 32 sums
+ *        k = j mod 32 ascending, then a halving tree over the lanes);
+ *   r  = 1 / sqrt(ss / d + eps), IEEE-rounded fp64 steps;
+ *   y_k = bf16((x_k * r) * gamma_k), fp64 products rounded once to bf16.
+ * x_bf16 : device, bf16 [T][d];  gamma_bf16 : device, bf16 [d]
+ * y_bf16 : device, bf16 [T][d] (written; must not overlap x)
+ * eps >= 0 and finite; d a multiple of 64; all pointers 16-byte aligned. */
+jmoe_status jmoe_rmsnorm(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                         float eps, void* y_bf16, void* stream);
+
+/* RMSNorm, then the router on the normalised rows: the pre-MoE prologue of a
+ * Jamba MoE layer.  y_bf16 receives the normalised rows (the expert input);
+ * the routing outputs are those of jmoe_route_ex on y.  For few tokens the
+ * normalisation is fused into the router kernel; otherwise jmoe_rmsnorm
+ * runs first.  Arguments as jmoe_rmsnorm and jmoe_route_ex. */
+jmoe_status jmoe_rmsnorm_route(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                               float eps, void* y_bf16, const float* w_router, const float* bias,
+                               int32_t E, int32_t top_k, uint32_t flags, int32_t* topk_ids,
+                               float* topk_w, float* logits, void* stream);
+
 /* Grouping of the T*top_k token->expert assignments by expert (the dispatch
  * step the fused MoE kernel performs; Jamba-1.5 summary, "Innovation 2").
  * Assignment a = t*top_k + j.  offsets: device int32 [E+1] (written),

@@ -24,7 +24,8 @@ JMOE_EWORKSPACE, JMOE_ECUDA, JMOE_ETIMEOUT, JMOE_EDEVICE = 4, 5, 6, 7
 JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 
 # Every C entry point the header declares.
-EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_permute", "jmoe_forward_workspace_size",
+EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_rmsnorm", "jmoe_rmsnorm_route",
+            "jmoe_permute", "jmoe_forward_workspace_size",
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
             "jmoe_profile_events", "jmoe_launch_count", "jmoe_last_error",
             "jmoe_status_string")
@@ -69,6 +70,9 @@ def load() -> ctypes.CDLL:
     lib.jmoe_route.argtypes = [vp, i64, i64, vp, vp, i32, i32, vp, vp, vp, vp]
     lib.jmoe_route_ex.argtypes = [vp, i64, i64, vp, vp, i32, i32, ctypes.c_uint32, vp, vp, vp,
                                   vp]
+    lib.jmoe_rmsnorm.argtypes = [vp, i64, i64, vp, ctypes.c_float, vp, vp]
+    lib.jmoe_rmsnorm_route.argtypes = [vp, i64, i64, vp, ctypes.c_float, vp, vp, vp, i32, i32,
+                                       ctypes.c_uint32, vp, vp, vp, vp]
     lib.jmoe_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp]
     lib.jmoe_forward_workspace_size.argtypes = [ctypes.POINTER(MoeDesc), i64, ctypes.POINTER(sz)]
     lib.jmoe_forward.argtypes = [ctypes.POINTER(MoeDesc), vp, i64, vp, vp, vp, vp, sz, vp]
@@ -162,6 +166,50 @@ def jmoe_route(x, w_router, top_k: int = 2, bias=None, topk_ids=None, topk_w=Non
                                                  top_k, flags, _ptr(topk_ids), _ptr(topk_w),
                                                  _ptr(logits), _stream(x)))
     return (topk_ids, topk_w, logits) if want_logits else (topk_ids, topk_w)
+
+
+def jmoe_rmsnorm(x, gamma, eps: float, out=None):
+    """RMSNorm of bf16 rows: bf16((x * r) * gamma), r = 1/sqrt(mean(x^2) + eps)."""
+    import torch
+
+    _need(x, torch.bfloat16, "x")
+    _need(gamma, torch.bfloat16, "gamma")
+    T, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _check("jmoe_rmsnorm", load().jmoe_rmsnorm(_ptr(x), T, d, _ptr(gamma), float(eps), _ptr(out),
+                                               _stream(x)))
+    return out
+
+
+def jmoe_rmsnorm_route(x, gamma, eps: float, w_router, top_k: int = 2, bias=None, x_norm=None,
+                       topk_ids=None, topk_w=None, logits=None, want_logits: bool = False,
+                       softmax_gates: bool = False):
+    """The pre-MoE prologue: RMSNorm, then the router on the normalised rows.
+    Returns (x_norm, topk_ids, topk_w[, logits])."""
+    import torch
+
+    _need(x, torch.bfloat16, "x")
+    _need(gamma, torch.bfloat16, "gamma")
+    _need(w_router, torch.float32, "w_router")
+    T, d = x.shape
+    E = w_router.shape[0]
+    if bias is not None:
+        _need(bias, torch.float32, "bias")
+    if x_norm is None:
+        x_norm = torch.empty_like(x)
+    if topk_ids is None:
+        topk_ids = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+    if want_logits and logits is None:
+        logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    flags = JMOE_ROUTE_SOFTMAX_GATES if softmax_gates else 0
+    _check("jmoe_rmsnorm_route", load().jmoe_rmsnorm_route(
+        _ptr(x), T, d, _ptr(gamma), float(eps), _ptr(x_norm), _ptr(w_router), _ptr(bias), E, top_k,
+        flags, _ptr(topk_ids), _ptr(topk_w), _ptr(logits), _stream(x)))
+    out = (x_norm, topk_ids, topk_w)
+    return out + (logits,) if want_logits else out
 
 
 def jmoe_permute(topk_ids, E: int):
@@ -301,6 +349,60 @@ def jmoe_last_error() -> int:
 
 def jmoe_status_string(status: int) -> str:
     return status_string(status)
+
+
+class MoeLayerGraph:
+    """A whole MoE layer -- RMSNorm + router (or router alone) + experts --
+    captured once in a CUDA graph for a fixed token count and replayed.
+
+    The graph reads the static input buffer ``x`` and writes ``out``; copy a
+    batch into ``x`` (or pass it to ``run``) before each replay.  Every buffer
+    the kernels touch (routing tables, workspace, normalised rows) is owned by
+    this object, so replays allocate nothing."""
+
+    def __init__(self, desc: MoeDesc, w_router, T: int, gamma=None, eps: float = 1e-6,
+                 bias=None, softmax_gates: bool = False, device=None):
+        import torch
+
+        device = device or w_router.device
+        d = desc.d_model
+        self.desc, self.w_router, self.gamma, self.eps = desc, w_router, gamma, eps
+        self.bias, self.softmax_gates = bias, softmax_gates
+        self.x = torch.zeros((T, d), dtype=torch.bfloat16, device=device)
+        self.x_norm = torch.empty_like(self.x) if gamma is not None else None
+        self.ids = torch.empty((T, desc.top_k), dtype=torch.int32, device=device)
+        self.gates = torch.empty((T, desc.top_k), dtype=torch.float32, device=device)
+        self.out = torch.empty_like(self.x)
+        self.ws = torch.empty(max(jmoe_forward_workspace_size(desc, T), 1), dtype=torch.uint8,
+                              device=device)
+        stream = torch.cuda.Stream(device=device)
+        stream.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(stream):
+            self._body()  # warm-up outside the capture (per-device first-use setup)
+        torch.cuda.current_stream(device).wait_stream(stream)
+        torch.cuda.synchronize(device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=stream):
+            self._body()
+
+    def _body(self):
+        if self.gamma is not None:
+            jmoe_rmsnorm_route(self.x, self.gamma, self.eps, self.w_router, self.desc.top_k,
+                               self.bias, x_norm=self.x_norm, topk_ids=self.ids,
+                               topk_w=self.gates, softmax_gates=self.softmax_gates)
+            xin = self.x_norm
+        else:
+            jmoe_route(self.x, self.w_router, self.desc.top_k, self.bias, topk_ids=self.ids,
+                       topk_w=self.gates, softmax_gates=self.softmax_gates)
+            xin = self.x
+        jmoe_forward(self.desc, xin, self.ids, self.gates, out=self.out, workspace=self.ws)
+
+    def run(self, x=None):
+        """Replay on the current stream (after copying ``x`` in, if given); returns ``out``."""
+        if x is not None:
+            self.x.copy_(x)
+        self.graph.replay()
+        return self.out
 
 
 def moe_layer(x, w_router, desc: MoeDesc, bias=None, workspace=None):

@@ -133,6 +133,21 @@ bool use_prefill(int32_t path, int64_t A) {
     return A >= kDecodeMaxAssignments && jmoe::prefill_available();
 }
 
+jmoe_status check_norm(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                       float eps, const void* y_bf16) {
+    if (T < 0 || d <= 0) return JMOE_EINVAL;
+    if (!(eps >= 0.0f) || eps > 3.0e38f) return JMOE_EINVAL;  // negative, NaN or inf
+    if (d % 64) return JMOE_EUNSUPPORTED;
+    if (T == 0) return JMOE_OK;
+    if (!x_bf16 || !gamma_bf16 || !y_bf16) return JMOE_EINVAL;
+    if (!aligned16(x_bf16) || !aligned16(gamma_bf16) || !aligned16(y_bf16)) return JMOE_EALIGN;
+    const char* xa = static_cast<const char*>(x_bf16);
+    const char* ya = static_cast<const char*>(y_bf16);
+    const size_t bytes = (size_t)T * (size_t)d * 2;
+    if (xa < ya + bytes && ya < xa + bytes) return JMOE_EINVAL;  // overlap
+    return JMOE_OK;
+}
+
 jmoe_status check_desc(const jmoe_moe_desc* desc) {
     if (!desc) return JMOE_EINVAL;
     if (desc->E < 1 || desc->E > 64) return JMOE_EUNSUPPORTED;
@@ -279,6 +294,33 @@ jmoe_status jmoe_route_ex(const void* x_bf16, int64_t T, int64_t d, const float*
     const int renorm = (flags & JMOE_ROUTE_SOFTMAX_GATES) ? 0 : 1;
     return from_cuda(jmoe::launch_route(x_bf16, T, d, w_router, bias, E, top_k, renorm, topk_ids, topk_w,
                                         logits, num_sms(), (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_rmsnorm(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                         float eps, void* y_bf16, void* stream) {
+    const jmoe_status st = check_norm(x_bf16, T, d, gamma_bf16, eps, y_bf16);
+    if (st != JMOE_OK || T == 0) return st;
+    return from_cuda(jmoe::launch_rmsnorm(x_bf16, T, d, gamma_bf16, eps, y_bf16, num_sms(),
+                                          (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_rmsnorm_route(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                               float eps, void* y_bf16, const float* w_router, const float* bias,
+                               int32_t E, int32_t top_k, uint32_t flags, int32_t* topk_ids,
+                               float* topk_w, float* logits, void* stream) {
+    jmoe_status st = check_norm(x_bf16, T, d, gamma_bf16, eps, y_bf16);
+    if (st != JMOE_OK) return st;
+    if (flags & ~JMOE_ROUTE_SOFTMAX_GATES) return JMOE_EINVAL;
+    if (E < 1 || E > 64 || top_k < 1 || top_k > 4 || top_k > E) return JMOE_EUNSUPPORTED;
+    if (T == 0) return JMOE_OK;
+    if (!w_router || !topk_ids || !topk_w) return JMOE_EINVAL;
+    if (!aligned16(w_router) || !aligned16(topk_ids) || !aligned16(topk_w) ||
+        (bias && !aligned16(bias)) || (logits && !aligned16(logits)))
+        return JMOE_EALIGN;
+    const int renorm = (flags & JMOE_ROUTE_SOFTMAX_GATES) ? 0 : 1;
+    return from_cuda(jmoe::launch_norm_route(x_bf16, T, d, gamma_bf16, eps, y_bf16, w_router, bias,
+                                             E, top_k, renorm, topk_ids, topk_w, logits, num_sms(),
+                                             (cudaStream_t)stream));
 }
 
 jmoe_status jmoe_permute(const int32_t* topk_ids, int64_t T, int32_t top_k, int32_t E,

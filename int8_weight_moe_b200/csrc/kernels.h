@@ -36,6 +36,15 @@ cudaError_t launch_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8
 cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
                          const float* bias, int E, int top_k, int renorm, int32_t* ids,
                          float* gates, float* logits, int num_sms, cudaStream_t stream);
+// RMSNorm y = bf16((x * r) * gamma), r = 1/sqrt(mean(x^2) + eps) (fp64, fixed order).
+cudaError_t launch_rmsnorm(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                           float eps, void* y_bf16, int num_sms, cudaStream_t stream);
+// Router on the RMS-normalised rows (written to y_bf16); gamma_bf16 == nullptr
+// routes x itself (as launch_route).
+cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                              float eps, void* y_bf16, const float* w_router, const float* bias,
+                              int E, int top_k, int renorm, int32_t* ids, float* gates,
+                              float* logits, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_t* offsets,
                            int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,

@@ -70,6 +70,25 @@ __device__ void select_topk(const float* l, int64_t t, int E, int top_k, int ren
     }
 }
 
+// RMSNorm of one bf16 row held by a warp's lanes in the canonical order:
+// ss = sum of x_k^2 with lane j summing k = j (mod 32) ascending and the
+// halving tree over the lanes (squares of bf16 values are exact in fp64),
+// r = 1 / sqrt(ss / d + eps), each step one IEEE-rounded fp64 operation (no
+// fused multiply-adds), so the result matches a plain fp64 evaluation.
+__device__ __forceinline__ double rms_inv(double lane_sum, int64_t d, float eps) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) lane_sum += __shfl_down_sync(0xffffffffu, lane_sum, o);
+    const double ss = __shfl_sync(0xffffffffu, lane_sum, 0);
+    return __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, (double)d), (double)eps)));
+}
+
+// y_k = bf16((x_k * r) * gamma_k), rounded once from fp64.
+__device__ __forceinline__ uint16_t rms_apply(uint16_t x, double r, uint16_t g) {
+    const double v = __dmul_rn(__dmul_rn((double)bf16_bits_to_f32(x), r),
+                               (double)bf16_bits_to_f32(g));
+    return __bfloat16_as_ushort(__double2bfloat16(v));
+}
+
 // Few tokens, very wide rows: one CTA of 16 warps per token, warp w computing
 // experts w, w + 16, ... (same per-lane order and halving tree).  The token
 // row is staged in shared memory once; each warp streams its expert's router
@@ -143,10 +162,15 @@ constexpr int kRouteCluster = 4;
 constexpr int kExpertsPerCta = kGroupE / kRouteCluster;
 constexpr size_t kClusterMaxSmem = 200 * 1024;
 
+// kNorm: the token row is RMS-normalised in shared memory first (every CTA
+// of the cluster computes the same r; the first one writes the normalised
+// row to y) and the logits are taken of the normalised row.
+template <bool kNorm>
 __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExpertsPerCta * 32)
     k_route_cluster(const uint16_t* __restrict__ x, int64_t d, const float* __restrict__ wr,
                     const float* __restrict__ bias, int E, int top_k, int renorm,
-                    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits) {
+                    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits,
+                    const uint16_t* __restrict__ gamma, float eps, uint16_t* __restrict__ y) {
     namespace cg = cooperative_groups;
     extern __shared__ __align__(16) uint8_t route_smem[];
     float* s_w = reinterpret_cast<float*>(route_smem);  // [kExpertsPerCta][d]
@@ -173,6 +197,26 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
     for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
         *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
     __syncthreads();
+    if (kNorm) {
+        __shared__ double s_r;
+        if (warp == 0) {
+            double acc = 0.0;
+            for (int64_t k = lane; k < d; k += 32) {
+                const double v = (double)bf16_bits_to_f32(s_x[k]);
+                acc = __dadd_rn(acc, __dmul_rn(v, v));
+            }
+            const double r = rms_inv(acc, d, eps);
+            if (lane == 0) s_r = r;
+        }
+        __syncthreads();
+        const double r = s_r;
+        for (int64_t k = threadIdx.x; k < d; k += blockDim.x) {
+            const uint16_t v = rms_apply(s_x[k], r, gamma[k]);
+            s_x[k] = v;
+            if (rank == 0) y[t * d + k] = v;
+        }
+        __syncthreads();
+    }
     float* dst = cluster.map_shared_rank(s_logit, 0);
     auto logit_of_row = [&](int e) {
         cp_async_wait<0>();
@@ -199,6 +243,24 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
     }
     cluster.sync();
     if (rank == 0 && threadIdx.x == 0) select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
+}
+
+// One warp per token.
+__global__ void __launch_bounds__(256)
+    k_rmsnorm(const uint16_t* __restrict__ x, int64_t T, int64_t d, const uint16_t* __restrict__ gamma,
+              float eps, uint16_t* __restrict__ y) {
+    const int lane = threadIdx.x & 31;
+    for (int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); t < T;
+         t += (int64_t)gridDim.x * 8) {
+        const uint16_t* xr = x + t * d;
+        double acc = 0.0;
+        for (int64_t k = lane; k < d; k += 32) {
+            const double v = (double)bf16_bits_to_f32(xr[k]);
+            acc = __dadd_rn(acc, __dmul_rn(v, v));
+        }
+        const double r = rms_inv(acc, d, eps);
+        for (int64_t k = lane; k < d; k += 32) y[t * d + k] = rms_apply(xr[k], r, gamma[k]);
+    }
 }
 
 // Many tokens: a CTA of 4 warps handles kTok tokens; for each group of 16
@@ -273,25 +335,58 @@ __global__ void __launch_bounds__(kWarps * 32)
 cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* w_router,
                          const float* bias, int E, int top_k, int renorm, int32_t* ids,
                          float* gates, float* logits, int num_sms, cudaStream_t stream) {
+    return launch_norm_route(x_bf16, T, d, nullptr, 0.0f, nullptr, w_router, bias, E, top_k,
+                             renorm, ids, gates, logits, num_sms, stream);
+}
+
+cudaError_t launch_rmsnorm(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                           float eps, void* y_bf16, int num_sms, cudaStream_t stream) {
     if (T == 0) return cudaSuccess;
-    // Few tokens: a cluster of 4 CTAs per token (or, for very wide rows, a
-    // 16-warp CTA streaming the router rows in chunks); many tokens: 4 tokens
-    // per 4-warp CTA, which cuts the router-weight traffic fourfold.
+    int64_t blocks = (T + 7) / 8;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    k_rmsnorm<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(x_bf16), T, d,
+                                                   static_cast<const uint16_t*>(gamma_bf16), eps,
+                                                   static_cast<uint16_t*>(y_bf16));
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
+                              float eps, void* y_bf16, const float* w_router, const float* bias,
+                              int E, int top_k, int renorm, int32_t* ids, float* gates,
+                              float* logits, int num_sms, cudaStream_t stream) {
+    if (T == 0) return cudaSuccess;
+    const bool norm = gamma_bf16 != nullptr;
+    // Few tokens: a cluster of 4 CTAs per token, the RMSNorm (if any) fused in
+    // front of the logits (or, for very wide rows, a 16-warp CTA streaming the
+    // router rows in chunks); many tokens: 4 tokens per 4-warp CTA, which cuts
+    // the router-weight traffic fourfold.  Outside the fused kernel the
+    // RMSNorm runs first, into y, and the router reads y.
     const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
     const size_t smem = (size_t)kGroupE * kChunkSmem + (size_t)d * sizeof(uint16_t);
     if (T < (int64_t)num_sms * 8 && csmem <= kClusterMaxSmem && T * kRouteCluster < (1LL << 31)) {
+        const auto kernel = norm ? k_route_cluster<true> : k_route_cluster<false>;
         const cudaError_t e = cudaFuncSetAttribute(
-            k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
+            kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(k_route_cluster, dim3((unsigned)(T * kRouteCluster)),
-                          dim3(kExpertsPerCta * 32), csmem, stream, (const uint16_t*)x_bf16, d,
-                          w_router, bias, E, top_k, renorm, ids, gates, logits);
-    } else if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
+        return launch_pdl(kernel, dim3((unsigned)(T * kRouteCluster)), dim3(kExpertsPerCta * 32),
+                          csmem, stream, (const uint16_t*)x_bf16, d, w_router, bias, E, top_k,
+                          renorm, ids, gates, logits, (const uint16_t*)gamma_bf16, eps,
+                          (uint16_t*)y_bf16);
+    }
+    const void* xr = x_bf16;
+    if (norm) {
+        const cudaError_t e = launch_rmsnorm(x_bf16, T, d, gamma_bf16, eps, y_bf16, num_sms, stream);
+        if (e != cudaSuccess) return e;
+        xr = y_bf16;
+    }
+    if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);
         if (e != cudaSuccess) return e;
         k_route_wide<<<(unsigned)T, kGroupE * 32, smem, stream>>>(
-            (const uint16_t*)x_bf16, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
+            (const uint16_t*)xr, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         note_launch();
     } else {
         int64_t blocks = (T + 3) / 4;
@@ -299,12 +394,10 @@ cudaError_t launch_route(const void* x_bf16, int64_t T, int64_t d, const float* 
         if (blocks > cap) blocks = cap;
         if (E <= kGroupE)
             k_route<4, false><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-                (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, renorm, ids, gates,
-                logits);
+                (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         else
             k_route<4, true><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-                (const uint16_t*)x_bf16, T, d, w_router, bias, E, top_k, renorm, ids, gates,
-                logits);
+                (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         note_launch();
     }
     return cudaGetLastError();

@@ -69,5 +69,11 @@ LARGE_DECODE = Workload("large_decode_T32_d8192_f24576_E16_top2", 3, 32, 8192, 2
 LARGE_PREFILL_SKEW = Workload("large_prefill_skewed_T8192_d8192_f24576_E16_top2", 4, 8192, 8192,
                               24576, bias=_skew(16), regime="prefill")
 
-ALL = [TINY, MINI_DECODE, MINI_PREFILL, MINI_DENSE, LARGE_DECODE, LARGE_PREFILL_SKEW]
+# generalised routing at Mini size: 64 experts, top-4 (a wider MoE, as in the
+# routing settings the layer also supports)
+MINI_DECODE_E64 = Workload("mini_decode_T8_d4096_f14336_E64_top4", 5, 8, 4096, 14336, E=64,
+                           top_k=4)
+
+ALL = [TINY, MINI_DECODE, MINI_PREFILL, MINI_DENSE, LARGE_DECODE, LARGE_PREFILL_SKEW,
+       MINI_DECODE_E64]
 BY_NAME = {w.name: w for w in ALL}

@@ -375,3 +375,63 @@ def test_forward_generalised_routing(E, top_k, T, path):
     ref = ora.forward_tokens(tokens, io, go)
     assert_close(bf16_to_f64(out)[tokens], ref, f"E={E} top_k={top_k}")
     assert jm.jmoe_last_error() == jm.JMOE_OK
+
+
+# ----------------------------------------------------------------------------- RMSNorm prologue
+
+
+def _bits(t):
+    """bf16 bit patterns of a torch bf16 tensor, as uint16."""
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _norm_inputs(T, d, seed=16):
+    x = synth.normal_bf16_gpu(seed, synth.X, 2.0, (T, d))
+    g = synth.normal_bf16_gpu(seed + 1, synth.X, 0.25, (d,))
+    g = (g.float() + 1.0).to(torch.bfloat16)  # gamma around 1
+    return x, g
+
+
+@pytest.mark.parametrize("T,d", [(37, 256), (1300, 4096), (2, 16384)])
+def test_rmsnorm_bitexact(T, d):
+    x, g = _norm_inputs(T, d)
+    y = jm.jmoe_rmsnorm(x, g, 1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.rmsnorm(_bits(x), _bits(g), 1e-5)
+    assert np.array_equal(_bits(y), ref)
+
+
+@pytest.mark.parametrize("T,d,E,top_k", [(8, 4096, 16, 2), (37, 256, 64, 4), (1300, 256, 16, 2),
+                                         (3, 12288, 16, 2)],
+                         ids=["fused", "fused_E64", "many_tokens", "wide_rows"])
+def test_rmsnorm_route_bitexact(T, d, E, top_k):
+    x, g = _norm_inputs(T, d, seed=17)
+    wr = synth.normal_f32_gpu(18, synth.WR, 0.02, (E, d))
+    xn, ids, gates, logits = jm.jmoe_rmsnorm_route(x, g, 1e-6, wr, top_k, want_logits=True)
+    torch.cuda.synchronize()
+    xn_ref = oracle.rmsnorm(_bits(x), _bits(g), 1e-6)
+    assert np.array_equal(_bits(xn), xn_ref)
+    lo, io, go = oracle.route(xn_ref, wr.cpu().numpy(), top_k)
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert np.abs(gates.cpu().numpy().astype(np.float64) - go).max() <= 4e-6
+
+
+@pytest.mark.parametrize("norm", [False, True], ids=["route", "rmsnorm_route"])
+def test_layer_graph_matches_eager(norm):
+    dev = DeviceLayer(TINY)
+    desc = dev.desc(jm.JMOE_PATH_AUTO)
+    g = _norm_inputs(1, TINY.d_model)[1] if norm else None
+    graph = jm.MoeLayerGraph(desc, dev.w_router, TINY.T, gamma=g, eps=1e-6)
+    for seed in (31, 32):
+        x = synth.normal_bf16_gpu(seed, synth.X, 1.0, (TINY.T, TINY.d_model))
+        out = graph.run(x).clone()
+        if norm:
+            xn, ids, gates = jm.jmoe_rmsnorm_route(x, g, 1e-6, dev.w_router, TINY.top_k)
+        else:
+            xn = x
+            ids, gates = jm.jmoe_route(x, dev.w_router, TINY.top_k)
+        ref = jm.jmoe_forward(desc, xn, ids, gates)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    assert jm.jmoe_last_error() == jm.JMOE_OK

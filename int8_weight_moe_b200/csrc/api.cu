@@ -193,7 +193,6 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         a.split_gu = w.split_gu; a.split_d = w.split_d;
         a.x16 = at(w.x16); a.xexp = static_cast<int32_t*>(at(w.xexp));
         a.hmax = static_cast<int32_t*>(at(w.hmax));
-        a.max_per_expert = T;  // distinct experts per token: at most T rows each
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;
         a.err = err;

@@ -59,17 +59,12 @@ constexpr int kMaxE = 64;
 
 enum { kGateUp = 0, kDown = 1 };
 
-// x (or h) fragment for one token row: 16 consecutive bf16 starting at p.
+// x (or h) fragment for one token row: 16 consecutive fp16 starting at p.
 __device__ __forceinline__ void load_b(const uint16_t* p, uint32_t (&b)[8]) {
-    if (p) {
-        const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(p));
-        const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(p + 8));
-        b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
-        b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = 0u;
-    }
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(p + 8));
+    b[0] = v0.x; b[1] = v0.y; b[2] = v0.z; b[3] = v0.w;
+    b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
 }
 
 // Four MMA steps of one 64-wide k-block: rows g (q0) and g+8 (q1).  Even and
@@ -146,6 +141,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     __shared__ uint64_t full[kWarpsPerBlock][kSlots];
     __shared__ int s_start[kMaxE + 1];  // first item of expert e
     __shared__ int s_off[kMaxE + 1];
+    __shared__ int s_np[kMaxE];         // passes of expert e
     __shared__ int s_abort;
     pdl_wait();
     pdl_launch_dependents();
@@ -169,9 +165,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     if (threadIdx.x == 0) {
         int run = 0;
         for (int e = 0; e < E; ++e) {
-            const int cnt = s_off[e + 1] - s_off[e];
+            const int np = (s_off[e + 1] - s_off[e] + 8 * NCH - 1) / (8 * NCH);
+            s_np[e] = np;
             s_start[e] = run;
-            run += cnt > 0 ? (cnt + 8 * NCH - 1) / (8 * NCH) * groups * S : 0;
+            run += np * groups * S;
         }
         s_start[E] = run;
     }
@@ -186,24 +183,34 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int64_t total = (int64_t)n_mine * nsl;
     if (total == 0) return;
 
-    auto item_of = [&](int it) {
+    // The warp's it-th item.  Items come in increasing order, so each cursor
+    // (producer, consumer) keeps its expert `e` and only moves it forward; the
+    // search stops below E because every index is below s_start[E].  The
+    // passes of one (unit, piece) are neighbours, so the warps that read the
+    // same weights run side by side and all but one hit in L2.
+    auto item_at = [&](int it, int& e) {
         const int idx = wid + it * W;
-        int e = 0;
-        while (e + 1 < E && s_start[e + 1] <= idx) ++e;
+        while (s_start[e + 1] <= idx) ++e;
         const int local = idx - s_start[e];
+        const int np = s_np[e];
+        int rest = local;
         Item r;
         r.e = e;
-        r.z = local % S;
-        r.group = (local / S) % groups;
-        r.pass = local / S / groups;
+        r.pass = 0;
+        if (np > 1) {
+            r.pass = local % np;
+            rest = local / np;
+        }
+        r.z = rest % S;
+        r.group = rest / S;
         return r;
     };
 
     // ---- producer cursor (lane 0 issues the TMA boxes of slot-sized pieces)
-    int pi = 0, pj = 0;
+    int pe = 0, pi = 0, pj = 0;
     int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
     auto set_prefetch_item = [&](int it) {
-        const Item u = item_of(it);
+        const Item u = item_at(it, pe);
         prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16
                                : u.e * (int)p.d + u.group * unit_rows<MODE>();
         pk = u.z * kb_item * 64;
@@ -230,7 +237,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     for (int q = 0; q < kSlots - 1; ++q)
         if (q < total) issue(q);
 
-    // ---- consumer state: activation fragments are loaded one slot ahead
+    // ---- consumer state: activation fragments are loaded one slot ahead,
+    // into the one of two register buffers the current slot does not use
     float acc[NCH][NMAT][2][4];
 #pragma unroll
     for (int n = 0; n < NCH; ++n)
@@ -243,63 +251,57 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         int base, cnt_pass;
         const uint16_t* b[NCH];
     };
+    int ce = 0;
     auto make_cur = [&](int it) {
         Cur r;
-        r.u = item_of(it);
+        r.u = item_at(it, ce);
         r.base = s_off[r.u.e] + r.u.pass * 8 * NCH;
         r.cnt_pass = min(8 * NCH, s_off[r.u.e + 1] - r.base);
         const int64_t kz = (int64_t)r.u.z * kb_item * 64;
 #pragma unroll
         for (int n = 0; n < NCH; ++n) {
-            const int slot = n * 8 + g8;
-            if (slot < r.cnt_pass) {
-                const int64_t row = MODE == kGateUp ? (int64_t)(p.perm[r.base + slot] / p.top_k)
-                                                    : (int64_t)(r.base + slot);
-                r.b[n] = p.b_src + row * K + 16 * c + kz;
-            } else {
-                r.b[n] = nullptr;
-            }
+            // A column without a token reads the pass's first row instead: the
+            // MMA keeps columns apart and that output column is never stored.
+            const int slot = n * 8 + g8 < r.cnt_pass ? n * 8 + g8 : 0;
+            const int64_t row = MODE == kGateUp ? (int64_t)(p.perm[r.base + slot] / p.top_k)
+                                                : (int64_t)(r.base + slot);
+            r.b[n] = p.b_src + row * K + 16 * c + kz;
         }
         return r;
     };
-    uint32_t bn[kNB][NCH][8];
-    auto load_slot_b = [&](const Cur& r, int j) {
+    using Frag = uint32_t[kNB][NCH][8];
+    auto load_slot_b = [&](const Cur& r, int j, Frag& dst) {
 #pragma unroll
-        for (int b = 0; b < kNB; ++b)
+        for (int b = 0; b < kNB; ++b) {
+            // a k-block past the item's end (odd count) is read but not used
+            const int kb = min(j * kNB + b, kb_item - 1);
 #pragma unroll
-            for (int n = 0; n < NCH; ++n) {
-                const int kb = j * kNB + b;
-                load_b(r.b[n] && kb < kb_item ? r.b[n] + kb * 64 : nullptr, bn[b][n]);
-            }
+            for (int n = 0; n < NCH; ++n) load_b(r.b[n] + kb * 64, dst[b][n]);
+        }
     };
+    Frag fa, fb;
     Cur cur = make_cur(0), nxt{};
-    load_slot_b(cur, 0);
+    load_slot_b(cur, 0, fa);
     int ci = 0, cj = 0, cslot = 0;
     uint32_t cphase = 0;
     bool ok = true;
-    for (int64_t q = 0; q < total && ok; ++q) {
-        // refill the slot consumed in the previous iteration
+    // Slot q: refill the slot consumed by q-1, fetch the fragments of q+1 into
+    // `fnext`, wait for q's weights and multiply them with `fcur`.
+    auto step = [&](int64_t q, const Frag& fcur, Frag& fnext) {
         if (q + kSlots - 1 < total) {
             __syncwarp();
             if (lane == 0) sm100::fence_proxy_async_smem();
             issue((int)((q + kSlots - 1) % kSlots));
         }
-        uint32_t bc[kNB][NCH][8];
-#pragma unroll
-        for (int b = 0; b < kNB; ++b)
-#pragma unroll
-            for (int n = 0; n < NCH; ++n)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) bc[b][n][i] = bn[b][n][i];
         if (cj + 1 < nsl) {
-            load_slot_b(cur, cj + 1);
+            load_slot_b(cur, cj + 1, fnext);
         } else if (ci + 1 < n_mine) {
             nxt = make_cur(ci + 1);
-            load_slot_b(nxt, 0);
+            load_slot_b(nxt, 0, fnext);
         }
         if (!sm100::mbar_wait(&full[warp][cslot], cphase, abort)) {
             ok = false;
-            break;
+            return;
         }
         const uint8_t* src = ring + cslot * kSlotBytes + g8 * 64 + 16 * c;
 #pragma unroll
@@ -314,8 +316,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int n = 0; n < NCH; ++n) {
                     if (n * 8 < cur.cnt_pass) {
-                        mma_block<true>(acc[n][0], wq[0], wq[1], bc[b][n]);
-                        mma_block<true>(acc[n][1], wq[2], wq[3], bc[b][n]);
+                        mma_block<true>(acc[n][0], wq[0], wq[1], fcur[b][n]);
+                        mma_block<true>(acc[n][1], wq[2], wq[3], fcur[b][n]);
                     }
                 }
             }
@@ -346,6 +348,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             cj = 0;
             if (++ci < n_mine) cur = nxt;
         }
+    };
+    for (int64_t q = 0; q < total; q += 2) {
+        step(q, fa, fb);
+        if (!ok || q + 1 >= total) break;
+        step(q + 1, fb, fa);
+        if (!ok) break;
     }
     // leave only when no copy is still landing in this warp's ring
     if (lane == 0) {
@@ -697,8 +705,10 @@ cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (a.T == 0) return cudaSuccess;
-    cudaError_t err = a.max_per_expert <= 8 ? launch_decode_nch<1>(a, stream)
-                                            : launch_decode_nch<2>(a, stream);
+    // One 8-token tile per pass: a 16-token tile needs 167 registers per
+    // thread (3 CTAs per SM instead of 4), which costs more than the extra
+    // passes of experts with more than 8 tokens, whose weights come from L2.
+    cudaError_t err = launch_decode_nch<1>(a, stream);
     if (err != cudaSuccess) return err;
     if (a.mark) a.mark(4, false, stream);
     err = launch_pdl(k_combine,

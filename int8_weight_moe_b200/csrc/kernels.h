@@ -79,7 +79,6 @@ struct DecodeArgs {
     float* P_gu;          // fp32 [split_gu][A][2f] partial sums (workspace)
     float* P_d;           // fp32 [split_d][A][d] partial sums (workspace; may alias P_gu)
     int split_gu, split_d;   // K pieces of the two GEMVs
-    int64_t max_per_expert;  // host-side bound used to size register tiles
     void* out;            // bf16 [T][d]
     int num_sms;
     StageMark mark;

@@ -67,6 +67,11 @@ __device__ __forceinline__ void load_b(const uint16_t* p, uint32_t (&b)[8]) {
     b[4] = v1.x; b[5] = v1.y; b[6] = v1.z; b[7] = v1.w;
 }
 
+// Bring the 128-byte line at p into L1 without waiting for it.
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // Four MMA steps of one 64-wide k-block: rows g (q0) and g+8 (q1).  Even and
 // odd steps accumulate into separate tiles (two independent MMA chains).
 // F16: weights converted to fp16 and fp16 MMA (activation operand in fp16);
@@ -298,6 +303,17 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         } else if (ci + 1 < n_mine) {
             nxt = make_cur(ci + 1);
             load_slot_b(nxt, 0, fnext);
+        }
+        // Warm L1 with the activation lines of slot q+2 (one per row and
+        // k-block; a prefetch holds no register).  While the weight stream
+        // keeps DRAM busy an L2 hit takes longer than one slot, so without
+        // this the loads above wait whenever several token rows share a pass.
+        if (cj + 2 < nsl && c == 0) {
+#pragma unroll
+            for (int b = 0; b < kNB; ++b)
+#pragma unroll
+                for (int n = 0; n < NCH; ++n)
+                    prefetch_l1(cur.b[n] + min((cj + 2) * kNB + b, kb_item - 1) * 64);
         }
         if (!sm100::mbar_wait(&full[warp][cslot], cphase, abort)) {
             ok = false;

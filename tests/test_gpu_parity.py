@@ -14,8 +14,8 @@ import oracle
 import synth
 from exact import bf16_bits
 from layers import DeviceLayer, OracleLayer, assert_close, bf16_to_f64
-from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DENSE,
-                             MINI_PREFILL, TINY, Workload)
+from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DECODE_E64,
+                             MINI_DENSE, MINI_PREFILL, TINY, Workload)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -200,6 +200,18 @@ def test_forward_large_decode_sampled():
     tokens = [0, 31]
     ref = ora.forward_tokens(tokens, io, go)
     assert_close(bf16_to_f64(out)[tokens], ref, "large decode")
+
+
+def test_forward_e64_top4_sampled():
+    # Mini sizes with 64 experts and top-4, the bench's launch configuration
+    dev, ora = DeviceLayer(MINI_DECODE_E64), OracleLayer(MINI_DECODE_E64)
+    ids, g, out = run_layer(dev)
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert np.allclose(g.cpu().numpy(), go, rtol=0, atol=4e-6)
+    tokens = [0, 7]
+    ref = ora.forward_tokens(tokens, io, go)
+    assert_close(bf16_to_f64(out)[tokens], ref, MINI_DECODE_E64.name)
 
 
 @pytest.mark.parametrize("wl,tokens", [

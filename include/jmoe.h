@@ -50,7 +50,7 @@ typedef enum {
     JMOE_OK = 0,
     JMOE_EINVAL = 1,       /* a null pointer, a negative size, an out-of-range count */
     JMOE_EALIGN = 2,       /* a pointer is not 16-byte aligned */
-    JMOE_EUNSUPPORTED = 3, /* a shape or option this build does not implement */
+    JMOE_EUNSUPPORTED = 3, /* a shape or option this library does not implement */
     JMOE_EWORKSPACE = 4,   /* workspace smaller than the size query returned */
     JMOE_ECUDA = 5,        /* a CUDA runtime call or launch failed */
     JMOE_ETIMEOUT = 6,     /* (device word) a bounded wait inside a kernel ran out */

@@ -184,6 +184,32 @@ class Layer:
     def weight_bytes(self):
         return self.w_gu.numel() + self.w_d.numel()
 
+    def expert_counts(self):
+        """Token->expert assignments per expert in the last routing."""
+        if self.wl.dense:
+            return np.array([self.wl.T])
+        return np.bincount(self.ids.cpu().numpy().reshape(-1), minlength=self.wl.E)
+
+
+def dequant_conversions(counts, d: int, f: int, prefill: bool) -> int:
+    """INT8 -> 16-bit weight conversions one step of the expert kernels makes
+    (the dequantisation work, reported apart from the FLOPs).  The decode
+    kernels convert an expert's 3*d*f weights once per pass over up to 8 of
+    its tokens; the tensor-core kernels once per 256-row tile of its rows,
+    which are padded to a multiple of 128."""
+    total = 0
+    for c in counts:
+        c = int(c)
+        if c <= 0:
+            continue
+        if prefill:
+            padded = -(-c // 128) * 128
+            passes = -(-padded // 256)
+        else:
+            passes = -(-c // 8)
+        total += passes * 3 * d * f
+    return total
+
 
 def kernel_work(layer: Layer):
     """Algorithmic work of the dominant kernel (the gate/up GEMM) per launch
@@ -198,8 +224,11 @@ def kernel_work(layer: Layer):
     touched = layer.touched_experts()
     gu_bytes = touched * 2 * f * d + T * d * 2
     step_bytes = touched * 3 * d * f + touched * (2 * f + d) * 4 + T * d * 2 * 2
+    conv = dequant_conversions(layer.expert_counts(), d, f, layer.prefill_path())
     return {"touched": touched, "gate_up_bytes": gu_bytes, "step_bytes": step_bytes,
-            "gate_up_flops": 4 * A * d * f, "step_flops": 6 * A * d * f}
+            "gate_up_flops": 4 * A * d * f, "step_flops": 6 * A * d * f,
+            "dequant": {"int8_conversions_per_step": conv,
+                        "per_touched_weight": round(conv / (touched * 3 * d * f), 3)}}
 
 
 def _primed_events(n: int):
@@ -619,7 +648,8 @@ def main():
                      "stages_ms": {k: round(v, 4) for k, v in bd.items()},
                      "roofline": roofline_entry(lay, st, peaks),
                      "step_hbm_gbs": round(w2["step_bytes"] / (oms * 1e-3) / 1e9, 1),
-                     "step_tflops": round(w2["step_flops"] / (oms * 1e-3) / 1e12, 2)}
+                     "step_tflops": round(w2["step_flops"] / (oms * 1e-3) / 1e12, 2),
+                     "dequant": w2["dequant"]}
             also.append(entry)
             del lay
             torch.cuda.empty_cache()
@@ -646,7 +676,8 @@ def main():
                                     "around every stage (the timed pass records only the "
                                     "gate/up pair)",
                 "step_hbm_gbs": round(step_gbs, 1),
-                "touched_experts": work["touched"], "graph": graph_line, "also": also}
+                "touched_experts": work["touched"], "dequant": work["dequant"],
+                "graph": graph_line, "also": also}
         print(json.dumps(line), flush=True)
     if dist_on:
         import torch.distributed as dist

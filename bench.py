@@ -242,14 +242,22 @@ def _primed_events(n: int):
     return evs
 
 
+def step_percentiles(ms_list):
+    """Median, 10th and 90th percentile of per-step times (ms)."""
+    xs = np.asarray(ms_list, dtype=np.float64)
+    return {"median": round(float(np.median(xs)), 4), "p10": round(float(np.percentile(xs, 10)), 4),
+            "p90": round(float(np.percentile(xs, 90)), 4)}
+
+
 def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool,
-              stages=("gate_up",), route: bool = False):
+              stages=("gate_up",), route: bool = False, spread=None):
     """Warm-up, then exactly `steps` timed steps between barriers.  Inside the
     timed region the library records a CUDA event pair on the launching
     stream around each stage named in `stages` (and the bench around the
     router if `route`); the other stages record nothing, so the step pays
     only for the events it needs.  Returns (total ms, mean ms per recorded
-    stage that ran, kernel launches in the timed region)."""
+    stage that ran, kernel launches in the timed region); if `spread` is a
+    dict, it receives the per-step percentiles of each recorded stage."""
     import torch
 
     import int8_weight_moe_b200 as jm
@@ -297,7 +305,10 @@ def timed_run(layer: Layer, steps: int, warmup: int, dist_on: bool,
         # a stage that does not run on this path leaves its primed pair, which
         # spans no step: report only stages whose events moved
         if stage_ran(pairs, start):
-            out[jm.STAGES[i]] = sum(a.elapsed_time(b) for a, b in pairs) / len(pairs)
+            per_step = [a.elapsed_time(b) for a, b in pairs]
+            out[jm.STAGES[i]] = sum(per_step) / len(per_step)
+            if spread is not None:
+                spread[jm.STAGES[i]] = step_percentiles(per_step)
     return total_ms, out, launches
 
 
@@ -615,13 +626,17 @@ def main():
 
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, stages, launches = timed_run(layer, args.steps, args.warmup, dist_on)
+    spread = {}
+    total_ms, stages, launches = timed_run(layer, args.steps, args.warmup, dist_on, spread=spread)
     clocks = sampler.stop()
     dev = torch.device("cuda", local)
     total_ms = max_over_ranks(total_ms, dev)
     ms = total_ms / args.steps
     value = whole_job_tokens_per_s(world, wl.T, ms)
     roof = roofline_entry(layer, stages, peaks)
+    if roof is not None and "gate_up" in spread:
+        # the dominant kernel's per-launch spread over the timed steps
+        roof["ms_per_launch"] = spread["gate_up"]
     breakdown = stage_breakdown(layer, min(args.steps, 50), dist_on)
     e2e = e2e_run(layer, max(args.steps // 2, 10), 3, dist_on)
     e2e_ms = max_over_ranks(e2e["ms_per_step"], dev)

@@ -1,7 +1,7 @@
-"""bench.py's algorithmic-work accounting, on CPU: the bytes and FLOPs the
-roofline divides by, and the dequantisation work reported beside them (INT8
-weight conversions per step), for hand-made routings whose answers follow
-from the tile rules by hand."""
+"""bench.py's host arithmetic, on CPU: the bytes and FLOPs the roofline
+divides by, the dequantisation work reported beside them (INT8 weight
+conversions per step) for hand-made routings whose answers follow from the
+tile rules by hand, and the per-step percentiles of the dominant kernel."""
 import types
 
 import numpy as np
@@ -67,3 +67,9 @@ def test_kernel_work_dense_layer():
     tiles = -(-(-(-wl.T // 128) * 128) // 256)
     assert w["dequant"]["int8_conversions_per_step"] == tiles * 3 * wl.d_model * wl.d_ff
     assert np.isclose(w["dequant"]["per_touched_weight"], tiles)
+
+
+def test_step_percentiles():
+    p = bench.step_percentiles([float(v) for v in range(1, 102)])  # 1..101
+    assert p == {"median": 51.0, "p10": 11.0, "p90": 91.0}
+    assert bench.step_percentiles([0.25]) == {"median": 0.25, "p10": 0.25, "p90": 0.25}

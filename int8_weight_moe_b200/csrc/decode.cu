@@ -26,15 +26,17 @@
 // 16c + 4s + {2,3} for columns 2c+8, 2c+9.
 //
 // Work decomposition: every warp is an independent streaming worker.  A work
-// item is (touched expert, 16 output channels, one pass of up to 8*NCH
-// tokens, one K piece of S): a slab of 16 rows (gate/up: 16 gate + the same
-// 16 up rows) x K/S bytes.  Items are small (16-32 KB) and dealt round-robin
-// to all warps of the GPU, the K pieces of a unit to neighbouring warps, so
-// the warps finish together and the rows being read at any moment are few
-// and shared by several warps (DRAM rows stay open for more of their bytes).
+// item is (touched expert, one unit of output channels, one pass of up to 8
+// tokens, one K piece of S): two 16-row matrices x K/S bytes (gate/up: 16
+// gate rows and the same 16 up rows; down: the two halves of 32 output
+// rows).  Items (32-112 KB at Mini sizes) are dealt round-robin to all warps
+// of the GPU, the K pieces and passes of a unit to neighbouring warps, so the
+// warps finish together and the rows being read at any moment are few and
+// shared by several warps (DRAM rows stay open for more of their bytes).
 // Each warp keeps a ring of 4 KB slots in its own shared memory, filled by
 // TMA two slots ahead of use and across item boundaries, with the matching
-// activation fragments loaded one slot ahead; there are no barriers.  An
+// activation fragments loaded one slot ahead (their lines prefetched into L1
+// two slots ahead); there are no barriers.  An
 // item stores its raw fp32 partial sums; the small follow-up kernels add the
 // S pieces in a fixed order (deterministic) and apply scales, SwiGLU, gates.
 // (Finishing units inside the streaming warps instead -- a counter per unit,

@@ -53,8 +53,9 @@ class Oracle:
     """
 
     def __init__(self, so_path: str = _SO):
-        if so_path == _SO and not os.path.exists(_SO):
-            build()
+        if so_path == _SO and (not os.path.exists(_SO) or
+                               os.path.getmtime(_SO) < os.path.getmtime(SOURCE)):
+            build()  # missing, or older than its source (a stale signature would crash)
         lib = ctypes.CDLL(so_path)
         vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         lib.oracle_quantize.argtypes = [vp, i64, i64, vp, vp]
@@ -70,9 +71,9 @@ class Oracle:
         lib.oracle_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp]
         lib.oracle_permute.restype = None
         lib.oracle_moe_forward.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp,
-                                           i32, vp]
+                                           vp]
         lib.oracle_moe_forward.restype = ctypes.c_int
-        lib.oracle_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, i32, vp]
+        lib.oracle_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         lib.oracle_mlp_forward.restype = None
         self.lib = lib
 
@@ -145,8 +146,8 @@ class Oracle:
 
     def moe_forward(self, x_bits: np.ndarray, ids: np.ndarray, gates: np.ndarray,
                     q_gu: Sequence[Optional[np.ndarray]], s_gu: Sequence[Optional[np.ndarray]],
-                    q_d: Sequence[Optional[np.ndarray]], s_d: Sequence[Optional[np.ndarray]],
-                    round_h_bf16: bool = False) -> np.ndarray:
+                    q_d: Sequence[Optional[np.ndarray]], s_d: Sequence[Optional[np.ndarray]]
+                    ) -> np.ndarray:
         """fp64 MoE output [T, d] = sum_j gates[t,j] * Expert_{ids[t,j]}(x_t).
 
         ``q_gu[e]`` is expert e's int8 gate/up matrix [2*d_ff, d] (gate rows
@@ -184,12 +185,12 @@ class Oracle:
         out = np.empty((T, d), dtype=np.float64)
         rc = self.lib.oracle_moe_forward(x.ctypes.data, T, d, f, E, k, i.ctypes.data,
                                          g.ctypes.data, t_qgu, t_sgu, t_qd, t_sd,
-                                         int(round_h_bf16), out.ctypes.data)
+                                         out.ctypes.data)
         if rc != 0:
             raise ValueError("oracle_moe_forward: a selected expert has no weights")
         return out
 
-    def mlp_forward(self, x_bits, q_gu, s_gu, q_d, s_d, round_h_bf16: bool = False) -> np.ndarray:
+    def mlp_forward(self, x_bits, q_gu, s_gu, q_d, s_d) -> np.ndarray:
         """fp64 dense SwiGLU MLP output [T, d] with INT8 weights (the E=1 entry)."""
         x = _c(x_bits, np.uint16)
         T, d = x.shape
@@ -198,8 +199,7 @@ class Oracle:
         f = qd.shape[1]
         out = np.empty((T, d), dtype=np.float64)
         self.lib.oracle_mlp_forward(x.ctypes.data, T, d, f, qgu.ctypes.data, sgu.ctypes.data,
-                                    qd.ctypes.data, sd.ctypes.data, int(round_h_bf16),
-                                    out.ctypes.data)
+                                    qd.ctypes.data, sd.ctypes.data, out.ctypes.data)
         return out
 
 
@@ -238,12 +238,12 @@ def permute(ids, E):
     return default().permute(ids, E)
 
 
-def moe_forward(x_bits, ids, gates, q_gu, s_gu, q_d, s_d, round_h_bf16=False):
-    return default().moe_forward(x_bits, ids, gates, q_gu, s_gu, q_d, s_d, round_h_bf16)
+def moe_forward(x_bits, ids, gates, q_gu, s_gu, q_d, s_d):
+    return default().moe_forward(x_bits, ids, gates, q_gu, s_gu, q_d, s_d)
 
 
-def mlp_forward(x_bits, q_gu, s_gu, q_d, s_d, round_h_bf16=False):
-    return default().mlp_forward(x_bits, q_gu, s_gu, q_d, s_d, round_h_bf16)
+def mlp_forward(x_bits, q_gu, s_gu, q_d, s_d):
+    return default().mlp_forward(x_bits, q_gu, s_gu, q_d, s_d)
 
 
 def tolerance_report(got: np.ndarray, ref: np.ndarray) -> dict:

@@ -50,20 +50,6 @@ static float bf16_to_f32(uint16_t b) {
     return f;
 }
 
-static double round_to_bf16(double v) {
-    /* round-to-nearest-even of an fp64 value to bfloat16 via fp32 (used only
-     * by the optional "bf16 hidden" variant that models the kernel's storage
-     * of h; the double rounding fp64->fp32->bf16 is the same one the GPU's
-     * fp32 accumulator goes through). */
-    float f = (float)v;
-    uint32_t u;
-    memcpy(&u, &f, 4);
-    u += 0x7fffu + ((u >> 16) & 1u);
-    u &= 0xffff0000u;
-    memcpy(&f, &u, 4);
-    return (double)f;
-}
-
 /* Round an fp64 value once, to nearest with ties to even, to the nearest     */
 /* bfloat16 (8 significant bits; fp32's exponent range, subnormals down to    */
 /* 2^-133); returns the bf16 bit pattern.  Scaling by powers of two and rint  */
@@ -251,8 +237,8 @@ void oracle_permute(const int32_t* ids, int64_t T, int top_k, int E, int32_t* of
 /*   h_n = silu(u_n) * u_{d_ff + n}                    n < d_ff               */
 /*   y_m = sum_n h_n * (q_d[m][n] * s_d[m])           m < d_model            */
 static void expert_ffn(const uint16_t* x, int64_t d, int64_t f, const int8_t* q_gu,
-                       const float* s_gu, const int8_t* q_d, const float* s_d, int round_h_bf16,
-                       double* u, double* h, double* y) {
+                       const float* s_gu, const int8_t* q_d, const float* s_d, double* u,
+                       double* h, double* y) {
     double* xd = (double*)malloc(sizeof(double) * (size_t)d);
     for (int64_t k = 0; k < d; ++k) xd[k] = (double)bf16_to_f32(x[k]);
 #pragma omp parallel for schedule(static)
@@ -266,7 +252,6 @@ static void expert_ffn(const uint16_t* x, int64_t d, int64_t f, const int8_t* q_
         double g = u[n];
         double silu = g / (1.0 + exp(-g));
         h[n] = silu * u[f + n];
-        if (round_h_bf16) h[n] = round_to_bf16(h[n]);
     }
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < d; ++m) {
@@ -282,13 +267,10 @@ static void expert_ffn(const uint16_t* x, int64_t d, int64_t f, const int8_t* q_
 /* The MoE layer output of [J15]/[J1]:  out_t = sum_j gates[t][j] *          */
 /* Expert_{ids[t][j]}(x_t).  Per-expert weights are passed as pointer tables */
 /* (an entry may be NULL for an expert no token selects).                   */
-/* round_h_bf16 = 1 rounds h to bf16 before the down projection (a variant   */
-/* that models the kernel's BF16 storage of h; 0 = the definition).         */
 int oracle_moe_forward(const uint16_t* x_bf16, int64_t T, int64_t d, int64_t f, int E,
                        int top_k, const int32_t* ids, const double* gates,
                        const int8_t* const* q_gu, const float* const* s_gu,
-                       const int8_t* const* q_d, const float* const* s_d, int round_h_bf16,
-                       double* out) {
+                       const int8_t* const* q_d, const float* const* s_d, double* out) {
     double* u = (double*)malloc(sizeof(double) * (size_t)(2 * f));
     double* h = (double*)malloc(sizeof(double) * (size_t)f);
     double* y = (double*)malloc(sizeof(double) * (size_t)d);
@@ -301,8 +283,7 @@ int oracle_moe_forward(const uint16_t* x_bf16, int64_t T, int64_t d, int64_t f, 
                 rc = 1;
                 break;
             }
-            expert_ffn(x_bf16 + t * d, d, f, q_gu[e], s_gu[e], q_d[e], s_d[e], round_h_bf16, u,
-                       h, y);
+            expert_ffn(x_bf16 + t * d, d, f, q_gu[e], s_gu[e], q_d[e], s_d[e], u, h, y);
             double g = gates[t * top_k + j];
             for (int64_t m = 0; m < d; ++m) out[t * d + m] += g * y[m];
         }
@@ -317,11 +298,11 @@ int oracle_moe_forward(const uint16_t* x_bf16, int64_t T, int64_t d, int64_t f, 
 /* SwiGLU MLP applied to every token, out_t = Expert(x_t).                  */
 void oracle_mlp_forward(const uint16_t* x_bf16, int64_t T, int64_t d, int64_t f,
                         const int8_t* q_gu, const float* s_gu, const int8_t* q_d, const float* s_d,
-                        int round_h_bf16, double* out) {
+                        double* out) {
     double* u = (double*)malloc(sizeof(double) * (size_t)(2 * f));
     double* h = (double*)malloc(sizeof(double) * (size_t)f);
     for (int64_t t = 0; t < T; ++t)
-        expert_ffn(x_bf16 + t * d, d, f, q_gu, s_gu, q_d, s_d, round_h_bf16, u, h, out + t * d);
+        expert_ffn(x_bf16 + t * d, d, f, q_gu, s_gu, q_d, s_d, u, h, out + t * d);
     free(u);
     free(h);
 }

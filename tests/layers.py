@@ -80,7 +80,7 @@ class OracleLayer:
     def route(self):
         return oracle.route(self.x_bits, self.w_router, self.wl.top_k, self.bias)
 
-    def forward_tokens(self, tokens, ids, gates, round_h_bf16=False):
+    def forward_tokens(self, tokens, ids, gates):
         """fp64 layer output for the rows ``tokens`` with the given routing."""
         tokens = np.asarray(tokens)
         ids_t = np.asarray(ids)[tokens]
@@ -91,11 +91,43 @@ class OracleLayer:
             for i, a in enumerate(self.expert(e)):
                 tables[i][e] = a
         return oracle.moe_forward(self.x_bits[tokens], ids_t, np.asarray(gates)[tokens],
-                                  *tables, round_h_bf16=round_h_bf16)
+                                  *tables)
 
     def dense_forward_tokens(self, tokens):
         qg, sg, qd, sd = self.expert(0)
         return oracle.mlp_forward(self.x_bits[np.asarray(tokens)], qg, sg, qd, sd)
+
+
+def gate_sum_bound(top_k: int) -> float:
+    """Largest |sum_j g_j - 1| the device's fp32 renormalisation can give:
+    the selected probabilities are summed in fp32 in selection order (top_k - 1
+    roundings of relative size <= 2^-24) and each gate is one correctly
+    rounded fp32 division (relative error <= 2^-24), so the sum is within
+    top_k * 2^-24 of 1, up to second-order terms (the 2^-20 slack)."""
+    return top_k * 2.0 ** -24 * (1.0 + 2.0 ** -20)
+
+
+def boundary_tokens(ids, E: int, top_k: int, tile: int = 128, experts=None):
+    """Tokens whose assignments sit where the expert kernels' tiling changes.
+
+    The assignments are grouped by expert with the oracle's stable counting
+    sort (the method's dispatch).  For every expert: its first and last
+    grouped row; for the experts in ``experts`` (all when None): both rows
+    on either side of every multiple of ``tile`` (the tensor-core path's
+    128-row MMA halves, 256-row tiles and raster groups all start at such
+    multiples).  Returns the sorted tokens of those rows."""
+    ids = np.asarray(ids, dtype=np.int32)
+    offsets, perm, _ = oracle.permute(ids, E)
+    rows = set()
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        rows.update((lo, hi - 1))
+        if experts is None or e in experts:
+            for b in range(tile, hi - lo, tile):
+                rows.update((lo + b - 1, lo + b))
+    return sorted(set(int(perm[r]) // top_k for r in rows))
 
 
 def assert_close(got, ref, what=""):

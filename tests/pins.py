@@ -454,18 +454,6 @@ def pin_silu_closed_form(o):
         assert np.allclose(out, ref, rtol=1e-14, atol=1e-300), (z, out, ref)
 
 
-def pin_bf16_h_variant(o):
-    """The variant that rounds h to bf16 stays within bf16 rounding of the
-    definition (used only to split error sources in the parity tests)."""
-    T, d, f = 6, 64, 96
-    x = _rand_bf16(46, synth.X, 1.0, (T, d))
-    qg, sg, qd, sd = _tiny_experts(o, 46, 1, d, f)
-    a = o.mlp_forward(x, qg[0], sg[0], qd[0], sd[0], round_h_bf16=False)
-    b = o.mlp_forward(x, qg[0], sg[0], qd[0], sd[0], round_h_bf16=True)
-    rel = np.abs(a - b).sum() / np.abs(a).sum()
-    assert 0 < rel < 5e-3, rel
-
-
 def _rmsnorm_exact(x_bits, g_bits, eps):
     """RMSNorm to ~60 digits (Fractions, Decimal square root), rounded once to
     bf16: the value the oracle must hit unless it lies within a few fp64 ulps

@@ -13,7 +13,8 @@ import pytest
 import oracle
 import synth
 from exact import bf16_bits
-from layers import DeviceLayer, OracleLayer, assert_close, bf16_to_f64
+from layers import (DeviceLayer, OracleLayer, assert_close, bf16_to_f64, boundary_tokens,
+                    gate_sum_bound)
 from synth.workloads import (LARGE_DECODE, LARGE_PREFILL_SKEW, MINI_DECODE, MINI_DECODE_E64,
                              MINI_DENSE, MINI_PREFILL, TINY, Workload)
 
@@ -98,7 +99,7 @@ def test_route_bitexact(wl):
     assert np.array_equal(ids.cpu().numpy(), io)
     gg = g.cpu().numpy().astype(np.float64)
     assert np.abs(gg - go).max() <= 1e-6
-    assert np.abs(gg.sum(axis=1) - 1.0).max() <= 2.0 ** -21
+    assert np.abs(gg.sum(axis=1) - 1.0).max() <= gate_sum_bound(wl.top_k)
     if wl.bias is not None:
         frac = float(np.isin(io, [0, 1]).mean())
         assert 0.33 <= frac <= 0.47, frac
@@ -192,39 +193,50 @@ def test_forward_mini_decode_all_tokens():
     assert_close(bf16_to_f64(out), ref, "mini decode")
 
 
-def test_forward_large_decode_sampled():
+def test_forward_large_decode_all_tokens():
+    # every token of the batch: all touched experts (about 15 of 16) and every
+    # 8-token pass of the decode kernels are compared
     dev, ora = DeviceLayer(LARGE_DECODE), OracleLayer(LARGE_DECODE)
     ids, g, out = run_layer(dev)
     _, io, go = ora.route()
     assert np.array_equal(ids.cpu().numpy(), io)
-    tokens = [0, 31]
+    assert np.unique(io).size >= 10
+    tokens = np.arange(LARGE_DECODE.T)
     ref = ora.forward_tokens(tokens, io, go)
-    assert_close(bf16_to_f64(out)[tokens], ref, "large decode")
+    assert_close(bf16_to_f64(out), ref, "large decode")
 
 
-def test_forward_e64_top4_sampled():
+def test_forward_e64_top4_all_tokens():
     # Mini sizes with 64 experts and top-4, the bench's launch configuration
     dev, ora = DeviceLayer(MINI_DECODE_E64), OracleLayer(MINI_DECODE_E64)
     ids, g, out = run_layer(dev)
     _, io, go = ora.route()
     assert np.array_equal(ids.cpu().numpy(), io)
     assert np.allclose(g.cpu().numpy(), go, rtol=0, atol=4e-6)
-    tokens = [0, 7]
+    tokens = np.arange(MINI_DECODE_E64.T)
     ref = ora.forward_tokens(tokens, io, go)
-    assert_close(bf16_to_f64(out)[tokens], ref, MINI_DECODE_E64.name)
+    assert_close(bf16_to_f64(out), ref, MINI_DECODE_E64.name)
 
 
-@pytest.mark.parametrize("wl,tokens", [
-    (MINI_PREFILL, [0, 1, 2, 511, 4097, 9000, 16382, 16383]),
-    (LARGE_PREFILL_SKEW, [0, 4095, 8191]),
-], ids=["mini_prefill", "large_prefill_skewed"])
-def test_forward_prefill_sampled(wl, tokens):
+@pytest.mark.parametrize("wl", [MINI_PREFILL, LARGE_PREFILL_SKEW],
+                         ids=["mini_prefill", "large_prefill_skewed"])
+def test_forward_prefill_tile_boundaries(wl):
+    """Full-size prefill, compared on the tokens whose assignments sit at each
+    expert's first and last grouped row and on both sides of every 128-row
+    boundary of every expert (the hot experts 0 and 1 of the skewed workload
+    included), plus the first and last token of the batch."""
     dev, ora = DeviceLayer(wl), OracleLayer(wl)
     ids, g, out = run_layer(dev)
     _, io, go = ora.route()
     assert np.array_equal(ids.cpu().numpy(), io)
+    tokens = sorted(set(boundary_tokens(io, wl.E, wl.top_k)) | {0, wl.T - 1})
+    assert len(tokens) >= 4 * wl.E
     ref = ora.forward_tokens(tokens, io, go)
-    assert_close(bf16_to_f64(out)[tokens], ref, wl.name)
+    got = bf16_to_f64(out)[tokens]
+    assert_close(got, ref, wl.name)
+    # every sampled row on its own, so no single bad row hides in the totals
+    for i, t in enumerate(tokens):
+        assert_close(got[i:i + 1], ref[i:i + 1], f"{wl.name} token {t}")
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -236,12 +248,17 @@ def test_dense_mlp_tiny(path):
     assert_close(bf16_to_f64(out), ora.dense_forward_tokens(np.arange(64)), "tiny dense")
 
 
-def test_dense_mlp_mini_sampled():
+def test_dense_mlp_mini_tile_boundaries():
+    # both rows on either side of every 128-row boundary, and the last row
     dev, ora = DeviceLayer(MINI_DENSE), OracleLayer(MINI_DENSE)
     out = jm.jmoe_mlp_forward(dev.x, dev.w_gu[0], dev.s_gu[0], dev.w_d[0], dev.s_d[0])
     torch.cuda.synchronize()
-    tokens = [0, 100, 8191, 16383]
-    assert_close(bf16_to_f64(out)[tokens], ora.dense_forward_tokens(tokens), "mini dense")
+    T = MINI_DENSE.T
+    tokens = sorted({0, T - 1} | {b + o for b in range(128, T, 128) for o in (-1, 0)})
+    got, ref = bf16_to_f64(out)[tokens], ora.dense_forward_tokens(tokens)
+    assert_close(got, ref, "mini dense")
+    for i, t in enumerate(tokens):
+        assert_close(got[i:i + 1], ref[i:i + 1], f"mini dense token {t}")
 
 
 # ----------------------------------------------------------------------------- edge cases
@@ -369,7 +386,7 @@ def test_route_generalised_bitexact(E, top_k, softmax_gates, T, d):
     # fp32 softmax: the denominator sums up to 64 terms, so up to ~64 ulp
     assert np.abs(gg - go).max() <= 4e-6
     if not softmax_gates:
-        assert np.abs(gg.sum(axis=1) - 1.0).max() <= 2.0 ** -20
+        assert np.abs(gg.sum(axis=1) - 1.0).max() <= gate_sum_bound(top_k)
 
 
 @pytest.mark.parametrize("E,top_k,T", [(64, 4, 37), (8, 2, 300), (32, 3, 129), (48, 4, 2)],

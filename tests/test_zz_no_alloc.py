@@ -4,10 +4,12 @@ HBM, or a latency-critical path that cannot afford cudaMalloc's implicit
 synchronisation).  Its scratch is a fixed array inside the library.
 
 The checks go through the C ABI (ctypes): two calls in a row, on different
-token batches, each compared with the workspace-taking jmoe_forward on the
-same inputs, within the parity tolerance of the other tests; and an oversized
-problem is refused before anything is launched.  The file is named so that
-pytest collects it last.
+token batches, each compared bit for bit with the workspace-taking
+jmoe_forward on the same inputs (both run the same deterministic decode
+kernels, so any difference is a scratch-layout or stale-scratch fault), the
+first batch also against the CPU oracle within the parity tolerance of the
+other tests; and an oversized problem is refused before anything is
+launched.  The file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -15,7 +17,7 @@ import numpy as np
 import pytest
 
 import synth
-from layers import DeviceLayer, assert_close, bf16_to_f64
+from layers import DeviceLayer, OracleLayer, assert_close, bf16_to_f64
 from synth.workloads import MINI_DECODE, Workload
 
 torch = pytest.importorskip("torch")
@@ -37,13 +39,19 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
     desc = dev.desc()
     batches = [dev.x, synth.normal_bf16_gpu(MINI_DECODE.seed + 100, synth.X, 1.0,
                                             tuple(dev.x.shape))]
-    for x in batches:
+    for i, x in enumerate(batches):
         ids, g = jm.jmoe_route(x, dev.w_router, MINI_DECODE.top_k)
         ref = jm.jmoe_forward(desc, x, ids, g)
         out = torch.full_like(x, float("nan"))
         assert _noalloc(desc, x, ids, g, out) == jm.JMOE_OK
         torch.cuda.synchronize()
-        assert_close(bf16_to_f64(out), bf16_to_f64(ref), "noalloc vs forward")
+        assert torch.equal(out, ref), f"batch {i}: noalloc differs from jmoe_forward"
+        if i == 0:
+            ora = OracleLayer(MINI_DECODE)
+            _, io, go = ora.route()
+            assert np.array_equal(ids.cpu().numpy(), io)
+            assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(MINI_DECODE.T), io, go),
+                         "noalloc vs oracle")
     assert jm.jmoe_last_error() == jm.JMOE_OK
 
 

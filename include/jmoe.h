@@ -218,7 +218,9 @@ jmoe_status jmoe_mlp_forward(const void* x_bf16, int64_t T, int64_t d_model, int
  *    and top-2 fit; 64 tokens at those sizes do not).
  *  - The first call on a device looks up the array's device address for that
  *    device (with that device current) and caches it; make that first call
- *    before capturing any stream work on the device.
+ *    before capturing any stream work on the device.  After a device reset
+ *    (cudaDeviceReset) the device has a new context, and the next call looks
+ *    the address up again: the cached one is tied to the context it came from.
  *  - All calls share the one array and it keeps whatever the last call left
  *    there.  Nothing in it has to start at zero for these kernels, so nothing
  *    is cleared.  Two calls whose work overlaps on the GPU (different

@@ -1,10 +1,12 @@
 // C ABI of libjmoe.so (declared in include/jmoe.h): argument validation,
 // workspace layout and kernel dispatch.  Nothing here allocates, frees or
 // synchronises, except jmoe_last_error.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/jmoe.h"
 #include "kernels.h"
@@ -18,7 +20,6 @@ constexpr int kMaxDevices = 64;
 constexpr int kStages = 6;
 cudaEvent_t g_stage_events[2 * kStages];
 std::atomic<bool> g_profile_on{false};
-std::atomic<unsigned*> g_err_ptr[kMaxDevices];
 std::atomic<int> g_num_sms[kMaxDevices];
 std::atomic<uint64_t> g_launches{0};
 
@@ -39,17 +40,61 @@ int current_device() {
     return dev;
 }
 
-unsigned* err_word() {
+// Unique id of the calling thread's current CUDA context (0 if the driver
+// cannot tell).  Device addresses of the library's __device__ arrays belong to
+// one context: after cudaDeviceReset the device gets a new primary context,
+// and addresses looked up in the old one are stale.
+unsigned long long current_context_id() {
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of a __device__ symbol in the current context, looked up
+// with cudaGetSymbolAddress the first time a device (or, after a device
+// reset, its new context) needs it, then cached per device.
+struct SymbolCache {
+    std::mutex mu;
+    unsigned long long ctx[kMaxDevices] = {};
+    void* addr[kMaxDevices] = {};
+};
+
+void* symbol_address(SymbolCache& c, const void* symbol) {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    unsigned* p = g_err_ptr[dev].load();
-    if (!p) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_jmoe_err_word) != cudaSuccess) return nullptr;
-        p = static_cast<unsigned*>(addr);
-        g_err_ptr[dev].store(p);
-    }
-    return p;
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(c.mu);
+    if (c.addr[dev] && c.ctx[dev] == ctx) return c.addr[dev];
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, symbol) != cudaSuccess || !addr) return nullptr;
+    c.addr[dev] = addr;
+    // the lookup has made the device's context current if nothing had yet
+    c.ctx[dev] = current_context_id();
+    return addr;
+}
+
+SymbolCache g_err_cache;
+
+unsigned* err_word() {
+    return static_cast<unsigned*>(symbol_address(g_err_cache, &g_jmoe_err_word));
 }
 
 int num_sms() {
@@ -227,22 +272,12 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
 // per device.  In host code its name is only a stand-in for the symbol; the
 // device address is looked up per device with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[JMOE_NOALLOC_SCRATCH_BYTES];
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+SymbolCache g_noalloc_cache;
 
 // The array's device address on the current device (looked up once per
-// device, with that device current), or nullptr if the lookup failed.
-void* noalloc_scratch() {
-    const int dev = current_device();
-    if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    void* p = g_noalloc_ptr[dev].load();
-    if (!p) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return nullptr;
-        g_noalloc_ptr[dev].store(addr);
-        p = addr;
-    }
-    return p;
-}
+// device and context, with that device current), or nullptr if the lookup
+// failed.
+void* noalloc_scratch() { return symbol_address(g_noalloc_cache, &g_noalloc_scratch); }
 
 }  // namespace
 

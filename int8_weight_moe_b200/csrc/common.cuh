@@ -66,35 +66,6 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// 16 bytes of int8 -> 8 packed bf16x2 words (element order preserved).
-__device__ __forceinline__ void i8x16_to_bf16x16(const uint4& q, uint32_t (&o)[8]) {
-    o[0] = i8x2_to_bf16x2<0>(q.x);
-    o[1] = i8x2_to_bf16x2<1>(q.x);
-    o[2] = i8x2_to_bf16x2<0>(q.y);
-    o[3] = i8x2_to_bf16x2<1>(q.y);
-    o[4] = i8x2_to_bf16x2<0>(q.z);
-    o[5] = i8x2_to_bf16x2<1>(q.z);
-    o[6] = i8x2_to_bf16x2<0>(q.w);
-    o[7] = i8x2_to_bf16x2<1>(q.w);
-}
-
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-// Streaming load for weights that are read exactly once.
-__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
 // 16-byte asynchronous global -> shared copy (bypasses L1).  src_bytes = 0
 // writes 16 zero bytes instead of reading.
 __device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src, uint32_t src_bytes) {
@@ -112,16 +83,6 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// D = A * B + D for one m16n8k16 tile, bf16 inputs, fp32 accumulators.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ float silu_f32(float z) {

@@ -75,27 +75,19 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 }
 
 // Four MMA steps of one 64-wide k-block: rows g (q0) and g+8 (q1).  Even and
-// odd steps accumulate into separate tiles (two independent MMA chains).
-// F16: weights converted to fp16 and fp16 MMA (activation operand in fp16);
-// otherwise bf16 conversion and bf16 MMA.
-template <bool F16>
+// odd steps accumulate into separate tiles (two independent MMA chains).  The
+// weights are converted to fp16 (the activation operand is fp16 too).
 __device__ __forceinline__ void mma_block(float (&acc)[2][4], const uint4& q0, const uint4& q1,
                                           const uint32_t (&b)[8]) {
     const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w};
     const uint32_t w1[4] = {q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-        if (F16) {
-            uint32_t l0, h0, l1, h1;
-            i8x4_to_f16x2x2(w0[s], l0, h0);
-            i8x4_to_f16x2x2(w1[s], l1, h1);
-            const uint32_t a[4] = {l0, l1, h0, h1};
-            mma_f16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
-        } else {
-            const uint32_t a[4] = {i8x2_to_bf16x2<0>(w0[s]), i8x2_to_bf16x2<0>(w1[s]),
-                                   i8x2_to_bf16x2<1>(w0[s]), i8x2_to_bf16x2<1>(w1[s])};
-            mma_bf16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
-        }
+        uint32_t l0, h0, l1, h1;
+        i8x4_to_f16x2x2(w0[s], l0, h0);
+        i8x4_to_f16x2x2(w1[s], l1, h1);
+        const uint32_t a[4] = {l0, l1, h0, h1};
+        mma_f16_16816(acc[s & 1], a, b[2 * s], b[2 * s + 1]);
     }
 }
 
@@ -103,8 +95,8 @@ struct Item {
     int e, group, pass, z;
 };
 
-// The last `slots` slot fills of a warp (the ones whose copies may still be
-// in flight when the warp leaves).
+// The first of the last `slots` slot fills a warp issued (the ones whose
+// copies may still be in flight when the warp leaves).
 __device__ __forceinline__ int64_t q_drain_begin(int64_t total, int slots) {
     return total > slots ? total - slots : 0;
 }
@@ -216,6 +208,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     // ---- producer cursor (lane 0 issues the TMA boxes of slot-sized pieces)
     int pe = 0, pi = 0, pj = 0;
     int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
+    int64_t issued = 0;    // slot fills issued so far (fill h uses slot h % kSlots)
     auto set_prefetch_item = [&](int it) {
         const Item u = item_at(it, pe);
         prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16
@@ -233,6 +226,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                     sm100::tma_load_2d(dst + (m * kNB + b) * 1024, &tmW, &full[warp][slot],
                                        pk + (pj * kNB + b) * 64, prow + m * moff);
         }
+        ++issued;
         if (++pj == nsl) {
             pj = 0;
             if (++pi < n_mine) set_prefetch_item(pi);
@@ -334,8 +328,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 #pragma unroll
                 for (int n = 0; n < NCH; ++n) {
                     if (n * 8 < cur.cnt_pass) {
-                        mma_block<true>(acc[n][0], wq[0], wq[1], fcur[b][n]);
-                        mma_block<true>(acc[n][1], wq[2], wq[3], fcur[b][n]);
+                        mma_block(acc[n][0], wq[0], wq[1], fcur[b][n]);
+                        mma_block(acc[n][1], wq[2], wq[3], fcur[b][n]);
                     }
                 }
             }
@@ -373,9 +367,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         step(q + 1, fb, fa);
         if (!ok) break;
     }
-    // leave only when no copy is still landing in this warp's ring
+    // leave only when no copy is still landing in this warp's ring: the last
+    // kSlots fills issued (all of them on the normal path, where issued equals
+    // total; fewer when a wait ran out), each the newest fill of its slot
     if (lane == 0) {
-        for (int64_t h = q_drain_begin(total, kSlots); h < total; ++h) {
+        for (int64_t h = q_drain_begin(issued, kSlots); h < issued; ++h) {
             const long long t0 = clock64();
             while (!sm100::mbar_try_wait(&full[warp][h % kSlots], (uint32_t)((h / kSlots) & 1)))
                 if (clock64() - t0 > sm100::kWaitCycles) break;

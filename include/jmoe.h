@@ -232,6 +232,45 @@ jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, 
                                  const int32_t* topk_ids, const float* topk_w, void* out_bf16,
                                  void* stream);
 
+/* Expert parallelism ("Jamba: A Hybrid Transformer-Mamba Language Model",
+ * paper summary, section "Training Infrastructure and Stabilization
+ * Techniques": expert parallelism with all-to-all communication that routes
+ * tokens to the GPU holding their selected experts; section
+ * "Mixture-of-Experts (MoE) in Jamba: Router, Top-K, and Load Balancing":
+ * MoE layers need all-to-all communication under expert parallelism).
+ * The E experts are split over G ranks: rank g owns the E/G consecutive
+ * experts g*E/G .. (g+1)*E/G - 1.  One layer forward on rank g is
+ *   jmoe_ep_dispatch  -> all-to-all of the send rows (and their local expert
+ *   ids) -> jmoe_forward on the received rows with the owned experts' weights
+ *   (desc.E = E/G, top_k = 1, gates 1) -> all-to-all back -> jmoe_ep_combine.
+ * The library does not communicate; the exchange is the caller's (the Python
+ * binding uses torch.distributed's all_to_all_single).
+ *
+ * jmoe_ep_dispatch groups the T*top_k assignments by expert (as jmoe_permute,
+ * which orders them by owner rank too) and builds the send buffer:
+ *   offsets   : device int32 [E+1] (written), as jmoe_permute; the rows for
+ *               rank r are offsets[r*E/G] .. offsets[(r+1)*E/G] - 1
+ *   perm, inv : device int32 [T*top_k] (written), as jmoe_permute
+ *   x_send    : device bf16 [T*top_k][d] (written up to row offsets[E] - 1):
+ *               x_send[i] = x[perm[i] / top_k]
+ *   local_ids : device int32 [T*top_k] (written): expert of perm[i] minus the
+ *               owner's first expert
+ * x_bf16 bf16 [T][d], topk_ids int32 [T][top_k].  E in 1..64, G >= 1 with
+ * E % G == 0, top_k in 1..4, d a multiple of 64.  Ids outside [0, E) are
+ * dropped (JMOE_EDEVICE in the device error word). */
+jmoe_status jmoe_ep_dispatch(const void* x_bf16, int64_t T, int64_t d, const int32_t* topk_ids,
+                             int32_t top_k, int32_t E, int32_t G, int32_t* offsets,
+                             int32_t* perm, int32_t* inv, void* x_send, int32_t* local_ids,
+                             void* stream);
+
+/* The combine after the return exchange: y_back bf16 [T*top_k][d] holds the
+ * expert output of send row i in row i; out_bf16 [T][d] (written):
+ *   out[t] = bf16( sum_j topk_w[t][j] * y_back[inv[t*top_k + j]] )
+ * summed in fp32 in assignment order (rows with inv < 0 add nothing).
+ * inv int32 [T*top_k] from jmoe_ep_dispatch, topk_w fp32 [T][top_k]. */
+jmoe_status jmoe_ep_combine(const void* y_back, const int32_t* inv, const float* topk_w,
+                            int64_t T, int64_t d, int32_t top_k, void* out_bf16, void* stream);
+
 /* Stage timing hook (diagnostics).  Registers `n` CUDA events (cudaEvent_t
  * handles passed as void*) that the following jmoe_forward / jmoe_mlp_forward
  * calls record on their stream around their kernels: events[2*i] before and
@@ -253,6 +292,25 @@ jmoe_status jmoe_profile_events(void* const* events, int32_t n);
  * difference around a region to count the launches inside it.  Never
  * synchronises.  Returns JMOE_EINVAL when count is NULL. */
 jmoe_status jmoe_launch_count(uint64_t* count);
+
+/* Test hook (diagnostics; the pages have no counterpart): exercises the
+ * bounded waits without any GPU fault.  Arms a stall for the next
+ * jmoe_forward / jmoe_mlp_forward call in the process (one call only, then it
+ * disarms itself):
+ *   JMOE_STALL_TENSOR_GEMM: the tensor-core path's gate/up GEMM; its weight
+ *     producers stop before their first tile, so the converter warps wait for
+ *     copies that never come;
+ *   JMOE_STALL_DECODE_GEMV: the decode path's gate/up GEMV; the first warp
+ *     never issues its first weight copy, so its consumer waits for nothing.
+ * During that call every mbarrier wait of the stalled kernel gives up after
+ * wait_cycles SM cycles (1000 .. 8e9; the default bound is about 2 s), the
+ * kernel drains the copies it did issue, frees its TMEM and sets
+ * JMOE_ETIMEOUT in the device error word; the call's output is undefined.
+ * The context stays usable and the next call runs normally.  target 0
+ * disarms; other values are JMOE_EINVAL. */
+#define JMOE_STALL_TENSOR_GEMM 1
+#define JMOE_STALL_DECODE_GEMV 2
+jmoe_status jmoe_test_stall(int32_t target, int64_t wait_cycles);
 
 /* Reads and clears the device error word of the current device.  Unlike the
  * other calls it synchronises the device.  Returns JMOE_OK when no kernel

@@ -27,10 +27,12 @@ JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_rmsnorm", "jmoe_rmsnorm_route",
             "jmoe_permute", "jmoe_forward_workspace_size",
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
-            "jmoe_profile_events", "jmoe_launch_count", "jmoe_last_error",
+            "jmoe_ep_dispatch", "jmoe_ep_combine",
+            "jmoe_profile_events", "jmoe_launch_count", "jmoe_test_stall", "jmoe_last_error",
             "jmoe_status_string")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
 JMOE_ROUTE_SOFTMAX_GATES = 1
+JMOE_STALL_TENSOR_GEMM, JMOE_STALL_DECODE_GEMV = 1, 2
 STAGES = ("permute", "gather", "gate_up", "down", "combine", "act")
 
 
@@ -79,8 +81,11 @@ def load() -> ctypes.CDLL:
     lib.jmoe_forward_noalloc.argtypes = [ctypes.POINTER(MoeDesc), vp, i64, vp, vp, vp, vp]
     lib.jmoe_mlp_workspace_size.argtypes = [i64, i64, i64, i32, ctypes.POINTER(sz)]
     lib.jmoe_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, sz, i32, vp]
+    lib.jmoe_ep_dispatch.argtypes = [vp, i64, i64, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.jmoe_ep_combine.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp]
     lib.jmoe_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.jmoe_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+    lib.jmoe_test_stall.argtypes = [i32, i64]
     lib.jmoe_last_error.argtypes = []
     for name in EXPORTED[:-1]:
         getattr(lib, name).restype = st
@@ -324,6 +329,42 @@ def jmoe_mlp_forward(x, w_gu, s_gu, w_d, s_d, out=None, workspace=None, path=JMO
     return out
 
 
+def jmoe_ep_dispatch(x, topk_ids, E: int, G: int):
+    """Expert-parallel send buffer (see jmoe.h) -> (offsets, perm, inv, x_send, local_ids)."""
+    import torch
+
+    _need(x, torch.bfloat16, "x")
+    _need(topk_ids, torch.int32, "topk_ids")
+    T, d = x.shape
+    k = topk_ids.shape[1]
+    dev = x.device
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    inv = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    x_send = torch.empty((max(T * k, 1), d), dtype=torch.bfloat16, device=dev)
+    local_ids = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+    _check("jmoe_ep_dispatch", load().jmoe_ep_dispatch(
+        _ptr(x), T, d, _ptr(topk_ids), k, E, G, _ptr(offsets), _ptr(perm), _ptr(inv),
+        _ptr(x_send), _ptr(local_ids), _stream(x)))
+    return offsets, perm[:T * k], inv[:T * k], x_send[:T * k], local_ids[:T * k]
+
+
+def jmoe_ep_combine(y_back, inv, topk_w, out=None):
+    """out[t] = bf16(sum_j topk_w[t, j] * y_back[inv[t * k + j]]) (see jmoe.h)."""
+    import torch
+
+    _need(y_back, torch.bfloat16, "y_back")
+    _need(inv, torch.int32, "inv")
+    _need(topk_w, torch.float32, "topk_w")
+    T, k = topk_w.shape
+    d = y_back.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=y_back.device)
+    _check("jmoe_ep_combine", load().jmoe_ep_combine(_ptr(y_back), _ptr(inv), _ptr(topk_w), T, d,
+                                                     k, _ptr(out), _stream(y_back)))
+    return out
+
+
 def jmoe_profile_events(events) -> None:
     """Register torch.cuda.Event objects (2 per stage, see jmoe.h; None skips a
     stage) or None to stop."""
@@ -340,6 +381,11 @@ def jmoe_launch_count() -> int:
     n = ctypes.c_uint64(0)
     _check("jmoe_launch_count", load().jmoe_launch_count(ctypes.byref(n)))
     return int(n.value)
+
+
+def jmoe_test_stall(target: int, wait_cycles: int = 0) -> None:
+    """Arm the bounded-wait test hook for the next forward call (see jmoe.h)."""
+    _check("jmoe_test_stall", load().jmoe_test_stall(target, wait_cycles))
 
 
 def jmoe_last_error() -> int:

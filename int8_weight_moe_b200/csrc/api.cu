@@ -23,6 +23,20 @@ std::atomic<bool> g_profile_on{false};
 std::atomic<int> g_num_sms[kMaxDevices];
 std::atomic<uint64_t> g_launches{0};
 
+// Test hook (jmoe_test_stall): armed for the next expert forward only.
+std::mutex g_stall_mu;
+int g_stall_target = 0;
+long long g_stall_wait_cycles = 0;
+
+// Takes the armed stall, if any, for this forward (and disarms it).
+void take_stall(int& target, long long& wait_cycles) {
+    std::lock_guard<std::mutex> lock(g_stall_mu);
+    target = g_stall_target;
+    wait_cycles = g_stall_wait_cycles;
+    g_stall_target = 0;
+    g_stall_wait_cycles = 0;
+}
+
 // The automatic path: the decode (GEMV-like) kernels while there are fewer
 // than max(128, 20 E) token->expert assignments, i.e. about 20 tokens per
 // expert; the tcgen05 grouped GEMM from there on.  The decode kernels re-read
@@ -236,6 +250,9 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
     int32_t* inv = static_cast<int32_t*>(at(w.inv));
     unsigned* err = err_word();
     const int sms = num_sms();
+    int stall = 0;
+    long long wait_cycles = 0;
+    take_stall(stall, wait_cycles);
 
     if (!prefill) {
         // grouping happens inside the decode path's first kernel
@@ -251,6 +268,8 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
         a.out = out; a.num_sms = sms;
         a.mark = stage_mark;
         a.err = err;
+        a.wait_cycles = wait_cycles;
+        a.fault = stall == JMOE_STALL_DECODE_GEMV ? 1 : 0;
         return from_cuda(jmoe::launch_decode(a, stream));
     }
     stage_mark(0, false, stream);
@@ -265,6 +284,8 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
     p.inv = inv; p.xperm = at(w.xperm); p.H = at(w.Hp); p.Yg = static_cast<float*>(at(w.Yg));
     p.rows_padded = w.rows_padded; p.out = out; p.num_sms = sms; p.err = err;
     p.mark = stage_mark; p.dense = dense;
+    p.wait_cycles = wait_cycles;
+    p.fault_tile = stall == JMOE_STALL_TENSOR_GEMM ? 0 : -1;
     return from_cuda(jmoe::launch_prefill(p, stream));
 }
 
@@ -489,6 +510,39 @@ jmoe_status jmoe_forward_noalloc(const jmoe_moe_desc* desc, const void* x_bf16, 
                        JMOE_NOALLOC_SCRATCH_BYTES, false, (cudaStream_t)stream);
 }
 
+jmoe_status jmoe_ep_dispatch(const void* x_bf16, int64_t T, int64_t d, const int32_t* topk_ids,
+                             int32_t top_k, int32_t E, int32_t G, int32_t* offsets, int32_t* perm,
+                             int32_t* inv, void* x_send, int32_t* local_ids, void* stream) {
+    if (T < 0 || d <= 0) return JMOE_EINVAL;
+    if (E < 1 || E > 64 || top_k < 1 || top_k > 4 || top_k > E) return JMOE_EUNSUPPORTED;
+    if (G < 1 || E % G != 0) return JMOE_EUNSUPPORTED;
+    if (d % 64) return JMOE_EUNSUPPORTED;
+    if (T * top_k > (1LL << 24)) return JMOE_EUNSUPPORTED;
+    if (!offsets) return JMOE_EINVAL;
+    if (T > 0 && (!x_bf16 || !topk_ids || !perm || !inv || !x_send || !local_ids))
+        return JMOE_EINVAL;
+    if (!aligned16(offsets) || (T > 0 && (!aligned16(x_bf16) || !aligned16(topk_ids) ||
+                                          !aligned16(perm) || !aligned16(inv) ||
+                                          !aligned16(x_send) || !aligned16(local_ids))))
+        return JMOE_EALIGN;
+    return from_cuda(jmoe::launch_ep_dispatch(x_bf16, T, d, topk_ids, top_k, E, E / G, offsets,
+                                              perm, inv, x_send, local_ids, err_word(), num_sms(),
+                                              (cudaStream_t)stream));
+}
+
+jmoe_status jmoe_ep_combine(const void* y_back, const int32_t* inv, const float* topk_w, int64_t T,
+                            int64_t d, int32_t top_k, void* out_bf16, void* stream) {
+    if (T < 0 || d <= 0) return JMOE_EINVAL;
+    if (top_k < 1 || top_k > 4) return JMOE_EUNSUPPORTED;
+    if (d % 64) return JMOE_EUNSUPPORTED;
+    if (T == 0) return JMOE_OK;
+    if (!y_back || !inv || !topk_w || !out_bf16) return JMOE_EINVAL;
+    if (!aligned16(y_back) || !aligned16(inv) || !aligned16(topk_w) || !aligned16(out_bf16))
+        return JMOE_EALIGN;
+    return from_cuda(jmoe::launch_ep_combine(y_back, inv, topk_w, T, d, top_k, out_bf16,
+                                             (cudaStream_t)stream));
+}
+
 jmoe_status jmoe_profile_events(void* const* events, int32_t n) {
     if (n == 0 || events == nullptr) {
         g_profile_on.store(false);
@@ -499,6 +553,16 @@ jmoe_status jmoe_profile_events(void* const* events, int32_t n) {
         if ((events[i] == nullptr) != (events[i + 1] == nullptr)) return JMOE_EINVAL;
     for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
     g_profile_on.store(true);
+    return JMOE_OK;
+}
+
+jmoe_status jmoe_test_stall(int32_t target, int64_t wait_cycles) {
+    if (target < 0 || target > JMOE_STALL_DECODE_GEMV) return JMOE_EINVAL;
+    if (target != 0 && (wait_cycles < 1000 || wait_cycles > jmoe::kMaxWaitCycles))
+        return JMOE_EINVAL;
+    std::lock_guard<std::mutex> lock(g_stall_mu);
+    g_stall_target = target;
+    g_stall_wait_cycles = target ? (long long)wait_cycles : 0;
     return JMOE_OK;
 }
 

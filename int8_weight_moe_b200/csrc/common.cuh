@@ -138,6 +138,8 @@ struct GemvParams {
     float* P;                  // partial sums [S][A][cols]
     int64_t A;
     unsigned* err;
+    long long wait_cycles;     // bound of every mbarrier wait (SM cycles)
+    int fault;                 // test hook: warp 0 of block 0 never issues its first copy
 };
 
 }  // namespace jmoe

@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     int pe = 0, pi = 0, pj = 0;
     int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
     int64_t issued = 0;    // slot fills issued so far (fill h uses slot h % kSlots)
+    int64_t skipped = -1;  // the fill the test hook left out (its barrier never completes)
     auto set_prefetch_item = [&](int it) {
         const Item u = item_at(it, pe);
         prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16
@@ -216,7 +217,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         pk = u.z * kb_item * 64;
     };
     auto issue = [&](int slot) {
-        if (lane == 0) {
+        const bool skip = p.fault && wid == 0 && issued == 0;
+        if (skip) skipped = issued;
+        if (lane == 0 && !skip) {
             uint8_t* dst = ring + slot * kSlotBytes;
             sm100::mbar_arrive_expect_tx(&full[warp][slot], kSlotBytes);
 #pragma unroll
@@ -311,7 +314,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                 for (int n = 0; n < NCH; ++n)
                     prefetch_l1(cur.b[n] + min((cj + 2) * kNB + b, kb_item - 1) * 64);
         }
-        if (!sm100::mbar_wait(&full[warp][cslot], cphase, abort)) {
+        // every lane waits; the vote keeps the warp on one path
+        if (!__all_sync(0xffffffffu,
+                        sm100::mbar_wait(&full[warp][cslot], cphase, abort, p.wait_cycles))) {
             ok = false;
             return;
         }
@@ -372,9 +377,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     // total; fewer when a wait ran out), each the newest fill of its slot
     if (lane == 0) {
         for (int64_t h = q_drain_begin(issued, kSlots); h < issued; ++h) {
+            if (h == skipped) continue;
             const long long t0 = clock64();
             while (!sm100::mbar_try_wait(&full[warp][h % kSlots], (uint32_t)((h / kSlots) & 1)))
-                if (clock64() - t0 > sm100::kWaitCycles) break;
+                if (clock64() - t0 > p.wait_cycles) break;
         }
         if (!ok && p.err) flag_error(p.err, kErrTimeout);
     }
@@ -656,6 +662,8 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.offsets = a.offsets;
     p.perm = a.perm;
     p.err = a.err;
+    p.wait_cycles = a.wait_cycles > 0 ? a.wait_cycles : sm100::kWaitCycles;
+    p.fault = a.fault;
     p.w = a.wgu;
     p.S = a.split_gu;
     p.b_src = static_cast<const uint16_t*>(a.x16);
@@ -686,6 +694,7 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     if (a.mark) a.mark(5, true, stream);
     if (err != cudaSuccess) return err;
     p.w = a.wd;
+    p.fault = 0;
     p.S = a.split_d;
     p.b_src = static_cast<const uint16_t*>(a.H);
     p.P = a.P_d;

@@ -25,6 +25,10 @@ enum : unsigned {
     kErrBadExpert = 2u,  // an expert id outside [0, E)
 };
 
+// Largest bound a caller may give the kernels' mbarrier waits (SM cycles,
+// about 4 s at 2 GHz).
+constexpr long long kMaxWaitCycles = 8000000000LL;
+
 // Rows of the tensor-core path's M tile; expert groups are padded to it.
 constexpr int kPrefillTileM = 128;
 
@@ -83,6 +87,8 @@ struct DecodeArgs {
     int num_sms;
     StageMark mark;
     unsigned* err;        // device error word
+    long long wait_cycles;  // bound of the kernels' mbarrier waits (0: the default)
+    int fault;            // test hook: the gate/up GEMV's first warp skips its first copy
 };
 
 // K pieces for a decode GEMV: the smallest divisor s of K/64 with s >= want
@@ -92,5 +98,13 @@ cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int
                             const int32_t* ids, void* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, float v, int64_t n, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Expert parallelism (ep.cu): grouping + send buffer, and the final combine.
+cudaError_t launch_ep_dispatch(const void* x, int64_t T, int64_t d, const int32_t* ids, int top_k,
+                               int E, int E_local, int32_t* offsets, int32_t* perm, int32_t* inv,
+                               void* x_send, int32_t* local_ids, unsigned* err, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_ep_combine(const void* y_back, const int32_t* inv, const float* gates,
+                              int64_t T, int64_t d, int top_k, void* out, cudaStream_t stream);
 
 }  // namespace jmoe

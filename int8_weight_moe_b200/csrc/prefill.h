@@ -31,6 +31,9 @@ struct PrefillArgs {
     unsigned* err;
     StageMark mark;
     bool dense;                    // one expert, every token routed to it with gate 1
+    long long wait_cycles;         // bound of the kernels' mbarrier waits (0: the default)
+    int fault_tile;                // test hook (< 0: off): the gate/up GEMM's weight
+                                   // producers stop before this tile
 };
 
 bool prefill_available();

@@ -1,6 +1,7 @@
 // Tensor-core path of the expert MLPs (many tokens per expert): a persistent
 // grouped GEMM on the 5th-generation tensor cores (tcgen05, accumulators in
-// TMEM), with the ExpertsInt8 dequantisation inside the kernel.
+// TMEM), run by CTA pairs, with the ExpertsInt8 dequantisation inside the
+// kernel.
 //
 // "Jamba-1.5: Hybrid Transformer-Mamba Models at Scale" (paper summary),
 // section "ExpertsInt8 Quantization (Section 3.1)", step 3: the INT8 weights
@@ -12,33 +13,47 @@
 // (sum_k x_k (q_k s) = s sum_k x_k q_k).  Activations stay BF16 (step 4);
 // accumulation is fp32 in TMEM.
 //
-// One CTA per SM, 16 warps:
-//   warp 0      TMA producer of the activation tile A [256 rows x 64 k] bf16
-//               (two 128-row boxes; the second is skipped when the expert ends)
-//   warp 1      TMEM allocator and MMA issuer of the first 128-row half
-//   warp 2      TMA producer of the INT8 weight tile [128 rows x 64 k]
-//   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled)
-//   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
-//   warp 15     MMA issuer of the second 128-row half
-// Two issuing threads, one per half (each with its own accumulator, so the
-// order of every accumulation stays fixed): a thread that waits on an
-// mbarrier stops issuing until the MMAs it already queued have been
-// dispatched, and the tensor pipe would idle through every such wait if one
-// thread issued everything; with two, the other thread's MMAs fill it.
-// Rings: A + converted B share 3 stages (48 KB each); the INT8 tiles, which
-// come from HBM, have 8 stages (8 KB each) to cover its latency.  Each weight tile, once converted, feeds two M = 128
-// MMAs (256 token rows), which halves the conversion work per multiply-add
-// compared with one 128-row MMA.  Two accumulators of 2 x 128 x 128 fp32
-// (512 TMEM columns) let the epilogue of one tile overlap the main loop of
-// the next.
+// A cluster of two CTAs (a pair, on two SMs) computes one tile of 256 token
+// rows x 256 output columns with CTA-pair MMAs (tcgen05.mma.cta_group::2,
+// M = 256, N = 256, K = 16): each CTA holds 128 of the token rows (A) and
+// converts 128 of the 256 weight rows (B); the tensor cores of both SMs read
+// both CTAs' halves, and each CTA's TMEM receives its 128 rows x 256 columns.
+// Per 64-wide k-step a CTA's shared memory carries 16 KB of A (TMA), 8 KB of
+// INT8 (TMA), the converters' 8 KB read + 16 KB write, and 32 KB of MMA
+// operand reads: 80 KB for 2 x 128 x 256 x 64 multiply-adds, about half of
+// what one CTA holding the whole 128-wide weight tile for 256 rows moves per
+// multiply-add, and each weight is converted once per 256 token rows.
 //
-// Tiles: 256 expert-grouped rows (each expert's rows are padded to a
-// multiple of 128, so a tile never mixes experts; its second half may be
-// absent) x 128 MMA columns.  Gate/up mode: the 128 columns are 64 gate
-// channels and the same 64 up channels, so the SwiGLU pairs sit in one
-// thread.  Down mode: 128 output channels; the epilogue multiplies by the
-// routing gate and writes one fp32 row per token->expert assignment.  Tiles
-// are visited expert by expert in groups of 16 m-tiles (see decode_tile).
+// Warps of each CTA (15):
+//   warp 0      TMA producer of the CTA's A rows [128 x 64 k] bf16 (skipped
+//               when the CTA's half of the tile lies past the expert's rows)
+//   warp 1      TMEM allocator (both CTAs); MMA issuer (even CTA only)
+//   warp 2      TMA producer of the CTA's INT8 weight rows [128 x 64 k]
+//   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled), in two
+//               groups of 4 that take alternate k-steps
+//   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
+//
+// Gate/up tiles: the even CTA converts 128 gate channels, the odd CTA the
+// same 128 up channels, so TMEM columns c and 128 + c of a row hold the gate
+// and up sums of one channel (the SwiGLU pair sits in one thread).  Down
+// tiles: 256 output channels, 128 per CTA.  Expert rows are padded to 128; a
+// pair tile whose second half lies past the expert's rows leaves the odd
+// CTA's A stale and stores nothing for it (the MMA rows are independent).
+//
+// Synchronisation (mbarriers; every wait is bounded and a wait that runs out
+// raises the abort flags of both CTAs, after which every role drains its own
+// copies and the pair frees its TMEM):
+//   a_full[s]   (each CTA)  its A copy of stage s landed
+//   b8_full/b8_empty (each CTA)  INT8 ring between its TMA and its converters
+//   full[s]     (even CTA)  the converter warps of both CTAs wrote stage s's
+//                           BF16 weights after seeing their CTA's A land
+//   empty[s]    (each CTA)  the MMAs of stage s are done (commit multicast)
+//   acc_full[b] (each CTA)  accumulator b is final (commit multicast)
+//   acc_empty[b] (even CTA) the epilogue warps of both CTAs read it
+// Two accumulators of 256 fp32 columns (all 512 TMEM columns) let the
+// epilogue of one tile overlap the main loop of the next.  Tiles are visited
+// expert by expert in groups of 16 m-tiles (see decode_tile).  No TMA load is
+// multicast; every copy reads global memory into its own CTA.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -51,28 +66,48 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BH = 128;       // rows of one MMA (a "half" of the tile)
-constexpr int BM = 2 * BH;    // token rows per tile: two MMAs share one weight tile
-constexpr int BN = 128, BK = 64;
-constexpr int kStagesAB = 3, kStages8 = 8;
-constexpr int kGroupM = 16;  // m-tiles per raster group (activation rows kept in L2)
-constexpr int kHalfBytes = BH * BK * 2;  // 16 KB
-constexpr int kABytes = 2 * kHalfBytes;  // 32 KB
-constexpr int kBbfBytes = BN * BK * 2;   // 16 KB
-constexpr int kB8Bytes = BN * BK;        // 8 KB
-constexpr int kABStage = kABytes + kBbfBytes;
-constexpr int kSmemAB = kStagesAB * kABStage;
+constexpr int BH = 128;       // token rows of one CTA (a half of the pair tile)
+constexpr int BM = 2 * BH;    // token rows of a pair tile
+constexpr int BN = 256;       // MMA N: output columns of a pair tile
+constexpr int BNC = BN / 2;   // weight rows each CTA converts
+constexpr int BK = 64;
+// Ring depths.  A (activations, mostly L2 hits) and the INT8 weights (HBM)
+// are fetched several k-steps ahead of the MMAs: a k-step's MMAs take about
+// 512 cycles, less than a TMA round trip under load.  The converted BF16
+// weights need only cover the converters' latency.  Even depths: stage s of
+// the BF16 and INT8 rings always goes to converter group s & 1.
+#ifndef JMOE_GEMM_STAGES_A
+#define JMOE_GEMM_STAGES_A 6
+#endif
+#ifndef JMOE_GEMM_STAGES_B
+#define JMOE_GEMM_STAGES_B 6
+#endif
+#ifndef JMOE_GEMM_STAGES_8
+#define JMOE_GEMM_STAGES_8 4
+#endif
+constexpr int kStagesA = JMOE_GEMM_STAGES_A, kStagesB = JMOE_GEMM_STAGES_B;
+constexpr int kStages8 = JMOE_GEMM_STAGES_8;
+constexpr int kGroupM = 16;  // pair m-tiles per raster group (activation rows kept in L2)
+constexpr int kABytes = BH * BK * 2;     // 16 KB
+constexpr int kBbfBytes = BNC * BK * 2;  // 16 KB
+constexpr int kB8Bytes = BNC * BK;       // 8 KB
+constexpr int kSmemA = kStagesA * kABytes;
+constexpr int kSmemB = kStagesB * kBbfBytes;
 constexpr int kSmem8 = kStages8 * kB8Bytes;
-constexpr uint32_t kTmemCols = 512;   // 2 buffers x 2 halves x 128 fp32 columns
-constexpr uint32_t kIdesc = idesc_bf16_f32(BH, BN);
+constexpr uint32_t kTmemCols = 512;   // 2 accumulators x 256 fp32 columns
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
+constexpr uint16_t kPairMask = 0x3;   // both CTAs of the cluster
 
 constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
-constexpr int kConvWarp0 = 3, kConvWarps = 8;
+constexpr int kConvWarp0 = 3, kConvGroupWarps = 4, kConvWarps = 2 * kConvGroupWarps;
+constexpr int kConvThreads = kConvGroupWarps * 32;  // threads of one converter group
 constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps, kEpiWarps = 4;
-constexpr int kWarpMMA2 = kEpiWarp0 + kEpiWarps;
-constexpr int kThreads = (kWarpMMA2 + 1) * 32;
-constexpr int kIssuers = 2;  // MMA-issuing threads (one per 128-row half)
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+constexpr int kChunks = kB8Bytes / 16 / kConvThreads;  // 16-byte INT8 chunks per thread per k-step
 constexpr int kMaxE = 64;
+
+static_assert(kStagesB % 2 == 0 && kStages8 % 2 == 0, "converter groups alternate k-steps");
+static_assert(kChunks * 16 * kConvThreads == kB8Bytes, "converter work split");
 
 enum Mode { kGateUp = 0, kDown = 1 };
 
@@ -91,10 +126,13 @@ struct GemmParams {
     uint16_t* H;          // gate/up output, bf16 [rows_padded][d_ff]
     float* Y;             // down output, fp32 [A][d_model]
     unsigned* err;
+    long long wait_cycles;  // bound of every mbarrier wait (SM cycles)
+    int fault_tile;         // < 0: none; else the weight producers stop before this tile
 };
 
 struct Shared {
-    uint64_t ab_full[kStagesAB], ab_empty[kStagesAB];
+    uint64_t full[kStagesB], empty_b[kStagesB];
+    uint64_t a_full[kStagesA], empty_a[kStagesA];
     uint64_t b8_full[kStages8], b8_empty[kStages8];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t drain;
@@ -105,14 +143,15 @@ struct Shared {
     int tile_start[kMaxE + 1];
 };
 
-constexpr int kSmemBytes = kSmemAB + kSmem8 + (int)sizeof(Shared) + 1024;
+constexpr int kSmemBytes = kSmemA + kSmemB + kSmem8 + (int)sizeof(Shared) + 1024;
+static_assert(kSmemBytes <= 232448, "more shared memory than a CTA can have");
 
 struct Tile {
     int e, row0, n, halves;  // halves: 1 or 2 valid 128-row halves
 };
 
 // Tile order inside an expert: groups of kGroupM m-tiles; within a group all
-// n-tiles, m fastest.  The CTAs of a wave then share a few weight tiles and
+// n-tiles, m fastest.  The pairs of a wave then share a few weight tiles and
 // at most kGroupM x 256 activation rows, which stay in L2.
 __device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int n_tiles, int tile) {
     int e = 0;
@@ -132,45 +171,50 @@ __device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int n_tiles,
     return t;
 }
 
-// Bounded wait that ignores the abort flag (used only while draining).
-__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
+// Bounded wait that ignores the abort flags (used only while draining).
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitCycles) return;
+        if (clock64() - t0 > limit) return;
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    Shared& S = *reinterpret_cast<Shared*>(smem + kSmemAB + kSmem8);
-    auto tileA = [&](int s) { return smem + s * kABStage; };
-    auto tileBbf = [&](int s) { return smem + s * kABStage + kABytes; };
-    auto tileB8 = [&](int s) { return smem + kSmemAB + s * kB8Bytes; };
+    Shared& S = *reinterpret_cast<Shared*>(smem + kSmemA + kSmemB + kSmem8);
+    auto tileA = [&](int s) { return smem + s * kABytes; };
+    auto tileBbf = [&](int s) { return smem + kSmemA + s * kBbfBytes; };
+    auto tileB8 = [&](int s) { return smem + kSmemA + kSmemB + s * kB8Bytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs; 1: its partner
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int E = p.E;
     const int KB = p.K / BK;
+    const long long limit = p.wait_cycles;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStagesAB; ++i) {
-            // the A producer's expect-tx arrival (plus the TMA bytes) and the
-            // converter warps' arrivals
-            mbar_init(&S.ab_full[i], 1 + kConvWarps);
-            mbar_init(&S.ab_empty[i], kIssuers);
+        for (int i = 0; i < kStagesB; ++i) {
+            mbar_init(&S.full[i], 2 * kConvGroupWarps);  // one converter group of each CTA
+            mbar_init(&S.empty_b[i], 1);                  // the MMA commit
+        }
+        for (int i = 0; i < kStagesA; ++i) {
+            mbar_init(&S.a_full[i], 1);                   // the A producer (+ TMA bytes)
+            mbar_init(&S.empty_a[i], 1);                  // the MMA commit
         }
         for (int i = 0; i < kStages8; ++i) {
             mbar_init(&S.b8_full[i], 1);
-            mbar_init(&S.b8_empty[i], kConvWarps);
+            mbar_init(&S.b8_empty[i], kConvGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.acc_full[i], kIssuers);
-            mbar_init(&S.acc_empty[i], kEpiWarps);
+            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_empty[i], 2 * kEpiWarps);
         }
-        mbar_init(&S.drain, kIssuers);
+        mbar_init(&S.drain, 1);
         S.abort = 0;
         fence_mbar_init();
     }
@@ -192,124 +236,136 @@ __global__ void __launch_bounds__(kThreads, 1)
         S.tile_start[E] = run;
     }
     if (warp == kWarpMMA) {
-        tmem_alloc(&S.tmem_base, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(&S.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
     }
+    // both CTAs' barriers initialised and TMEM allocated before any role
+    // touches the partner
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     const int total = S.tile_start[E];
     volatile int* abort = &S.abort;
+    const uint32_t peer_abort = mapa_shared(smem_u32(&S.abort), rank ^ 1u);
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        return mbar_wait_pair(bar, parity, abort, peer_abort, limit);
+    };
 
     if (warp == kWarpProdA) {
         if (lane == 0) {
             uint32_t g = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+            for (int tile = pair; tile < total && !*abort; tile += npairs) {
                 const Tile t = decode_tile(S, E, p.n_tiles, tile);
+                const bool mine = (int)rank < t.halves;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = g % kStagesAB;
-                    const uint32_t ph = (g / kStagesAB) & 1;
-                    if (!mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) break;
-                    mbar_arrive_expect_tx(&S.ab_full[s], t.halves * kHalfBytes);
-                    tma_load_2d(tileA(s), &tmA, &S.ab_full[s], kb * BK, t.row0);
-                    if (t.halves == 2)
-                        tma_load_2d(tileA(s) + kHalfBytes, &tmA, &S.ab_full[s], kb * BK,
-                                    t.row0 + BH);
+                    const int s = g % kStagesA;
+                    const uint32_t ph = (g / kStagesA) & 1;
+                    if (!wait(&S.empty_a[s], ph ^ 1)) break;
+                    if (mine) {
+                        mbar_arrive_expect_tx(&S.a_full[s], kABytes);
+                        tma_load_2d(tileA(s), &tmA, &S.a_full[s], kb * BK, t.row0 + (int)rank * BH);
+                    } else {
+                        mbar_arrive(&S.a_full[s]);
+                    }
                 }
             }
-            // make sure no copy is still landing in shared memory when the CTA exits
-            for (uint32_t h = (g > (uint32_t)kStagesAB ? g - kStagesAB : 0); h < g; ++h)
-                wait_drain(&S.ab_full[h % kStagesAB], (h / kStagesAB) & 1);
+            // leave only when no copy is still landing in shared memory
+            for (uint32_t h = (g > (uint32_t)kStagesA ? g - kStagesA : 0); h < g; ++h)
+                wait_drain(&S.a_full[h % kStagesA], (h / kStagesA) & 1, limit);
         }
     } else if (warp == kWarpProdB) {
         if (lane == 0) {
             uint32_t g = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x) {
+            for (int tile = pair; tile < total && !*abort; tile += npairs) {
+                if (tile == p.fault_tile) break;  // test hook: this tile's weights never come
                 const Tile t = decode_tile(S, E, p.n_tiles, tile);
+                // gate/up: the even CTA's gate rows, the odd CTA's up rows of the same
+                // channels; down: the CTA's half of the 256 output channels
+                const int y = MODE == kGateUp ? t.e * p.w_rows + (int)rank * p.up_offset + t.n * BNC
+                                              : t.e * p.w_rows + t.n * BN + (int)rank * BNC;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages8;
                     const uint32_t ph = (g / kStages8) & 1;
-                    if (!mbar_wait(&S.b8_empty[s], ph ^ 1, abort)) break;
+                    if (!wait(&S.b8_empty[s], ph ^ 1)) break;
                     mbar_arrive_expect_tx(&S.b8_full[s], kB8Bytes);
-                    if (MODE == kGateUp) {
-                        const int y = t.e * p.w_rows + t.n * (BN / 2);
-                        tma_load_2d(tileB8(s), &tmB, &S.b8_full[s], kb * BK, y);
-                        tma_load_2d(tileB8(s) + kB8Bytes / 2, &tmB, &S.b8_full[s], kb * BK,
-                                    y + p.up_offset);
-                    } else {
-                        tma_load_2d(tileB8(s), &tmB, &S.b8_full[s], kb * BK,
-                                    t.e * p.w_rows + t.n * BN);
-                    }
+                    tma_load_2d(tileB8(s), &tmB, &S.b8_full[s], kb * BK, y);
                 }
             }
             for (uint32_t h = (g > (uint32_t)kStages8 ? g - kStages8 : 0); h < g; ++h)
-                wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1);
+                wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1, limit);
         }
-    } else if (warp == kWarpMMA || warp == kWarpMMA2) {
-        if (lane == 0) {
-            const int h = warp == kWarpMMA ? 0 : 1;  // the 128-row half this thread issues
+    } else if (warp == kWarpMMA) {
+        if (rank == 0 && lane == 0) {
             uint32_t g = 0;
             int it = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
-                const bool active = h < decode_tile(S, E, p.n_tiles, tile).halves;
+            for (int tile = pair; tile < total && !*abort; tile += npairs, ++it) {
                 const int buf = it & 1;
-                if (!mbar_wait(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort)) break;
+                if (!mbar_wait_pair(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, peer_abort, limit))
+                    break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * 2 * BN + h * BN;
+                const uint32_t d_tmem = tmem + buf * BN;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = g % kStagesAB;
-                    const uint32_t ph = (g / kStagesAB) & 1;
-                    if (!mbar_wait(&S.ab_full[s], ph, abort)) {
+                    const int sa = g % kStagesA;
+                    const int s = g % kStagesB;
+                    const uint32_t ph = (g / kStagesB) & 1;
+                    if (!mbar_wait_pair(&S.full[s], ph, abort, peer_abort, limit)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    if (active) {
-                        const uint32_t a0 = smem_u32(tileA(s)) + h * kHalfBytes;
-                        const uint32_t b0 = smem_u32(tileBbf(s));
+                    const uint32_t a0 = smem_u32(tileA(sa));
+                    const uint32_t b0 = smem_u32(tileBbf(s));
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_bf16_ss(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
-                                        kIdesc, (kb | kk) != 0);
-                    }
-                    mma_commit(&S.ab_empty[s]);
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_ss_pair(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
+                                         kIdesc, (kb | kk) != 0);
+                    mma_commit_pair_mc(&S.empty_a[sa], kPairMask);
+                    mma_commit_pair_mc(&S.empty_b[s], kPairMask);
                 }
                 if (!ok) break;
-                mma_commit(&S.acc_full[buf]);
+                mma_commit_pair_mc(&S.acc_full[buf], kPairMask);
             }
-            mma_commit(&S.drain);
-            wait_drain(&S.drain, 0);
+            // every MMA done (both CTAs' TMEM written, both CTAs' shared memory read)
+            mma_commit_pair(&S.drain);
+            wait_drain(&S.drain, 0, limit);
         }
     } else if (warp >= kConvWarp0 && warp < kConvWarp0 + kConvWarps) {
-        // Thread ct converts the 16-byte int8 chunks q = ct and ct + 256 of the
-        // tile (row q / 4, bytes 16 (q % 4) .. +16): both loads are issued
-        // before any conversion, and each chunk becomes two 16-byte bf16 units
-        // 2 (q % 4) and 2 (q % 4) + 1 of the row's 128-byte swizzled line.
-        const int ct = threadIdx.x - kConvWarp0 * 32;  // 0..255
+        // Group G converts the k-steps g with g % 2 == G.  Thread ct converts the
+        // 16-byte INT8 chunks q = ct + 128 j (row q / 4, bytes 16 (q % 4) ..
+        // +16) of the CTA's 128 x 64 tile: all loads first, then each chunk
+        // becomes the two 16-byte bf16 units 2 (q % 4) and 2 (q % 4) + 1 of the
+        // row's 128-byte swizzled line.
+        const int G = (warp - kConvWarp0) / kConvGroupWarps;
+        const int ct = threadIdx.x - (kConvWarp0 + G * kConvGroupWarps) * 32;  // 0..127
+        const uint32_t full_leader = mapa_shared(smem_u32(&S.full[0]), 0);
         uint32_t g = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok && !*abort; tile += gridDim.x) {
+        for (int tile = pair; tile < total && ok && !*abort; tile += npairs) {
             for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = g % kStagesAB;
-                const uint32_t ph = (g / kStagesAB) & 1;
+                if ((int)(g & 1) != G) continue;
+                const int s = g % kStagesB;
+                const uint32_t ph = (g / kStagesB) & 1;
+                const int sa = g % kStagesA;
+                const uint32_t pha = (g / kStagesA) & 1;
                 const int s8 = g % kStages8;
                 const uint32_t ph8 = (g / kStages8) & 1;
-                if (!mbar_wait(&S.b8_full[s8], ph8, abort) ||
-                    !mbar_wait(&S.ab_empty[s], ph ^ 1, abort)) {
+                // every lane waits; the vote keeps the warp together if one lane
+                // gave up just as the phase completed for another
+                if (!__all_sync(0xffffffffu, wait(&S.b8_full[s8], ph8) && wait(&S.empty_b[s], ph ^ 1))) {
                     ok = false;
                     break;
                 }
                 const uint8_t* src = tileB8(s8);
                 uint8_t* dst = tileBbf(s);
-                uint4 v[2];
+                uint4 v[kChunks];
 #pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    v[j] = *reinterpret_cast<const uint4*>(src + (ct + 256 * j) * 16);
+                for (int j = 0; j < kChunks; ++j)
+                    v[j] = *reinterpret_cast<const uint4*>(src + (ct + kConvThreads * j) * 16);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int q = ct + 256 * j, row = q >> 2, u0 = 2 * (q & 3);
+                for (int j = 0; j < kChunks; ++j) {
+                    const int q = ct + kConvThreads * j, row = q >> 2, u0 = 2 * (q & 3);
                     uint8_t* line = dst + (row >> 3) * 1024 + (row & 7) * 128;
                     const uint4 o0 = make_uint4(i8x2_to_bf16x2<0>(v[j].x), i8x2_to_bf16x2<1>(v[j].x),
                                                 i8x2_to_bf16x2<0>(v[j].y), i8x2_to_bf16x2<1>(v[j].y));
@@ -320,60 +376,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
+                int good = 1;
                 if (lane == 0) {
-                    mbar_arrive(&S.ab_full[s]);
                     mbar_arrive(&S.b8_empty[s8]);
+                    // the stage is complete in this CTA once its A rows landed too
+                    if (wait(&S.a_full[sa], pha))
+                        mbar_arrive_cluster(full_leader + s * (uint32_t)sizeof(uint64_t));
+                    else
+                        good = 0;
+                }
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    ok = false;
+                    break;
                 }
             }
         }
     } else {
-        // epilogue warps: TMEM lane quadrant = warp % 4, both halves of the tile
+        // epilogue warps: TMEM lane quadrant = warp % 4, the CTA's 128 rows
         const int quad = warp & 3;
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(&S.acc_empty[0]), 0);
         int it = 0;
-        for (int tile = blockIdx.x; tile < total && !*abort; tile += gridDim.x, ++it) {
+        for (int tile = pair; tile < total && !*abort; tile += npairs, ++it) {
             const Tile t = decode_tile(S, E, p.n_tiles, tile);
             const int buf = it & 1;
-            if (!mbar_wait(&S.acc_full[buf], (it >> 1) & 1, abort)) break;
+            if (!__all_sync(0xffffffffu, wait(&S.acc_full[buf], (it >> 1) & 1))) break;
             tc_fence_after();
-            __syncwarp();
-            for (int h = 0; h < t.halves; ++h) {
-                const uint32_t taddr =
-                    tmem + buf * 2 * BN + h * BN + ((uint32_t)(quad * 32) << 16);
-                const int row = t.row0 + h * BH + quad * 32 + lane;
+            if ((int)rank < t.halves) {
+                const uint32_t taddr = tmem + buf * BN + ((uint32_t)(quad * 32) << 16);
+                const int row = t.row0 + (int)rank * BH + quad * 32 + lane;
                 if (MODE == kGateUp) {
-                    const int n0 = t.n * (BN / 2);
+                    const int n0 = t.n * BNC;
                     const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
                     const float* su = sg + p.up_offset;
 #pragma unroll 1
-                    for (int c = 0; c < BN / 2 / 32; ++c) {
+                    for (int c = 0; c < BNC / 32; ++c) {
+                        const int ch = n0 + c * 32;
+                        if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
                         uint32_t gv[32], uv[32];
                         tmem_ld_32x32b_x32(taddr + c * 32, gv);
-                        tmem_ld_32x32b_x32(taddr + BN / 2 + c * 32, uv);
+                        tmem_ld_32x32b_x32(taddr + BNC + c * 32, uv);
                         tmem_ld_wait();
-                        const int ch = n0 + c * 32;
-                        if (ch < p.n_valid) {
-                            uint32_t packed[16];
+                        uint32_t packed[16];
 #pragma unroll
-                            for (int j = 0; j < 32; j += 4) {
-                                const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
-                                const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
-                                const float g0 = g4.x * __uint_as_float(gv[j]);
-                                const float g1 = g4.y * __uint_as_float(gv[j + 1]);
-                                const float g2 = g4.z * __uint_as_float(gv[j + 2]);
-                                const float g3 = g4.w * __uint_as_float(gv[j + 3]);
-                                const float u0 = u4.x * __uint_as_float(uv[j]);
-                                const float u1 = u4.y * __uint_as_float(uv[j + 1]);
-                                const float u2 = u4.z * __uint_as_float(uv[j + 2]);
-                                const float u3 = u4.w * __uint_as_float(uv[j + 3]);
-                                packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-                                packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1],
-                                                    packed[4 * q + 2], packed[4 * q + 3]);
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
+                            const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
+                            const float g0 = g4.x * __uint_as_float(gv[j]);
+                            const float g1 = g4.y * __uint_as_float(gv[j + 1]);
+                            const float g2 = g4.z * __uint_as_float(gv[j + 2]);
+                            const float g3 = g4.w * __uint_as_float(gv[j + 3]);
+                            const float u0 = u4.x * __uint_as_float(uv[j]);
+                            const float u1 = u4.y * __uint_as_float(uv[j + 1]);
+                            const float u2 = u4.z * __uint_as_float(uv[j + 2]);
+                            const float u3 = u4.w * __uint_as_float(uv[j + 3]);
+                            packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                            packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
                         }
+                        uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                                packed[4 * q + 3]);
                     }
                 } else {
                     const int m0 = t.n * BN;
@@ -384,11 +447,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float* sd = p.scale + (size_t)t.e * p.w_rows;
 #pragma unroll 1
                     for (int c = 0; c < BN / 32; ++c) {
+                        const int m = m0 + c * 32;
+                        if (m >= p.n_valid) break;  // n_valid is a multiple of 64
                         uint32_t v[32];
                         tmem_ld_32x32b_x32(taddr + c * 32, v);
                         tmem_ld_wait();
-                        const int m = m0 + c * 32;
-                        if (valid && m < p.n_valid) {
+                        if (valid) {
                             float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {
@@ -406,31 +470,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+            if (lane == 0) mbar_arrive_cluster(acc_empty_leader + buf * (uint32_t)sizeof(uint64_t));
         }
     }
 
+    // Neither CTA frees its TMEM or leaves before every MMA (which reads both
+    // CTAs' shared memory and writes both CTAs' TMEM) and every arrival on the
+    // partner's barriers is done: the issuer waited for its drain commit above,
+    // and the cluster barrier orders everything before it.
     tc_fence_before();
-    __syncthreads();
+    __syncwarp();
+    cluster_sync();
     if (threadIdx.x == 0 && S.abort) flag_error(p.err, kErrTimeout);
     if (warp == kWarpMMA) {
-        __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
 // ----------------------------------------------------------------------------- host side
 
+// CTA pairs resident at once (one CTA per SM), at most `want`.  The kernel's
+// cluster shape is fixed at compile time, so the query leaves it unspecified.
+template <int MODE>
+int resident_pairs(int num_sms, int want) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * want);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, k_grouped_gemm<MODE>, &cfg) != cudaSuccess ||
+        clusters < 1)
+        clusters = num_sms / 2;
+    return clusters < want ? clusters : want;
+}
+
 template <int MODE>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmParams& p,
-                        int num_sms, cudaStream_t stream) {
+                        int num_sms, int tiles, cudaStream_t stream) {
+    if (tiles <= 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    k_grouped_gemm<MODE><<<num_sms, kThreads, kSmemBytes, stream>>>(a, b, p);
+    const int pairs = resident_pairs<MODE>(num_sms, tiles);
+    k_grouped_gemm<MODE><<<2 * pairs, kThreads, kSmemBytes, stream>>>(a, b, p);
     note_launch();
     return cudaGetLastError();
+}
+
+// Pair tiles of one GEMM: per expert, ceil(128-row halves / 2) m-tiles times
+// n_tiles (the kernel derives the same count from the padded offsets; the
+// host only needs an upper bound to size the grid).
+int64_t tile_bound(const PrefillArgs& a, int n_tiles) {
+    const int64_t halves = a.rows_padded / BH;
+    return (halves / 2 + a.E) * n_tiles;
 }
 
 }  // namespace
@@ -454,10 +547,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
         encode_2d(&mA1, a.xperm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.d, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
         encode_2d(&mB1, a.wgu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * 2 * a.f, a.d,
-                 BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                 BNC, BK, CU_TENSOR_MAP_SWIZZLE_NONE) &&
         encode_2d(&mA2, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.rows_padded, a.f, BH, BK,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-        encode_2d(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BN, BK,
+        encode_2d(&mB2, a.wd, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.d, a.f, BNC, BK,
                  CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
 
@@ -466,7 +559,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     g1.E = a.E;
     g1.K = (int)a.d;
     g1.n_valid = (int)a.f;
-    g1.n_tiles = (int)((a.f + BN / 2 - 1) / (BN / 2));
+    g1.n_tiles = (int)((a.f + BNC - 1) / BNC);
     g1.w_rows = (int)(2 * a.f);
     g1.up_offset = (int)a.f;
     g1.poff = a.padded_offsets;
@@ -476,8 +569,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     g1.gates = a.gates;
     g1.H = static_cast<uint16_t*>(a.H);
     g1.err = a.err;
+    g1.wait_cycles = a.wait_cycles > 0 ? a.wait_cycles : kWaitCycles;
+    g1.fault_tile = a.fault_tile;
     if (a.mark) a.mark(2, false, stream);
-    err = launch_gemm<kGateUp>(mA1, mB1, g1, a.num_sms, stream);
+    err = launch_gemm<kGateUp>(mA1, mB1, g1, a.num_sms, (int)tile_bound(a, g1.n_tiles), stream);
     if (a.mark) a.mark(2, true, stream);
     if (err != cudaSuccess) return err;
 
@@ -491,8 +586,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     g2.scale = a.sd;
     g2.H = nullptr;
     g2.Y = a.Yg;
+    g2.fault_tile = -1;
     if (a.mark) a.mark(3, false, stream);
-    err = launch_gemm<kDown>(mA2, mB2, g2, a.num_sms, stream);
+    err = launch_gemm<kDown>(mA2, mB2, g2, a.num_sms, (int)tile_bound(a, g2.n_tiles), stream);
     if (a.mark) a.mark(3, true, stream);
     if (err != cudaSuccess) return err;
 

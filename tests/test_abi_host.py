@@ -126,3 +126,13 @@ def test_launch_counter_counts_nothing_for_rejected_calls():
     assert lib.jmoe_quantize(None, 4, 16, GOOD, GOOD, None) == jm.JMOE_EINVAL
     assert lib.jmoe_permute(GOOD, 4, 2, 16, None, GOOD, GOOD, None) == jm.JMOE_EINVAL
     assert jm.jmoe_launch_count() == n0
+
+
+def test_stall_hook_validation():
+    lib = jm.load()
+    assert lib.jmoe_test_stall(3, 2_000_000) == jm.JMOE_EINVAL
+    assert lib.jmoe_test_stall(-1, 2_000_000) == jm.JMOE_EINVAL
+    assert lib.jmoe_test_stall(jm.JMOE_STALL_TENSOR_GEMM, 10) == jm.JMOE_EINVAL
+    assert lib.jmoe_test_stall(jm.JMOE_STALL_DECODE_GEMV, 10 ** 10) == jm.JMOE_EINVAL
+    assert lib.jmoe_test_stall(jm.JMOE_STALL_DECODE_GEMV, 2_000_000) == jm.JMOE_OK
+    assert lib.jmoe_test_stall(0, 0) == jm.JMOE_OK  # disarms

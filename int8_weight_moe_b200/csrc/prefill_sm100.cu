@@ -15,39 +15,43 @@
 //
 // A cluster of two CTAs (a pair, on two SMs) computes one tile of 256 token
 // rows x 256 output columns with CTA-pair MMAs (tcgen05.mma.cta_group::2,
-// M = 256, N = 256, K = 16): each CTA holds 128 of the token rows (A) and
-// converts 128 of the 256 weight rows (B); the tensor cores of both SMs read
-// both CTAs' halves, and each CTA's TMEM receives its 128 rows x 256 columns.
-// Per 64-wide k-step a CTA's shared memory carries 16 KB of A (TMA), 8 KB of
-// INT8 (TMA), the converters' 8 KB read + 16 KB write, and 32 KB of MMA
-// operand reads: 80 KB for 2 x 128 x 256 x 64 multiply-adds, about half of
-// what one CTA holding the whole 128-wide weight tile for 256 rows moves per
-// multiply-add, and each weight is converted once per 256 token rows.
+// M = 256, K = 16): each CTA holds 128 of the token rows (A) and converts 128
+// of the 256 weight rows (B); the tensor cores of both SMs read both CTAs'
+// halves, and each CTA's TMEM receives its 128 rows x 256 columns.  Two
+// issuing threads each own half of the columns (N = 128 per MMA), so that
+// while one waits for its next stage the MMAs the other queued keep the
+// tensor pipe busy.  Per 64-wide k-step a CTA's shared memory carries 16 KB
+// of A (TMA), 8 KB of INT8 (TMA), the converters' 8 KB read + 16 KB write,
+// and the MMAs' operand reads; each weight is converted once per 256 token
+// rows (half the conversions of a single CTA holding 256 rows and the whole
+// 128-wide weight tile, and less shared-memory traffic per multiply-add).
 //
-// Warps of each CTA (15):
+// Warps of each CTA (16):
 //   warp 0      TMA producer of the CTA's A rows [128 x 64 k] bf16 (skipped
 //               when the CTA's half of the tile lies past the expert's rows)
-//   warp 1      TMEM allocator (both CTAs); MMA issuer (even CTA only)
+//   warp 1      TMEM allocator (both CTAs); first MMA issuer (even CTA only)
 //   warp 2      TMA producer of the CTA's INT8 weight rows [128 x 64 k]
 //   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled), in two
 //               groups of 4 that take alternate k-steps
 //   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
+//   warp 15     second MMA issuer (even CTA only)
 //
 // Gate/up tiles: the even CTA converts 128 gate channels, the odd CTA the
-// same 128 up channels, so TMEM columns c and 128 + c of a row hold the gate
-// and up sums of one channel (the SwiGLU pair sits in one thread).  Down
-// tiles: 256 output channels, 128 per CTA.  Expert rows are padded to 128; a
-// pair tile whose second half lies past the expert's rows leaves the odd
-// CTA's A stale and stores nothing for it (the MMA rows are independent).
+// same 128 up channels, so a row's gate and up sums of one channel sit in
+// TMEM columns of the same thread (the SwiGLU pair).  Down tiles: 256
+// output channels, 128 per CTA.  Expert rows are padded to 128; a pair tile
+// whose second half lies past the expert's rows leaves the odd CTA's A
+// stale and stores nothing for it (the MMA rows are independent).
 //
 // Synchronisation (mbarriers; every wait is bounded and a wait that runs out
 // raises the abort flags of both CTAs, after which every role drains its own
 // copies and the pair frees its TMEM):
 //   a_full[s]   (each CTA)  its A copy of stage s landed
+//   empty_a[s]  (each CTA)  the MMAs reading A stage s are done (commit multicast)
 //   b8_full/b8_empty (each CTA)  INT8 ring between its TMA and its converters
 //   full[s]     (even CTA)  the converter warps of both CTAs wrote stage s's
 //                           BF16 weights after seeing their CTA's A land
-//   empty[s]    (each CTA)  the MMAs of stage s are done (commit multicast)
+//   empty_b[s]  (each CTA)  the MMAs reading BF16 stage s are done
 //   acc_full[b] (each CTA)  accumulator b is final (commit multicast)
 //   acc_empty[b] (even CTA) the epilogue warps of both CTAs read it
 // Two accumulators of 256 fp32 columns (all 512 TMEM columns) let the
@@ -95,14 +99,24 @@ constexpr int kSmemA = kStagesA * kABytes;
 constexpr int kSmemB = kStagesB * kBbfBytes;
 constexpr int kSmem8 = kStages8 * kB8Bytes;
 constexpr uint32_t kTmemCols = 512;   // 2 accumulators x 256 fp32 columns
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
+// MMA-issuing threads (in the even CTA), each owning an N slice of BNI
+// columns of the accumulator: while one thread waits for its next stage,
+// the MMAs the other queued keep the tensor pipe busy.
+#ifndef JMOE_GEMM_ISSUERS
+#define JMOE_GEMM_ISSUERS 2
+#endif
+constexpr int kIssuers = JMOE_GEMM_ISSUERS;
+constexpr int BNI = BN / kIssuers;    // MMA N of one issuer (half from each CTA)
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BNI);
+static_assert(kIssuers == 1 || kIssuers == 2, "one or two issuers");
 constexpr uint16_t kPairMask = 0x3;   // both CTAs of the cluster
 
 constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
 constexpr int kConvWarp0 = 3, kConvGroupWarps = 4, kConvWarps = 2 * kConvGroupWarps;
 constexpr int kConvThreads = kConvGroupWarps * 32;  // threads of one converter group
 constexpr int kEpiWarp0 = kConvWarp0 + kConvWarps, kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+constexpr int kWarpMMA2 = kEpiWarp0 + kEpiWarps;  // second issuer (kIssuers == 2)
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps + kIssuers - 1) * 32;
 constexpr int kChunks = kB8Bytes / 16 / kConvThreads;  // 16-byte INT8 chunks per thread per k-step
 constexpr int kMaxE = 64;
 
@@ -200,21 +214,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesB; ++i) {
             mbar_init(&S.full[i], 2 * kConvGroupWarps);  // one converter group of each CTA
-            mbar_init(&S.empty_b[i], 1);                  // the MMA commit
+            mbar_init(&S.empty_b[i], kIssuers);           // the issuers' MMA commits
         }
         for (int i = 0; i < kStagesA; ++i) {
             mbar_init(&S.a_full[i], 1);                   // the A producer (+ TMA bytes)
-            mbar_init(&S.empty_a[i], 1);                  // the MMA commit
+            mbar_init(&S.empty_a[i], kIssuers);           // the issuers' MMA commits
         }
         for (int i = 0; i < kStages8; ++i) {
             mbar_init(&S.b8_full[i], 1);
             mbar_init(&S.b8_empty[i], kConvGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.acc_full[i], 1);
+            mbar_init(&S.acc_full[i], kIssuers);
             mbar_init(&S.acc_empty[i], 2 * kEpiWarps);
         }
-        mbar_init(&S.drain, 1);
+        mbar_init(&S.drain, kIssuers);
         S.abort = 0;
         fence_mbar_init();
     }
@@ -295,8 +309,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (uint32_t h = (g > (uint32_t)kStages8 ? g - kStages8 : 0); h < g; ++h)
                 wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1, limit);
         }
-    } else if (warp == kWarpMMA) {
+    } else if (warp == kWarpMMA || (kIssuers == 2 && warp == kWarpMMA2)) {
         if (rank == 0 && lane == 0) {
+            // issuer h: accumulator columns [h BNI, (h+1) BNI), i.e. B rows
+            // [h BNI/2, (h+1) BNI/2) of each CTA's weight tile
+            const int h = warp == kWarpMMA ? 0 : 1;
             uint32_t g = 0;
             int it = 0;
             for (int tile = pair; tile < total && !*abort; tile += npairs, ++it) {
@@ -304,7 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!mbar_wait_pair(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, peer_abort, limit))
                     break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * BN;
+                const uint32_t d_tmem = tmem + buf * BN + h * BNI;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int sa = g % kStagesA;
@@ -316,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(tileA(sa));
-                    const uint32_t b0 = smem_u32(tileBbf(s));
+                    const uint32_t b0 = smem_u32(tileBbf(s)) + h * (BNI / 2) * (BK * 2);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
                         mma_bf16_ss_pair(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
@@ -412,9 +429,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < BNC / 32; ++c) {
                         const int ch = n0 + c * 32;
                         if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
+                        // gate channel n0 + r is B row r of the even CTA: column
+                        // (r / (BNI/2)) BNI + r % (BNI/2); its up channel is the odd
+                        // CTA's row r, BNI/2 columns further
+                        const int r0 = c * 32;
+                        const uint32_t gcol = (r0 / (BNI / 2)) * BNI + r0 % (BNI / 2);
                         uint32_t gv[32], uv[32];
-                        tmem_ld_32x32b_x32(taddr + c * 32, gv);
-                        tmem_ld_32x32b_x32(taddr + BNC + c * 32, uv);
+                        tmem_ld_32x32b_x32(taddr + gcol, gv);
+                        tmem_ld_32x32b_x32(taddr + gcol + BNI / 2, uv);
                         tmem_ld_wait();
                         uint32_t packed[16];
 #pragma unroll
@@ -447,12 +469,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const float* sd = p.scale + (size_t)t.e * p.w_rows;
 #pragma unroll 1
                     for (int c = 0; c < BN / 32; ++c) {
-                        const int m = m0 + c * 32;
-                        if (m >= p.n_valid) break;  // n_valid is a multiple of 64
+                        // column 32c: issuer slice hh, CTA half `half` of it, row j0
+                        // of that CTA's weight tile -> channel m0 + half 128 + hh BNI/2 + j0
+                        const int hh = (c * 32) / BNI, within = (c * 32) % BNI;
+                        const int m = m0 + (within / (BNI / 2)) * BNC + hh * (BNI / 2) +
+                                      within % (BNI / 2);
                         uint32_t v[32];
                         tmem_ld_32x32b_x32(taddr + c * 32, v);
                         tmem_ld_wait();
-                        if (valid) {
+                        if (valid && m < p.n_valid) {
                             float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
 #pragma unroll
                             for (int q = 0; q < 8; ++q) {

@@ -85,8 +85,12 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// silu(z) = z / (1 + e^-z), with the fast exponential and the fast division
+// (a reciprocal and a multiply, within 2 ulp of the quotient in fp32): the
+// result is rounded to bf16 (8 significant bits) before anyone reads it.
+// For z < -88, e^-z overflows to inf and the quotient is 0.
 __device__ __forceinline__ float silu_f32(float z) {
-    return z / (1.0f + __expf(-z));
+    return __fdividef(z, 1.0f + __expf(-z));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -13,50 +13,55 @@
 // (sum_k x_k (q_k s) = s sum_k x_k q_k).  Activations stay BF16 (step 4);
 // accumulation is fp32 in TMEM.
 //
-// A cluster of two CTAs (a pair, on two SMs) computes one tile of 256 token
+// A cluster of two CTAs (a pair, on two SMs) computes one tile of 512 token
 // rows x 256 output columns with CTA-pair MMAs (tcgen05.mma.cta_group::2,
-// M = 256, K = 16): each CTA holds 128 of the token rows (A) and converts 128
-// of the 256 weight rows (B); the tensor cores of both SMs read both CTAs'
-// halves, and each CTA's TMEM receives its 128 rows x 256 columns.  Two
-// issuing threads each own half of the columns (N = 128 per MMA), so that
-// while one waits for its next stage the MMAs the other queued keep the
-// tensor pipe busy.  Per 64-wide k-step a CTA's shared memory carries 16 KB
-// of A (TMA), 8 KB of INT8 (TMA), the converters' 8 KB read + 16 KB write,
-// and the MMAs' operand reads; each weight is converted once per 256 token
-// rows (half the conversions of a single CTA holding 256 rows and the whole
-// 128-wide weight tile, and less shared-memory traffic per multiply-add).
+// M = 256, N = 256, K = 16).  The tile's rows are four quarters of 128: CTA
+// r holds quarters r and 2 + r of A and converts 128 of the 256 weight rows
+// (B).  Issuer h (two threads of the even CTA) multiplies quarters 2h (even
+// CTA) and 2h + 1 (odd CTA) by the whole B into accumulator h; the tensor
+// cores of both SMs read both CTAs' operands, and each CTA's TMEM receives
+// its rows x 256 columns.  While one issuer waits for its next stage the
+// MMAs the other queued keep the tensor pipe busy.  Every converted weight
+// tile feeds both issuers: each weight is converted once per 512 token rows,
+// and per 64-wide k-step a CTA's shared memory carries 32 KB of A (TMA),
+// 8 KB of INT8 (TMA), the converters' 8 KB read + 16 KB write and 64 KB of
+// MMA operand reads for 256 x 256 x 64 multiply-adds.
 //
 // Warps of each CTA (16):
-//   warp 0      TMA producer of the CTA's A rows [128 x 64 k] bf16 (skipped
-//               when the CTA's half of the tile lies past the expert's rows)
-//   warp 1      TMEM allocator (both CTAs); first MMA issuer (even CTA only)
+//   warp 0      TMA producer of the CTA's two A quarters [128 x 64 k] bf16
+//               (a quarter past the expert's rows is not loaded)
+//   warp 1      TMEM allocator (both CTAs); issuer 0 (even CTA only)
 //   warp 2      TMA producer of the CTA's INT8 weight rows [128 x 64 k]
 //   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled), in two
 //               groups of 4 that take alternate k-steps
 //   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
-//   warp 15     second MMA issuer (even CTA only)
+//   warp 15     issuer 1 (even CTA only)
 //
 // Gate/up tiles: the even CTA converts 128 gate channels, the odd CTA the
-// same 128 up channels, so a row's gate and up sums of one channel sit in
-// TMEM columns of the same thread (the SwiGLU pair).  Down tiles: 256
-// output channels, 128 per CTA.  Expert rows are padded to 128; a pair tile
-// whose second half lies past the expert's rows leaves the odd CTA's A
-// stale and stores nothing for it (the MMA rows are independent).
+// same 128 up channels, so TMEM columns r and 128 + r of a row hold the gate
+// and up sums of one channel (the SwiGLU pair sits in one thread).  Down
+// tiles: 256 output channels, 128 per CTA.  Expert rows are padded to 128.
+// An issuer whose two quarters lie past the expert's rows issues no MMAs
+// for the tile (it still takes part in every stage's hand-over); a quarter
+// of the odd CTA past the expert's rows leaves that CTA's A stale and
+// nothing is stored for it (the MMA rows are independent).
 //
 // Synchronisation (mbarriers; every wait is bounded and a wait that runs out
 // raises the abort flags of both CTAs, after which every role drains its own
 // copies and the pair frees its TMEM):
-//   a_full[s]   (each CTA)  its A copy of stage s landed
-//   empty_a[s]  (each CTA)  the MMAs reading A stage s are done (commit multicast)
+//   a_full[s]   (each CTA)  its A copies of stage s landed
+//   empty_a[s]  (each CTA)  both issuers' MMAs reading A stage s are done
+//                           (commit multicast)
 //   b8_full/b8_empty (each CTA)  INT8 ring between its TMA and its converters
 //   full[s]     (even CTA)  the converter warps of both CTAs wrote stage s's
 //                           BF16 weights after seeing their CTA's A land
-//   empty_b[s]  (each CTA)  the MMAs reading BF16 stage s are done
-//   acc_full[b] (each CTA)  accumulator b is final (commit multicast)
-//   acc_empty[b] (even CTA) the epilogue warps of both CTAs read it
-// Two accumulators of 256 fp32 columns (all 512 TMEM columns) let the
-// epilogue of one tile overlap the main loop of the next.  Tiles are visited
-// expert by expert in groups of 16 m-tiles (see decode_tile).  No TMA load is
+//   empty_b[s]  (each CTA)  both issuers' MMAs reading BF16 stage s are done
+//   acc_full[h] (each CTA)  accumulator h is final (issuer h's commit multicast)
+//   acc_empty[h] (even CTA) the epilogue warps of both CTAs read it
+// The two accumulators of 256 fp32 columns take all 512 TMEM columns; the
+// epilogue reads accumulator 0 first, so issuer 0 starts its next tile while
+// the epilogue still reads accumulator 1.  Tiles are visited expert by
+// expert in groups of 16 m-tiles (see decode_tile).  No TMA load is
 // multicast; every copy reads global memory into its own CTA.
 #include <cuda.h>
 
@@ -70,45 +75,39 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BH = 128;       // token rows of one CTA (a half of the pair tile)
-constexpr int BM = 2 * BH;    // token rows of a pair tile
+constexpr int BH = 128;       // token rows of one quarter of the pair tile (one CTA, one issuer)
+constexpr int BM = 4 * BH;    // token rows of a pair tile: each CTA holds 2 quarters
 constexpr int BN = 256;       // MMA N: output columns of a pair tile
 constexpr int BNC = BN / 2;   // weight rows each CTA converts
 constexpr int BK = 64;
-// Ring depths.  A (activations, mostly L2 hits) and the INT8 weights (HBM)
-// are fetched several k-steps ahead of the MMAs: a k-step's MMAs take about
-// 512 cycles, less than a TMA round trip under load.  The converted BF16
-// weights need only cover the converters' latency.  Even depths: stage s of
-// the BF16 and INT8 rings always goes to converter group s & 1.
+// Ring depths (4 x 32 KB of A, 4 x 16 KB of BF16 weights, 4 x 8 KB of INT8
+// weights: 224 KB).  A k-step's MMAs take about 1024 cycles.  Even depths:
+// stage s of the BF16 and INT8 rings always goes to converter group s & 1.
 #ifndef JMOE_GEMM_STAGES_A
-#define JMOE_GEMM_STAGES_A 6
+#define JMOE_GEMM_STAGES_A 4
 #endif
 #ifndef JMOE_GEMM_STAGES_B
-#define JMOE_GEMM_STAGES_B 6
+#define JMOE_GEMM_STAGES_B 4
 #endif
 #ifndef JMOE_GEMM_STAGES_8
 #define JMOE_GEMM_STAGES_8 4
 #endif
 constexpr int kStagesA = JMOE_GEMM_STAGES_A, kStagesB = JMOE_GEMM_STAGES_B;
 constexpr int kStages8 = JMOE_GEMM_STAGES_8;
-constexpr int kGroupM = 16;  // pair m-tiles per raster group (activation rows kept in L2)
+#ifndef JMOE_GEMM_GROUP_M
+#define JMOE_GEMM_GROUP_M 16
+#endif
+constexpr int kGroupM = JMOE_GEMM_GROUP_M;  // pair m-tiles per raster group (rows kept in L2)
 constexpr int kABytes = BH * BK * 2;     // 16 KB
 constexpr int kBbfBytes = BNC * BK * 2;  // 16 KB
 constexpr int kB8Bytes = BNC * BK;       // 8 KB
-constexpr int kSmemA = kStagesA * kABytes;
+constexpr int kAStage = 2 * kABytes;     // the CTA's two quarters
+constexpr int kSmemA = kStagesA * kAStage;
 constexpr int kSmemB = kStagesB * kBbfBytes;
 constexpr int kSmem8 = kStages8 * kB8Bytes;
 constexpr uint32_t kTmemCols = 512;   // 2 accumulators x 256 fp32 columns
-// MMA-issuing threads (in the even CTA), each owning an N slice of BNI
-// columns of the accumulator: while one thread waits for its next stage,
-// the MMAs the other queued keep the tensor pipe busy.
-#ifndef JMOE_GEMM_ISSUERS
-#define JMOE_GEMM_ISSUERS 2
-#endif
-constexpr int kIssuers = JMOE_GEMM_ISSUERS;
-constexpr int BNI = BN / kIssuers;    // MMA N of one issuer (half from each CTA)
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BNI);
-static_assert(kIssuers == 1 || kIssuers == 2, "one or two issuers");
+constexpr int kIssuers = 2;           // issuer h: quarters 2h, 2h+1 (M = 256), N = 256
+constexpr uint32_t kIdesc = idesc_bf16_f32(2 * BH, BN);
 constexpr uint16_t kPairMask = 0x3;   // both CTAs of the cluster
 
 constexpr int kWarpProdA = 0, kWarpMMA = 1, kWarpProdB = 2;
@@ -161,18 +160,18 @@ constexpr int kSmemBytes = kSmemA + kSmemB + kSmem8 + (int)sizeof(Shared) + 1024
 static_assert(kSmemBytes <= 232448, "more shared memory than a CTA can have");
 
 struct Tile {
-    int e, row0, n, halves;  // halves: 1 or 2 valid 128-row halves
+    int e, row0, n, quarters;  // quarters: 1..4 valid 128-row quarters
 };
 
 // Tile order inside an expert: groups of kGroupM m-tiles; within a group all
 // n-tiles, m fastest.  The pairs of a wave then share a few weight tiles and
-// at most kGroupM x 256 activation rows, which stay in L2.
+// at most kGroupM x 512 activation rows, which stay in L2.
 __device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int n_tiles, int tile) {
     int e = 0;
     while (e + 1 < E && s.tile_start[e + 1] <= tile) ++e;
     const int local = tile - s.tile_start[e];
-    const int nh = (s.poff[e + 1] - s.poff[e]) / BH;  // 128-row halves of this expert
-    const int mt = (nh + 1) / 2;
+    const int nh = (s.poff[e + 1] - s.poff[e]) / BH;  // 128-row quarters of this expert
+    const int mt = (nh + 3) / 4;
     const int mg = local / (kGroupM * n_tiles);
     const int gm = min(kGroupM, mt - mg * kGroupM);  // m-tiles in this group
     const int rem = local - mg * kGroupM * n_tiles;
@@ -181,7 +180,7 @@ __device__ __forceinline__ Tile decode_tile(const Shared& s, int E, int n_tiles,
     t.n = rem / gm;
     const int m = mg * kGroupM + rem % gm;
     t.row0 = s.poff[e] + m * BM;
-    t.halves = min(2, nh - 2 * m);
+    t.quarters = min(4, nh - 4 * m);
     return t;
 }
 
@@ -200,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Shared& S = *reinterpret_cast<Shared*>(smem + kSmemA + kSmemB + kSmem8);
-    auto tileA = [&](int s) { return smem + s * kABytes; };
+    auto tileA = [&](int s) { return smem + s * kAStage; };
     auto tileBbf = [&](int s) { return smem + kSmemA + s * kBbfBytes; };
     auto tileB8 = [&](int s) { return smem + kSmemA + kSmemB + s * kB8Bytes; };
 
@@ -225,7 +224,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&S.b8_empty[i], kConvGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.acc_full[i], kIssuers);
+            mbar_init(&S.acc_full[i], 1);  // issuer i's commit
             mbar_init(&S.acc_empty[i], 2 * kEpiWarps);
         }
         mbar_init(&S.drain, kIssuers);
@@ -245,7 +244,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int run = 0;
         for (int e = 0; e < E; ++e) {
             S.tile_start[e] = run;
-            run += ((S.poff[e + 1] - S.poff[e]) / BH + 1) / 2 * p.n_tiles;
+            run += ((S.poff[e + 1] - S.poff[e]) / BH + 3) / 4 * p.n_tiles;
         }
         S.tile_start[E] = run;
     }
@@ -271,14 +270,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t g = 0;
             for (int tile = pair; tile < total && !*abort; tile += npairs) {
                 const Tile t = decode_tile(S, E, p.n_tiles, tile);
-                const bool mine = (int)rank < t.halves;
+                // this CTA's quarters of the tile: 2h + rank for h = 0, 1
+                const int nq = ((int)rank < t.quarters) + (2 + (int)rank < t.quarters);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStagesA;
                     const uint32_t ph = (g / kStagesA) & 1;
                     if (!wait(&S.empty_a[s], ph ^ 1)) break;
-                    if (mine) {
-                        mbar_arrive_expect_tx(&S.a_full[s], kABytes);
-                        tma_load_2d(tileA(s), &tmA, &S.a_full[s], kb * BK, t.row0 + (int)rank * BH);
+                    if (nq > 0) {
+                        mbar_arrive_expect_tx(&S.a_full[s], nq * kABytes);
+                        for (int h = 0; h < nq; ++h)
+                            tma_load_2d(tileA(s) + h * kABytes, &tmA, &S.a_full[s], kb * BK,
+                                        t.row0 + (2 * h + (int)rank) * BH);
                     } else {
                         mbar_arrive(&S.a_full[s]);
                     }
@@ -309,19 +311,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (uint32_t h = (g > (uint32_t)kStages8 ? g - kStages8 : 0); h < g; ++h)
                 wait_drain(&S.b8_full[h % kStages8], (h / kStages8) & 1, limit);
         }
-    } else if (warp == kWarpMMA || (kIssuers == 2 && warp == kWarpMMA2)) {
+    } else if (warp == kWarpMMA || warp == kWarpMMA2) {
         if (rank == 0 && lane == 0) {
-            // issuer h: accumulator columns [h BNI, (h+1) BNI), i.e. B rows
-            // [h BNI/2, (h+1) BNI/2) of each CTA's weight tile
+            // issuer h: M slice h (quarter 2h from this CTA, 2h + 1 from the
+            // partner) into accumulator h; an issuer whose slice lies past the
+            // expert's rows still waits and commits every stage, without MMAs
             const int h = warp == kWarpMMA ? 0 : 1;
             uint32_t g = 0;
-            int it = 0;
-            for (int tile = pair; tile < total && !*abort; tile += npairs, ++it) {
-                const int buf = it & 1;
-                if (!mbar_wait_pair(&S.acc_empty[buf], ((it >> 1) & 1) ^ 1, abort, peer_abort, limit))
-                    break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + buf * BN + h * BNI;
+            int uses = 0;
+            for (int tile = pair; tile < total && !*abort; tile += npairs) {
+                const bool active = 2 * h < decode_tile(S, E, p.n_tiles, tile).quarters;
+                if (active) {
+                    if (!mbar_wait_pair(&S.acc_empty[h], (uses & 1) ^ 1, abort, peer_abort, limit))
+                        break;
+                    tc_fence_after();
+                }
+                const uint32_t d_tmem = tmem + h * BN;
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int sa = g % kStagesA;
@@ -332,17 +337,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(tileA(sa));
-                    const uint32_t b0 = smem_u32(tileBbf(s)) + h * (BNI / 2) * (BK * 2);
+                    const uint32_t a0 = smem_u32(tileA(sa)) + h * kABytes;
+                    const uint32_t b0 = smem_u32(tileBbf(s));
+                    if (active) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_bf16_ss_pair(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
-                                         kIdesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_bf16_ss_pair(d_tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32),
+                                             kIdesc, (kb | kk) != 0);
+                    }
                     mma_commit_pair_mc(&S.empty_a[sa], kPairMask);
                     mma_commit_pair_mc(&S.empty_b[s], kPairMask);
                 }
                 if (!ok) break;
-                mma_commit_pair_mc(&S.acc_full[buf], kPairMask);
+                if (active) {
+                    mma_commit_pair_mc(&S.acc_full[h], kPairMask);
+                    ++uses;
+                }
             }
             // every MMA done (both CTAs' TMEM written, both CTAs' shared memory read)
             mma_commit_pair(&S.drain);
@@ -409,93 +419,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // epilogue warps: TMEM lane quadrant = warp % 4, the CTA's 128 rows
+        // epilogue warps: TMEM lane quadrant = warp % 4; per tile, accumulator h
+        // holds this CTA's quarter 2h + rank (128 rows x 256 columns)
         const int quad = warp & 3;
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(&S.acc_empty[0]), 0);
-        int it = 0;
-        for (int tile = pair; tile < total && !*abort; tile += npairs, ++it) {
+        int uses[2] = {0, 0};
+        bool ok = true;
+        for (int tile = pair; tile < total && ok && !*abort; tile += npairs) {
             const Tile t = decode_tile(S, E, p.n_tiles, tile);
-            const int buf = it & 1;
-            if (!__all_sync(0xffffffffu, wait(&S.acc_full[buf], (it >> 1) & 1))) break;
-            tc_fence_after();
-            if ((int)rank < t.halves) {
-                const uint32_t taddr = tmem + buf * BN + ((uint32_t)(quad * 32) << 16);
-                const int row = t.row0 + (int)rank * BH + quad * 32 + lane;
-                if (MODE == kGateUp) {
-                    const int n0 = t.n * BNC;
-                    const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
-                    const float* su = sg + p.up_offset;
+            for (int h = 0; h < 2; ++h) {
+                if (2 * h >= t.quarters) break;  // issuer h had no rows in this tile
+                if (!__all_sync(0xffffffffu, wait(&S.acc_full[h], uses[h] & 1))) {
+                    ok = false;
+                    break;
+                }
+                ++uses[h];
+                tc_fence_after();
+                const int q = 2 * h + (int)rank;
+                if (q < t.quarters) {
+                    const uint32_t taddr = tmem + h * BN + ((uint32_t)(quad * 32) << 16);
+                    const int row = t.row0 + q * BH + quad * 32 + lane;
+                    if (MODE == kGateUp) {
+                        const int n0 = t.n * BNC;
+                        const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
+                        const float* su = sg + p.up_offset;
 #pragma unroll 1
-                    for (int c = 0; c < BNC / 32; ++c) {
-                        const int ch = n0 + c * 32;
-                        if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
-                        // gate channel n0 + r is B row r of the even CTA: column
-                        // (r / (BNI/2)) BNI + r % (BNI/2); its up channel is the odd
-                        // CTA's row r, BNI/2 columns further
-                        const int r0 = c * 32;
-                        const uint32_t gcol = (r0 / (BNI / 2)) * BNI + r0 % (BNI / 2);
-                        uint32_t gv[32], uv[32];
-                        tmem_ld_32x32b_x32(taddr + gcol, gv);
-                        tmem_ld_32x32b_x32(taddr + gcol + BNI / 2, uv);
-                        tmem_ld_wait();
-                        uint32_t packed[16];
+                        for (int c = 0; c < BNC / 32; ++c) {
+                            const int ch = n0 + c * 32;
+                            if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
+                            // gate channel n0 + r: column r (the even CTA's B row r);
+                            // its up channel: column 128 + r (the odd CTA's row r)
+                            uint32_t gv[32], uv[32];
+                            tmem_ld_32x32b_x32(taddr + c * 32, gv);
+                            tmem_ld_32x32b_x32(taddr + BNC + c * 32, uv);
+                            tmem_ld_wait();
+                            uint32_t packed[16];
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
-                            const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
-                            const float g0 = g4.x * __uint_as_float(gv[j]);
-                            const float g1 = g4.y * __uint_as_float(gv[j + 1]);
-                            const float g2 = g4.z * __uint_as_float(gv[j + 2]);
-                            const float g3 = g4.w * __uint_as_float(gv[j + 3]);
-                            const float u0 = u4.x * __uint_as_float(uv[j]);
-                            const float u1 = u4.y * __uint_as_float(uv[j + 1]);
-                            const float u2 = u4.z * __uint_as_float(uv[j + 2]);
-                            const float u3 = u4.w * __uint_as_float(uv[j + 3]);
-                            packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-                            packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
+                            for (int j = 0; j < 32; j += 4) {
+                                const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
+                                const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
+                                const float g0 = g4.x * __uint_as_float(gv[j]);
+                                const float g1 = g4.y * __uint_as_float(gv[j + 1]);
+                                const float g2 = g4.z * __uint_as_float(gv[j + 2]);
+                                const float g3 = g4.w * __uint_as_float(gv[j + 3]);
+                                const float u0 = u4.x * __uint_as_float(uv[j]);
+                                const float u1 = u4.y * __uint_as_float(uv[j + 1]);
+                                const float u2 = u4.z * __uint_as_float(uv[j + 2]);
+                                const float u3 = u4.w * __uint_as_float(uv[j + 3]);
+                                packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                                packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
+                            }
+                            uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq)
+                                dst[qq] = make_uint4(packed[4 * qq], packed[4 * qq + 1], packed[4 * qq + 2],
+                                                     packed[4 * qq + 3]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                                                packed[4 * q + 3]);
-                    }
-                } else {
-                    const int m0 = t.n * BN;
-                    const int r = row - S.poff[t.e];
-                    const bool valid = r < S.off[t.e + 1] - S.off[t.e];
-                    const int a = valid ? p.perm[S.off[t.e] + r] : 0;
-                    const float gate = valid ? p.gates[a] : 0.0f;
-                    const float* sd = p.scale + (size_t)t.e * p.w_rows;
+                    } else {
+                        const int m0 = t.n * BN;
+                        const int r = row - S.poff[t.e];
+                        const bool valid = r < S.off[t.e + 1] - S.off[t.e];
+                        const int a = valid ? p.perm[S.off[t.e] + r] : 0;
+                        const float gate = valid ? p.gates[a] : 0.0f;
+                        const float* sd = p.scale + (size_t)t.e * p.w_rows;
 #pragma unroll 1
-                    for (int c = 0; c < BN / 32; ++c) {
-                        // column 32c: issuer slice hh, CTA half `half` of it, row j0
-                        // of that CTA's weight tile -> channel m0 + half 128 + hh BNI/2 + j0
-                        const int hh = (c * 32) / BNI, within = (c * 32) % BNI;
-                        const int m = m0 + (within / (BNI / 2)) * BNC + hh * (BNI / 2) +
-                                      within % (BNI / 2);
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(taddr + c * 32, v);
-                        tmem_ld_wait();
-                        if (valid && m < p.n_valid) {
-                            float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
+                        for (int c = 0; c < BN / 32; ++c) {
+                            const int m = m0 + c * 32;  // column c: the even CTA's rows, then the odd's
+                            if (m >= p.n_valid) break;  // n_valid is a multiple of 64
+                            uint32_t v[32];
+                            tmem_ld_32x32b_x32(taddr + c * 32, v);
+                            tmem_ld_wait();
+                            if (valid) {
+                                float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + q);
-                                float4 o;
-                                o.x = gate * (s4.x * __uint_as_float(v[4 * q]));
-                                o.y = gate * (s4.y * __uint_as_float(v[4 * q + 1]));
-                                o.z = gate * (s4.z * __uint_as_float(v[4 * q + 2]));
-                                o.w = gate * (s4.w * __uint_as_float(v[4 * q + 3]));
-                                dst[q] = o;
+                                for (int qq = 0; qq < 8; ++qq) {
+                                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + qq);
+                                    float4 o;
+                                    o.x = gate * (s4.x * __uint_as_float(v[4 * qq]));
+                                    o.y = gate * (s4.y * __uint_as_float(v[4 * qq + 1]));
+                                    o.z = gate * (s4.z * __uint_as_float(v[4 * qq + 2]));
+                                    o.w = gate * (s4.w * __uint_as_float(v[4 * qq + 3]));
+                                    dst[qq] = o;
+                                }
                             }
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader + h * (uint32_t)sizeof(uint64_t));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_leader + buf * (uint32_t)sizeof(uint64_t));
         }
     }
 
@@ -543,12 +556,12 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmPa
     return cudaGetLastError();
 }
 
-// Pair tiles of one GEMM: per expert, ceil(128-row halves / 2) m-tiles times
+// Pair tiles of one GEMM: per expert, ceil(128-row quarters / 4) m-tiles times
 // n_tiles (the kernel derives the same count from the padded offsets; the
 // host only needs an upper bound to size the grid).
 int64_t tile_bound(const PrefillArgs& a, int n_tiles) {
-    const int64_t halves = a.rows_padded / BH;
-    return (halves / 2 + a.E) * n_tiles;
+    const int64_t quarters = a.rows_padded / BH;
+    return (quarters / 4 + a.E) * n_tiles;
 }
 
 }  // namespace

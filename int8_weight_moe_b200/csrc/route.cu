@@ -14,9 +14,9 @@
 // is added in fp64 and the result rounded once to fp32.  The products are
 // exact in fp64 (8-bit x 24-bit significands).
 //
-// Work split: for many tokens a CTA of 4 warps handles kTok tokens; warp w
-// owns experts w, w+4, w+8, w+12, so each lane keeps 4 x kTok independent
-// fp64 accumulators and every router weight it loads serves kTok tokens.
+// Work split: for many tokens a CTA of 8 warps handles 16 tokens with the
+// router rows and token rows staged in shared memory (k_route_tiles: each
+// lane keeps 8 tokens x 4 experts of fp64 partial sums).
 // For few tokens (decode) one warp per expert: a cluster of 4 CTAs per token
 // (each warp's router row copied to shared memory in one round trip, logits
 // gathered in the first CTA through distributed shared memory), or for rows
@@ -30,11 +30,9 @@
 namespace jmoe {
 namespace {
 
-constexpr int kWarps = 4;
 constexpr int kMaxE = 64;      // experts
 constexpr int kMaxTopK = 4;
 constexpr int kGroupE = 16;    // experts computed together (one warp each, or 4 per warp)
-constexpr int kPerWarp = kGroupE / kWarps;
 
 // Top-k on one token's fp32 logits: k passes of a strict '>' argmax over the
 // experts not yet chosen (the lower index wins ties), fp32 softmax over all E
@@ -263,69 +261,115 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Many tokens: a CTA of 4 warps handles kTok tokens; for each group of 16
-// experts, warp w owns experts w, w+4, w+8, w+12 of the group, so each lane
-// keeps 4 x kTok independent fp64 accumulators and every router weight it
-// loads serves kTok tokens.
-template <int kTok, bool kMultiGroup>
-__global__ void __launch_bounds__(kWarps * 32)
-    k_route(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
-            const float* __restrict__ bias, int E, int top_k, int renorm, int32_t* __restrict__ ids,
-            float* __restrict__ gates, float* __restrict__ logits) {
-    __shared__ float s_logit[kTok][kMaxE];
+// Many tokens: a CTA of 8 warps computes the logits of 16 tokens, one group
+// of 16 experts at a time.  The group's router rows and the tokens' rows go
+// through shared memory in k-chunks of 512 (16-byte cp.async copies, the next
+// chunk landing while this one is summed); warp w keeps the fp64 partial sums
+// of tokens 8 (w / 4) .. +7 for experts w % 4, w % 4 + 4, w % 4 + 8, w % 4 + 12
+// of the group.  Lane j accumulates k = j (mod 32) in ascending k across the
+// chunks (the canonical order), so every router weight a lane reads serves 8
+// tokens and every token value 4 experts, and a CTA reads each router row
+// once per 16 tokens.
+constexpr int kTileTok = 16, kTileWarps = 8, kTileChunk = 512;
+constexpr int kTileTokPerWarp = 8, kTileExpPerWarp = 4;
+constexpr int kTileWBytes = kGroupE * kTileChunk * 4;     // 32 KB of router rows
+constexpr int kTileXBytes = kTileTok * kTileChunk * 2;    // 16 KB of token rows
+constexpr size_t kTileSmem = 2 * (size_t)(kTileWBytes + kTileXBytes);
+static_assert(kTileWarps * kTileTokPerWarp * kTileExpPerWarp == kTileTok * kGroupE,
+              "the warps cover the 16 tokens x 16 experts of a group");
+
+__global__ void __launch_bounds__(kTileWarps * 32, 2)
+    k_route_tiles(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
+                  const float* __restrict__ bias, int E, int top_k, int renorm,
+                  int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits) {
+    extern __shared__ __align__(16) uint8_t tile_smem[];
+    __shared__ float s_logit[kTileTok][kMaxE];
+    float* const sw0 = reinterpret_cast<float*>(tile_smem);
+    uint16_t* const sx0 = reinterpret_cast<uint16_t*>(tile_smem + kTileWBytes);
+    const size_t buf_bytes = kTileWBytes + kTileXBytes;
+    auto sw = [&](int b) { return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sw0) + b * buf_bytes); };
+    auto sx = [&](int b) {
+        return reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(sx0) + b * buf_bytes);
+    };
+    pdl_wait();  // the previous step may still read ids and gates
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int64_t t0 = (int64_t)blockIdx.x * kTok; t0 < T; t0 += (int64_t)gridDim.x * kTok) {
-        const uint16_t* xr[kTok];
+    const int tg = warp / kTileExpPerWarp, eg = warp % kTileExpPerWarp;
+    const int nchunks = (int)((d + kTileChunk - 1) / kTileChunk);
+    for (int64_t t0 = (int64_t)blockIdx.x * kTileTok; t0 < T; t0 += (int64_t)gridDim.x * kTileTok) {
+        for (int e0 = 0; e0 < E; e0 += kGroupE) {
+            // copies of chunk c into buffer b: the group's router rows and the
+            // tokens' rows (tokens past T repeat the last one; never written)
+            auto stage = [&](int c, int b) {
+                const int64_t base = (int64_t)c * kTileChunk;
+                const int n = (int)(d - base < kTileChunk ? d - base : (int64_t)kTileChunk);
+                const int wu = n / 4, xu = n / 8;  // 16-byte units per row
+                float* w_dst = sw(b);
+                uint16_t* x_dst = sx(b);
+                for (int i = threadIdx.x; i < kGroupE * wu; i += blockDim.x) {
+                    const int r = i / wu, u = i - r * wu;
+                    if (e0 + r < E)
+                        cp_async_16(w_dst + r * kTileChunk + 4 * u, wr + (int64_t)(e0 + r) * d + base + 4 * u, 16);
+                }
+                for (int i = threadIdx.x; i < kTileTok * xu; i += blockDim.x) {
+                    const int r = i / xu, u = i - r * xu;
+                    const int64_t tok = t0 + r < T ? t0 + r : T - 1;
+                    cp_async_16(x_dst + r * kTileChunk + 8 * u, x + tok * d + base + 8 * u, 16);
+                }
+                cp_async_commit();
+            };
+            double acc[kTileTokPerWarp][kTileExpPerWarp];
 #pragma unroll
-        for (int t = 0; t < kTok; ++t) xr[t] = x + min(t0 + t, T - 1) * d;  // clamp: tail tokens
-        // one group of 16 experts unless kMultiGroup (a compile-time bound
-        // keeps the single-group loop as tight as a straight body)
-        const int groups_end = kMultiGroup ? E : 1;
-        for (int eg = 0; eg < groups_end; eg += kGroupE) {
-            double acc[kTok][kPerWarp];
+            for (int t = 0; t < kTileTokPerWarp; ++t)
 #pragma unroll
-            for (int t = 0; t < kTok; ++t)
+                for (int i = 0; i < kTileExpPerWarp; ++i) acc[t][i] = 0.0;
+            stage(0, 0);
+            for (int c = 0; c < nchunks; ++c) {
+                if (c + 1 < nchunks) {
+                    stage(c + 1, (c + 1) & 1);
+                    cp_async_wait<1>();
+                } else {
+                    cp_async_wait<0>();
+                }
+                __syncthreads();
+                const float* W = sw(c & 1);
+                const uint16_t* X = sx(c & 1) + tg * kTileTokPerWarp * kTileChunk;
+                const int n = (int)(d - (int64_t)c * kTileChunk < kTileChunk ? d - (int64_t)c * kTileChunk
+                                                                            : (int64_t)kTileChunk);
+#pragma unroll 2
+                for (int k = lane; k < n; k += 32) {
+                    double xv[kTileTokPerWarp];
 #pragma unroll
-                for (int i = 0; i < kPerWarp; ++i) acc[t][i] = 0.0;
-#pragma unroll 4
-            for (int64_t k = lane; k < d; k += 32) {
-                double xk[kTok];
+                    for (int t = 0; t < kTileTokPerWarp; ++t)
+                        xv[t] = (double)bf16_bits_to_f32(X[t * kTileChunk + k]);
 #pragma unroll
-                for (int t = 0; t < kTok; ++t) xk[t] = (double)bf16_bits_to_f32(__ldg(xr[t] + k));
+                    for (int i = 0; i < kTileExpPerWarp; ++i) {
+                        const int e = eg + kTileExpPerWarp * i;
+                        if (e0 + e < E) {
+                            const double w = (double)W[e * kTileChunk + k];
 #pragma unroll
-                for (int i = 0; i < kPerWarp; ++i) {
-                    const int e = eg + warp + kWarps * i;
-                    if (e < E) {
-                        const double w = (double)__ldg(wr + (int64_t)e * d + k);
-#pragma unroll
-                        for (int t = 0; t < kTok; ++t) acc[t][i] = fma(xk[t], w, acc[t][i]);
+                            for (int t = 0; t < kTileTokPerWarp; ++t) acc[t][i] = fma(xv[t], w, acc[t][i]);
+                        }
                     }
                 }
+                __syncthreads();  // buffer c & 1 is refilled for chunk c + 2
             }
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1)
+            for (int t = 0; t < kTileTokPerWarp; ++t)
 #pragma unroll
-                for (int t = 0; t < kTok; ++t)
+                for (int i = 0; i < kTileExpPerWarp; ++i) {
+                    double v = acc[t][i];
 #pragma unroll
-                    for (int i = 0; i < kPerWarp; ++i)
-                        acc[t][i] += __shfl_down_sync(0xffffffffu, acc[t][i], o);
-            if (lane == 0) {
-#pragma unroll
-                for (int i = 0; i < kPerWarp; ++i) {
-                    const int e = eg + warp + kWarps * i;
-                    if (e < E) {
-                        const double b = bias ? (double)bias[e] : 0.0;
-#pragma unroll
-                        for (int t = 0; t < kTok; ++t)
-                            s_logit[t][e] = __double2float_rn(acc[t][i] + b);
-                    }
+                    for (int o = 16; o >= 1; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+                    const int e = e0 + eg + kTileExpPerWarp * i;
+                    if (lane == 0 && e < E)
+                        s_logit[tg * kTileTokPerWarp + t][e] =
+                            __double2float_rn(v + (bias ? (double)bias[e] : 0.0));
                 }
-            }
         }
         __syncthreads();
-        if (threadIdx.x < kTok && t0 + threadIdx.x < T)
-            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, renorm, ids, gates,
-                        logits);
+        if (threadIdx.x < kTileTok && t0 + threadIdx.x < T)
+            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, renorm, ids, gates, logits);
         __syncthreads();
     }
 }
@@ -360,8 +404,8 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
     const bool norm = gamma_bf16 != nullptr;
     // Few tokens: a cluster of 4 CTAs per token, the RMSNorm (if any) fused in
     // front of the logits (or, for very wide rows, a 16-warp CTA streaming the
-    // router rows in chunks); many tokens: 4 tokens per 4-warp CTA, which cuts
-    // the router-weight traffic fourfold.  Outside the fused kernel the
+    // router rows in chunks); many tokens: 16 tokens per 8-warp CTA with the
+    // rows staged in shared memory (k_route_tiles).  Outside the fused kernel the
     // RMSNorm runs first, into y, and the router reads y.
     const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
     const size_t smem = (size_t)kGroupE * kChunkSmem + (size_t)d * sizeof(uint16_t);
@@ -389,16 +433,15 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
             (const uint16_t*)xr, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         note_launch();
     } else {
-        int64_t blocks = (T + 3) / 4;
-        const int64_t cap = (int64_t)num_sms * 16;
+        int64_t blocks = (T + kTileTok - 1) / kTileTok;
+        const int64_t cap = (int64_t)num_sms * 2;  // one wave: two CTAs per SM
         if (blocks > cap) blocks = cap;
-        if (E <= kGroupE)
-            k_route<4, false><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-                (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
-        else
-            k_route<4, true><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-                (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
-        note_launch();
+        const cudaError_t e = cudaFuncSetAttribute(
+            k_route_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTileSmem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(k_route_tiles, dim3((unsigned)blocks), dim3(kTileWarps * 32), kTileSmem,
+                          stream, (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids,
+                          gates, logits);
     }
     return cudaGetLastError();
 }

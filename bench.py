@@ -411,17 +411,20 @@ def roofline_entry(layer: Layer, stages: dict, peaks: dict):
             "ms": round(ms, 4), "peak_source": peaks["source"] + " hbm copy"}
 
 
-def graph_run(layer: Layer, steps: int, warmup: int = 3):
-    """The whole layer with its RMSNorm prologue -- RMSNorm + router + experts
-    -- captured once in a CUDA graph (int8_weight_moe_b200.MoeLayerGraph) and
+def graph_run(layer: Layer, steps: int, warmup: int = 3, prologue: bool = True):
+    """The whole layer -- with its RMSNorm prologue (RMSNorm + router +
+    experts) or without it (router + experts, the timed eager step's work) --
+    captured once in a CUDA graph (int8_weight_moe_b200.MoeLayerGraph) and
     replayed; ms per replay from CUDA events on the replay stream."""
     import torch
 
     import int8_weight_moe_b200 as jm
 
     wl = layer.wl
-    gamma = (synth.normal_bf16_gpu(wl.seed + 7, synth.X, 0.25, (wl.d_model,),
-                                   device=layer.device).float() + 1.0).to(torch.bfloat16)
+    gamma = None
+    if prologue:
+        gamma = (synth.normal_bf16_gpu(wl.seed + 7, synth.X, 0.25, (wl.d_model,),
+                                       device=layer.device).float() + 1.0).to(torch.bfloat16)
     g = jm.MoeLayerGraph(layer.desc, layer.w_router, wl.T, gamma=gamma, eps=1e-6,
                          bias=layer.bias)
     g.x.copy_(layer.x)
@@ -436,7 +439,8 @@ def graph_run(layer: Layer, steps: int, warmup: int = 3):
     stop.record()
     torch.cuda.synchronize()
     ms = start.elapsed_time(stop) / steps
-    return {"workload": wl.name + " + RMSNorm prologue, CUDA graph", "ms_per_step": round(ms, 4),
+    what = " + RMSNorm prologue" if prologue else " (router + experts, as the eager step)"
+    return {"workload": wl.name + what + ", CUDA graph", "ms_per_step": round(ms, 4),
             "tokens_per_s": round(wl.T / (ms * 1e-3), 1)}
 
 
@@ -683,7 +687,12 @@ def main():
     e2e_ms = max_over_ranks(e2e["ms_per_step"], dev)
     e2e["ms_per_step"] = round(e2e_ms, 4)
     e2e["value"] = round(whole_job_tokens_per_s(world, wl.T, e2e_ms), 1)
-    graph_line = graph_run(layer, max(args.steps // 2, 10)) if not wl.dense else None
+    graph_line = None
+    if not wl.dense:
+        graph_line = graph_run(layer, max(args.steps // 2, 10))
+        # like for like with the timed eager step: the same kernels, replayed
+        graph_line["without_prologue"] = graph_run(layer, max(args.steps // 2, 10),
+                                                   prologue=False)
     work = kernel_work(layer)
     step_gbs = work["step_bytes"] / (ms * 1e-3) / 1e9
     del layer

@@ -200,7 +200,7 @@ def dequant_conversions(counts, d: int, f: int, prefill: bool) -> int:
     """INT8 -> 16-bit weight conversions one step of the expert kernels makes
     (the dequantisation work, reported apart from the FLOPs).  The decode
     kernels convert an expert's 3*d*f weights once per pass over up to 8 of
-    its tokens; the tensor-core kernels once per 256-row tile of its rows,
+    its tokens; the tensor-core kernels once per 512-row tile of its rows,
     which are padded to a multiple of 128."""
     total = 0
     for c in counts:
@@ -209,7 +209,7 @@ def dequant_conversions(counts, d: int, f: int, prefill: bool) -> int:
             continue
         if prefill:
             padded = -(-c // 128) * 128
-            passes = -(-padded // 256)
+            passes = -(-padded // 512)
         else:
             passes = -(-c // 8)
         total += passes * 3 * d * f

@@ -24,9 +24,9 @@ def test_dequant_conversions_decode_passes():
 def test_dequant_conversions_tensor_core_tiles():
     d, f = 64, 128
     unit = 3 * d * f
-    # rows padded to 128, tiles of 256: 1 -> 128 -> 1, 128 -> 1, 129 -> 256 -> 1,
-    # 300 -> 384 -> 2, 513 -> 640 -> 3
-    assert bench.dequant_conversions([1, 128, 129, 300, 513], d, f, prefill=True) == 8 * unit
+    # rows padded to 128, tiles of 512: 1 -> 128 -> 1, 128 -> 1, 129 -> 256 -> 1,
+    # 513 -> 640 -> 2, 1100 -> 1152 -> 3
+    assert bench.dequant_conversions([1, 128, 129, 513, 1100], d, f, prefill=True) == 8 * unit
 
 
 def _fake_layer(wl, ids, prefill):
@@ -64,7 +64,7 @@ def test_kernel_work_dense_layer():
     wl = MINI_DENSE  # one expert, every token
     w = bench.kernel_work(_fake_layer(wl, None, prefill=True))
     assert w["touched"] == 1
-    tiles = -(-(-(-wl.T // 128) * 128) // 256)
+    tiles = -(-(-(-wl.T // 128) * 128) // 512)
     assert w["dequant"]["int8_conversions_per_step"] == tiles * 3 * wl.d_model * wl.d_ff
     assert np.isclose(w["dequant"]["per_touched_weight"], tiles)
 

@@ -106,7 +106,9 @@ constexpr int kSlots = 3;  // ring slots per warp: two 4 KB slots in flight
 // Every item reads two 16-row weight matrices that share the activation
 // fragments: gate/up, the 16 gate rows and the same 16 up rows of a unit of 16
 // channels; down, the two 16-row halves of a unit of 32 output channels.  A
-// ring slot holds 2 k-blocks of 64 bytes of both: 4 KB.
+// ring slot holds 2 k-blocks (one 128-byte line per row) of both: 4 KB, filled
+// by a single TMA box (gate/up: a 4-D view that puts the up rows f rows below
+// the gate rows; down: 32 adjacent rows).
 template <int MODE>
 constexpr int nb_of() {
     return 2;
@@ -118,8 +120,11 @@ constexpr int unit_rows() {
     return MODE == kGateUp ? 16 : 32;
 }
 
-// Shared memory of one warp: kSlots x [matrix][k-block][16 rows][64 B]; the
-// dense 64-byte row pitch makes the fragment reads of a warp conflict-free.
+// Shared memory of one warp: kSlots x [matrix][16 rows][128 B], stored with
+// the TMA 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r & 7)), so
+// that the fragment reads of a warp -- 8 rows x the same 4 chunks -- hit all
+// banks once.  The swizzle needs 1024-byte aligned slots; the extra 1 KB of
+// the allocation pays for aligning the ring.
 template <int MODE>
 constexpr int slot_bytes() {
     return 2 * nb_of<MODE>() * 16 * 64;
@@ -127,7 +132,7 @@ constexpr int slot_bytes() {
 
 template <int MODE>
 constexpr int gemv_smem() {
-    return kWarpsPerBlock * kSlots * slot_bytes<MODE>();
+    return kWarpsPerBlock * kSlots * slot_bytes<MODE>() + 1024;
 }
 
 template <int MODE, int NCH>
@@ -136,30 +141,38 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     constexpr int NMAT = 2;
     constexpr int kNB = nb_of<MODE>();
     constexpr int kSlotBytes = slot_bytes<MODE>();
-    extern __shared__ __align__(128) uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full[kWarpsPerBlock][kSlots];
     __shared__ int s_start[kMaxE + 1];  // first item of expert e
     __shared__ int s_off[kMaxE + 1];
     __shared__ int s_np[kMaxE];         // passes of expert e
     __shared__ int s_abort;
-    pdl_wait();
-    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g8 = lane >> 2, c = lane & 3;
-    uint8_t* ring = smem_raw + warp * kSlots * kSlotBytes;
+    uint8_t* const ring_base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* ring = ring_base + warp * kSlots * kSlotBytes;
     const int E = p.E, S = p.S;
     const int64_t K = MODE == kGateUp ? p.d : p.f;
     const int64_t rows_out = MODE == kGateUp ? p.f : p.d;
     const int groups = (int)(rows_out / unit_rows<MODE>());
-    // row offset of the second matrix: the up rows (f below the gate rows) or
-    // the second 16-row half of the down unit
-    const int moff = MODE == kGateUp ? (int)p.f : 16;
-    if (threadIdx.x <= E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
-    if (lane == 0)
+    if (lane == 0) {
         for (int i = 0; i < kSlots; ++i) sm100::mbar_init(&full[warp][i], 1);
+        sm100::tma_prefetch_desc(&tmW);
+    }
     if (threadIdx.x == 0) {
         s_abort = 0;
         sm100::fence_mbar_init();
     }
+    // The gate/up GEMV reads the grouping tables of the kernel it follows, so
+    // it waits first.  The down GEMV follows k_h16, which lets it start only
+    // after its own wait, i.e. once k_swiglu and everything before it (the
+    // grouping tables included) are complete: it plans its items and starts
+    // its first weight copies, and waits only before it reads hidden rows.
+    if (MODE == kGateUp) {
+        pdl_wait();
+        pdl_launch_dependents();
+    }
+    if (threadIdx.x <= E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
     __syncthreads();
     if (threadIdx.x == 0) {
         int run = 0;
@@ -207,13 +220,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 
     // ---- producer cursor (lane 0 issues the TMA boxes of slot-sized pieces)
     int pe = 0, pi = 0, pj = 0;
-    int prow = 0, pk = 0;  // first weight row of the item, first k byte of the piece
+    int pexp = 0, prow = 0, pk = 0;  // expert, first weight row of the item, first k byte of the piece
     int64_t issued = 0;    // slot fills issued so far (fill h uses slot h % kSlots)
     int64_t skipped = -1;  // the fill the test hook left out (its barrier never completes)
     auto set_prefetch_item = [&](int it) {
         const Item u = item_at(it, pe);
-        prow = MODE == kGateUp ? u.e * (int)(2 * p.f) + u.group * 16
-                               : u.e * (int)p.d + u.group * unit_rows<MODE>();
+        pexp = u.e;
+        prow = MODE == kGateUp ? u.group * 16 : u.e * (int)p.d + u.group * unit_rows<MODE>();
         pk = u.z * kb_item * 64;
     };
     auto issue = [&](int slot) {
@@ -222,12 +235,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         if (lane == 0 && !skip) {
             uint8_t* dst = ring + slot * kSlotBytes;
             sm100::mbar_arrive_expect_tx(&full[warp][slot], kSlotBytes);
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                for (int b = 0; b < kNB; ++b)
-                    sm100::tma_load_2d(dst + (m * kNB + b) * 1024, &tmW, &full[warp][slot],
-                                       pk + (pj * kNB + b) * 64, prow + m * moff);
+            if (MODE == kGateUp)  // [expert][gate|up][row][k]: 16 rows of both halves
+                sm100::tma_load_4d(dst, &tmW, &full[warp][slot], pk + pj * kNB * 64, prow, 0, pexp);
+            else                  // [row][k]: the unit's 32 rows
+                sm100::tma_load_2d(dst, &tmW, &full[warp][slot], pk + pj * kNB * 64, prow);
         }
         ++issued;
         if (++pj == nsl) {
@@ -236,10 +247,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         }
     };
     set_prefetch_item(0);
-    if (lane == 0) sm100::tma_prefetch_desc(&tmW);
 #pragma unroll
     for (int q = 0; q < kSlots - 1; ++q)
         if (q < total) issue(q);
+    if (MODE == kDown) {
+        pdl_wait();
+        pdl_launch_dependents();
+    }
 
     // ---- consumer state: activation fragments are loaded one slot ahead,
     // into the one of two register buffers the current slot does not use
@@ -320,15 +334,18 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             ok = false;
             return;
         }
-        const uint8_t* src = ring + cslot * kSlotBytes + g8 * 64 + 16 * c;
+        // rows g8 and g8 + 8 of matrix m: byte m * 2048 + row * 128 + the
+        // swizzled position of chunk 4b + c (row & 7 == g8 for both rows)
+        const uint8_t* src = ring + cslot * kSlotBytes + g8 * 128;
 #pragma unroll
         for (int b = 0; b < kNB; ++b) {
             if (cj * kNB + b < kb_item) {
                 uint4 wq[2 * NMAT];
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m) {
-                    wq[2 * m] = *reinterpret_cast<const uint4*>(src + (m * kNB + b) * 1024);
-                    wq[2 * m + 1] = *reinterpret_cast<const uint4*>(src + (m * kNB + b) * 1024 + 8 * 64);
+                    const int off = m * 2048 + (((4 * b + c) ^ g8) << 4);
+                    wq[2 * m] = *reinterpret_cast<const uint4*>(src + off);
+                    wq[2 * m + 1] = *reinterpret_cast<const uint4*>(src + off + 8 * 128);
                 }
 #pragma unroll
                 for (int n = 0; n < NCH; ++n) {
@@ -465,11 +482,13 @@ __global__ void __launch_bounds__(256)
     __shared__ int s_e;
     __shared__ float s_sx;
     __shared__ int red[8];
-    pdl_wait();
-    pdl_launch_dependents();
-    const int used = offsets[E];  // dropped assignments leave trailing slots unused
     const int64_t n = (int64_t)blockIdx.x * kSwigluChunk + threadIdx.x * 4;
-    for (int slot = blockIdx.y; slot < used; slot += gridDim.y) {
+    // The slot's expert, its token's shift and the channel scales depend only
+    // on the grouping kernel's tables, complete before the gate/up GEMV (the
+    // kernel this one follows) started: the first slot's lookups run before
+    // the wait, which only the partial sums P need.
+    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+    auto lookup = [&](int slot) {
         if (threadIdx.x == 0) {
             int e = 0;
             while (e + 1 < E && offsets[e + 1] <= slot) ++e;
@@ -477,6 +496,18 @@ __global__ void __launch_bounds__(256)
             s_sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
         }
         __syncthreads();
+        if (n < f) {
+            const float* sg = sgu + (int64_t)s_e * 2 * f;
+            s0 = __ldg(reinterpret_cast<const float4*>(sg + n));
+            s1 = __ldg(reinterpret_cast<const float4*>(sg + f + n));
+        }
+    };
+    const int used = offsets[E];  // dropped assignments leave trailing slots unused
+    int slot = blockIdx.y;
+    if (slot < used) lookup(slot);
+    pdl_wait();
+    pdl_launch_dependents();
+    for (; slot < used; slot += gridDim.y) {
         int ex = 0;
         if (n < f) {
             const float sx = s_sx;
@@ -489,9 +520,6 @@ __global__ void __launch_bounds__(256)
                 vg[0] += g.x; vg[1] += g.y; vg[2] += g.z; vg[3] += g.w;
                 vu[0] += u.x; vu[1] += u.y; vu[2] += u.z; vu[3] += u.w;
             }
-            const float* sg = sgu + (int64_t)s_e * 2 * f;
-            const float4 s0 = __ldg(reinterpret_cast<const float4*>(sg + n));
-            const float4 s1 = __ldg(reinterpret_cast<const float4*>(sg + f + n));
             const float sgv[4] = {s0.x, s0.y, s0.z, s0.w}, suv[4] = {s1.x, s1.y, s1.z, s1.w};
             uint16_t hb[4];
 #pragma unroll
@@ -505,6 +533,7 @@ __global__ void __launch_bounds__(256)
         }
         const int m = block_max_int(ex, red);  // ends with a barrier: s_e, s_sx reusable
         if (threadIdx.x == 0 && m > 0) atomicMax(&hmax[slot], m);
+        if (slot + (int)gridDim.y < used) lookup(slot + (int)gridDim.y);
     }
 }
 
@@ -515,6 +544,8 @@ __global__ void __launch_bounds__(256)
     k_h16(const uint16_t* __restrict__ Hb, int64_t f, const int32_t* __restrict__ offsets, int E,
           const int32_t* __restrict__ hmax, uint16_t* __restrict__ H16) {
     pdl_wait();
+    // only after the wait: the down GEMV relies on it (it reads the grouping
+    // tables before its own wait)
     pdl_launch_dependents();
     const int64_t total = (int64_t)offsets[E] * f / 2;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -542,10 +573,13 @@ __global__ void __launch_bounds__(256)
               const float* __restrict__ sd, uint16_t* __restrict__ out) {
     __shared__ int s_slot[kMaxTopK], s_e[kMaxTopK];
     __shared__ float s_gw[kMaxTopK], s_hs[kMaxTopK];
-    pdl_wait();
-    pdl_launch_dependents();
     const int64_t m = (int64_t)blockIdx.x * kCombineChunk + threadIdx.x * 4;
-    for (int64_t t = blockIdx.y; t < T; t += gridDim.y) {
+    // The token's slots, experts, gates, hidden-row shifts and the scales are
+    // all final before the down GEMV (the kernel this one follows) starts: the
+    // first token's lookups run before the wait, which only the partial sums P
+    // need.
+    float4 sv[kMaxTopK];
+    auto lookup = [&](int64_t t) {
         if (threadIdx.x < top_k) {
             const int64_t a = t * top_k + threadIdx.x;
             const int e = ids[a];
@@ -557,10 +591,21 @@ __global__ void __launch_bounds__(256)
             s_hs[threadIdx.x] = ok ? ldexpf(1.0f, row_shift(hmax[slot])) : 0.0f;
         }
         __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            if (j < top_k && m < d && s_slot[j] >= 0)
+                sv[j] = __ldg(reinterpret_cast<const float4*>(sd + (int64_t)s_e[j] * d + m));
+    };
+    int64_t t = blockIdx.y;
+    if (t < T) lookup(t);
+    pdl_wait();
+    pdl_launch_dependents();
+    for (; t < T; t += gridDim.y) {
         if (m < d) {
             float o[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int j = 0; j < top_k; ++j) {
-                const int slot = s_slot[j];
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                const int slot = j < top_k ? s_slot[j] : -1;
                 if (slot < 0) continue;
                 float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
@@ -570,20 +615,21 @@ __global__ void __launch_bounds__(256)
                     y[0] += q.x; y[1] += q.y; y[2] += q.z; y[3] += q.w;
                 }
                 const float hs = s_hs[j];
-                const float4 sv =
-                    __ldg(reinterpret_cast<const float4*>(sd + (int64_t)s_e[j] * d + m));
                 const float gw = s_gw[j];
-                o[0] += gw * (sv.x * (y[0] * hs));
-                o[1] += gw * (sv.y * (y[1] * hs));
-                o[2] += gw * (sv.z * (y[2] * hs));
-                o[3] += gw * (sv.w * (y[3] * hs));
+                o[0] += gw * (sv[j].x * (y[0] * hs));
+                o[1] += gw * (sv[j].y * (y[1] * hs));
+                o[2] += gw * (sv[j].z * (y[2] * hs));
+                o[3] += gw * (sv[j].w * (y[3] * hs));
             }
             uint2 r;
             r.x = pack_bf16x2(o[0], o[1]);
             r.y = pack_bf16x2(o[2], o[3]);
             *reinterpret_cast<uint2*>(out + t * d + m) = r;
         }
-        __syncthreads();  // the next token's lookups overwrite the shared values
+        if (t + (int64_t)gridDim.y < T) {
+            __syncthreads();  // the next token's lookups overwrite the shared values
+            lookup(t + gridDim.y);
+        }
     }
 }
 
@@ -636,13 +682,22 @@ int gemv_grid(int num_sms) {
 
 template <int MODE, int NCH>
 cudaError_t launch_gemv(const GemvParams& p, int num_sms, cudaStream_t stream) {
-    // weights [rows][K] int8, boxes of 64 bytes x 16 rows
-    const int64_t K = MODE == kGateUp ? p.d : p.f;
-    const int64_t rows = MODE == kGateUp ? (int64_t)p.E * 2 * p.f : (int64_t)p.E * p.d;
+    // int8 weights, one 4 KB box per ring slot, 128-byte swizzle.  gate/up
+    // [E][2f][d] seen as 4-D [E][2][f][d]: box 128 bytes x 16 rows x both
+    // halves; down [E*d][f]: box 128 bytes x 32 rows.
     CUtensorMap map;
-    if (!encode_2d(&map, p.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, K, 16, 64,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    bool ok;
+    if (MODE == kGateUp) {
+        const uint64_t K = (uint64_t)p.d, f = (uint64_t)p.f;
+        const uint64_t dims[4] = {K, f, 2, (uint64_t)p.E};
+        const uint64_t strides[3] = {K, f * K, 2 * f * K};
+        const uint32_t box[4] = {128, 16, 2, 1};
+        ok = encode_4d_u8(&map, p.w, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        ok = encode_2d(&map, p.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.E * p.d,
+                       (uint64_t)p.f, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (!ok) return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(k_gemv<MODE, NCH>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            gemv_smem<MODE>());

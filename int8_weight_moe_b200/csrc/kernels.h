@@ -7,17 +7,25 @@
 
 namespace jmoe {
 
-// TMA tensor map of a row-major 2-D tensor [rows][cols] with boxes of
-// box_rows x box_cols elements (false if the driver entry point is missing or
-// the encoder rejects the arguments).
-bool tensormap_available();
-
 // Counts one kernel launch (process-wide, all devices); every launch site in
 // the library calls it right after the launch.
 void note_launch();
+
+// Whether the driver's tensor-map encoder could be looked up.
+bool tensormap_available();
+
+// TMA tensor map of a row-major 2-D tensor [rows][cols] with boxes of
+// box_rows x box_cols elements (false if the driver entry point is missing or
+// the encoder rejects the arguments).
 bool encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType type, int elem_bytes,
                uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
                CUtensorMapSwizzle swizzle);
+
+// TMA tensor map of a 4-D byte tensor: dims innermost first, byte strides of
+// dims 1..3, box extents innermost first (false as for encode_2d).
+bool encode_4d_u8(CUtensorMap* map, const void* base, const uint64_t (&dims)[4],
+                  const uint64_t (&strides)[3], const uint32_t (&box)[4],
+                  CUtensorMapSwizzle swizzle);
 
 // Bits of the sticky device error word (see jmoe_last_error).
 enum : unsigned {

@@ -21,7 +21,7 @@
 // (each warp's router row copied to shared memory in one round trip, logits
 // gathered in the first CTA through distributed shared memory), or for rows
 // too wide for that a 16-warp CTA per token streaming the rows in chunks.
-// Softmax (fp32) and top-k run in one thread per token afterwards.
+// Softmax (fp32) and top-k run in one warp per token afterwards.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -34,37 +34,83 @@ constexpr int kMaxE = 64;      // experts
 constexpr int kMaxTopK = 4;
 constexpr int kGroupE = 16;    // experts computed together (one warp each, or 4 per warp)
 
-// Top-k on one token's fp32 logits: k passes of a strict '>' argmax over the
-// experts not yet chosen (the lower index wins ties), fp32 softmax over all E
-// experts, then the chosen probabilities -- renormalised over the selection
-// (in selection order) when `renorm`, as they are otherwise.
-__device__ void select_topk(const float* l, int64_t t, int E, int top_k, int renorm,
-                            int32_t* ids, float* gates, float* logits) {
-    if (logits)
-        for (int e = 0; e < E; ++e) logits[t * E + e] = l[e];
+// Top-k on one token's fp32 logits (E <= 64), by one whole warp: k passes of
+// a strict '>' argmax over the experts not yet chosen, scanning in index
+// order (the lower index wins ties), fp32 softmax over all E experts, then
+// the chosen probabilities -- renormalised over the selection (in selection
+// order) when `renorm`, as they are otherwise.
+//
+// Lane i holds experts i and i + 32.  A scan in index order that starts at
+// the first candidate f and moves on only to a strictly larger value ends at
+// f when l[f] is NaN (nothing compares larger), and otherwise at the lowest
+// index holding the largest non-NaN value; each pass takes exactly that,
+// the second case by a shuffle reduction over (value, index).  The sum z of
+// the exponentials runs in index order in every lane (shuffles), so the
+// result is the same as one thread's loop.
+__device__ __forceinline__ void warp_select_topk(const float* l, int64_t t, int E, int top_k,
+                                                 int renorm, int32_t* ids, float* gates,
+                                                 float* logits) {
+    const int lane = threadIdx.x & 31;
+    const bool has0 = lane < E, has1 = lane + 32 < E;
+    const float v0 = has0 ? l[lane] : 0.0f, v1 = has1 ? l[lane + 32] : 0.0f;
+    if (logits) {
+        if (has0) logits[t * E + lane] = v0;
+        if (has1) logits[t * E + lane + 32] = v1;
+    }
+    bool free0 = has0, free1 = has1;
     int chosen[kMaxTopK];
-    for (int j = 0; j < top_k; ++j) {
-        int best = -1;
-        for (int e = 0; e < E; ++e) {
-            bool taken = false;
-            for (int i = 0; i < j; ++i) taken |= chosen[i] == e;
-            if (!taken && (best < 0 || l[e] > l[best])) best = e;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= top_k) break;
+        const unsigned b0 = __ballot_sync(0xffffffffu, free0), b1 = __ballot_sync(0xffffffffu, free1);
+        const int f = b0 ? __ffs(b0) - 1 : 32 + __ffs(b1) - 1;  // first candidate
+        const float lf = f < 32 ? __shfl_sync(0xffffffffu, v0, f) : __shfl_sync(0xffffffffu, v1, f - 32);
+        int best;
+        if (isnan(lf)) {
+            best = f;
+        } else {
+            // this lane's best non-NaN candidate (its lower index first), then
+            // the warp's: the larger value, the lower index on equal values
+            float bv = 0.0f;
+            int bi = -1;
+            if (free0 && !isnan(v0)) { bv = v0; bi = lane; }
+            if (free1 && !isnan(v1) && (bi < 0 || v1 > bv)) { bv = v1; bi = lane + 32; }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                const bool take = oi >= 0 && (bi < 0 || ov > bv || (ov == bv && oi < bi));
+                if (take) { bv = ov; bi = oi; }
+            }
+            best = bi;
         }
         chosen[j] = best;
+        if (best == lane) free0 = false;
+        if (best == lane + 32) free1 = false;
     }
-    float p[kMaxE];
-    const float m = l[chosen[0]];
+    const int c0 = chosen[0];
+    const float m = c0 < 32 ? __shfl_sync(0xffffffffu, v0, c0) : __shfl_sync(0xffffffffu, v1, c0 - 32);
+    const float p0 = has0 ? expf(v0 - m) : 0.0f, p1 = has1 ? expf(v1 - m) : 0.0f;
     float z = 0.0f;
-    for (int e = 0; e < E; ++e) {
-        p[e] = expf(l[e] - m);
-        z += p[e];
-    }
-    for (int e = 0; e < E; ++e) p[e] = p[e] / z;
+    for (int e = 0; e < E && e < 32; ++e) z += __shfl_sync(0xffffffffu, p0, e);
+    for (int e = 32; e < E; ++e) z += __shfl_sync(0xffffffffu, p1, e - 32);
+    float q[kMaxTopK];
     float sel = 0.0f;
-    for (int j = 0; j < top_k; ++j) sel += p[chosen[j]];
-    for (int j = 0; j < top_k; ++j) {
-        ids[t * top_k + j] = chosen[j];
-        gates[t * top_k + j] = renorm ? p[chosen[j]] / sel : p[chosen[j]];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= top_k) break;
+        const int c = chosen[j];
+        const float pc = c < 32 ? __shfl_sync(0xffffffffu, p0, c) : __shfl_sync(0xffffffffu, p1, c - 32);
+        q[j] = pc / z;
+        sel += q[j];
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        if (j >= top_k) break;
+        if (lane == j) {
+            ids[t * top_k + j] = chosen[j];
+            gates[t * top_k + j] = renorm ? q[j] / sel : q[j];
+        }
     }
 }
 
@@ -146,7 +192,7 @@ __global__ void __launch_bounds__(kGroupE * 32)
         if (lane == 0) s_logit[e] = __double2float_rn(acc + (bias ? (double)bias[e] : 0.0));
     }
     __syncthreads();
-    if (threadIdx.x == 0) select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
+    if (warp == 0) warp_select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
 }
 
 // Few tokens, d_model up to about 11k: a cluster of 4 CTAs per token, 4
@@ -178,8 +224,6 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
     // first half of a cluster barrier: no CTA writes into another CTA's shared
     // memory before every CTA of the cluster has started (the wait is below)
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-    pdl_wait();  // the previous step may still read ids and gates
-    pdl_launch_dependents();
     const unsigned rank = cluster.block_rank();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = blockIdx.x / kRouteCluster;
@@ -189,8 +233,12 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
         for (int64_t i = lane; i < d / 4; i += 32) cp_async_16(row + 4 * i, w + 4 * i, 16);
         cp_async_commit();
     };
+    // The router rows are weights no kernel of the stream writes: their copy
+    // starts before the wait for the previous kernel.
     const int e0 = (int)rank * kExpertsPerCta + warp;
     if (e0 < E) copy_row(e0);
+    pdl_wait();  // the token rows come from, and ids/gates may still be read by, earlier kernels
+    pdl_launch_dependents();
     const uint16_t* xr = x + t * d;
     for (int64_t k = threadIdx.x * 8; k < d; k += (int64_t)blockDim.x * 8)
         *reinterpret_cast<uint4*>(s_x + k) = __ldg(reinterpret_cast<const uint4*>(xr + k));
@@ -240,7 +288,7 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kExperts
         if (lane == 0) dst[e] = l;
     }
     cluster.sync();
-    if (rank == 0 && threadIdx.x == 0) select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
+    if (rank == 0 && warp == 0) warp_select_topk(s_logit, t, E, top_k, renorm, ids, gates, logits);
 }
 
 // One warp per token.
@@ -368,8 +416,8 @@ __global__ void __launch_bounds__(kTileWarps * 32, 2)
                 }
         }
         __syncthreads();
-        if (threadIdx.x < kTileTok && t0 + threadIdx.x < T)
-            select_topk(s_logit[threadIdx.x], t0 + threadIdx.x, E, top_k, renorm, ids, gates, logits);
+        for (int r = warp; r < kTileTok; r += kTileWarps)
+            if (t0 + r < T) warp_select_topk(s_logit[r], t0 + r, E, top_k, renorm, ids, gates, logits);
         __syncthreads();
     }
 }

@@ -144,8 +144,12 @@ def test_route_top1_and_ties():
 @pytest.mark.parametrize("T,k,E,mode", [(64, 2, 16, "uniform"), (37, 2, 16, "skew"),
                                          (1, 2, 16, "uniform"), (5000, 2, 16, "skew"),
                                          (16384, 2, 16, "uniform"), (300, 1, 1, "uniform"),
-                                         (129, 2, 16, "one")])
+                                         (129, 2, 16, "one"), (200, 4, 64, "uniform"),
+                                         (512, 2, 16, "skew"), (1025, 1, 40, "uniform"),
+                                         (33, 1, 40, "skew"), (7, 3, 64, "one")])
 def test_permute_bitexact(T, k, E, mode):
+    """Up to 1024 assignments one warp sorts, above that the whole block: both
+    sides of that boundary, 33 to 64 experts (two per lane) and ragged chunks."""
     rng = np.random.default_rng(T + k + E)
     ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
     if mode == "skew":
@@ -157,6 +161,31 @@ def test_permute_bitexact(T, k, E, mode):
     assert np.array_equal(off.cpu().numpy(), oo)
     assert np.array_equal(perm.cpu().numpy(), po)
     assert np.array_equal(inv.cpu().numpy(), io)
+
+
+@pytest.mark.parametrize("T,k,E", [(40, 2, 16), (900, 2, 40), (3000, 2, 16)])
+def test_permute_leaves_out_invalid_ids(T, k, E):
+    """Ids outside [0, E) take no slot (inv = -1) and raise the device error
+    word; the valid ones are grouped exactly as a stable sort of them alone
+    (numpy's stable argsort here), on the warp path and the block path."""
+    assert jm.jmoe_last_error() in (jm.JMOE_OK, jm.JMOE_EDEVICE)
+    rng = np.random.default_rng(T * 7 + E)
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    flat = ids.reshape(-1)
+    bad = rng.choice(flat.size, size=max(3, flat.size // 50), replace=False)
+    flat[bad] = rng.choice(np.array([-1, E, 99, -7], dtype=np.int32), size=bad.size)
+    off, perm, inv = jm.jmoe_permute(torch.from_numpy(ids).cuda(), E)
+    torch.cuda.synchronize()
+    assert jm.jmoe_last_error() == jm.JMOE_EDEVICE
+    valid = (flat >= 0) & (flat < E)
+    want_perm = np.flatnonzero(valid)[np.argsort(flat[valid], kind="stable")]
+    want_off = np.concatenate([[0], np.cumsum(np.bincount(flat[valid], minlength=E))])
+    want_inv = np.full(flat.size, -1, dtype=np.int64)
+    want_inv[want_perm] = np.arange(want_perm.size)
+    n = want_perm.size
+    assert np.array_equal(off.cpu().numpy(), want_off)
+    assert np.array_equal(perm.cpu().numpy()[:n], want_perm)
+    assert np.array_equal(inv.cpu().numpy(), want_inv)
 
 
 # ----------------------------------------------------------------------------- forward

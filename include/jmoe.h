@@ -320,6 +320,11 @@ jmoe_status jmoe_last_error(void);
 /* A static, human-readable name for a status. */
 const char* jmoe_status_string(jmoe_status status);
 
+/* The CUDA runtime's description of the error behind the calling thread's
+ * most recent JMOE_ECUDA ("no CUDA error" if there was none).  Static
+ * storage; it stays until a later JMOE_ECUDA on the same thread. */
+const char* jmoe_cuda_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif

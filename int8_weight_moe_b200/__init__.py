@@ -29,7 +29,7 @@ EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_rmsnorm", "jmo
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
             "jmoe_ep_dispatch", "jmoe_ep_combine",
             "jmoe_profile_events", "jmoe_launch_count", "jmoe_test_stall", "jmoe_last_error",
-            "jmoe_status_string")
+            "jmoe_status_string", "jmoe_cuda_error_string")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
 JMOE_ROUTE_SOFTMAX_GATES = 1
 JMOE_STALL_TENSOR_GEMM, JMOE_STALL_DECODE_GEMV = 1, 2
@@ -41,7 +41,10 @@ class JmoeError(RuntimeError):
 
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)}")
+        msg = f"{fn} failed: {status_string(status)}"
+        if status == JMOE_ECUDA:
+            msg += f" ({load().jmoe_cuda_error_string().decode()})"
+        super().__init__(msg)
 
 
 class MoeDesc(ctypes.Structure):
@@ -87,10 +90,12 @@ def load() -> ctypes.CDLL:
     lib.jmoe_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
     lib.jmoe_test_stall.argtypes = [i32, i64]
     lib.jmoe_last_error.argtypes = []
-    for name in EXPORTED[:-1]:
+    for name in EXPORTED[:-2]:
         getattr(lib, name).restype = st
     lib.jmoe_status_string.argtypes = [st]
     lib.jmoe_status_string.restype = ctypes.c_char_p
+    lib.jmoe_cuda_error_string.argtypes = []
+    lib.jmoe_cuda_error_string.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -391,6 +396,11 @@ def jmoe_test_stall(target: int, wait_cycles: int = 0) -> None:
 def jmoe_last_error() -> int:
     """Read and clear the device error word (synchronises the device)."""
     return load().jmoe_last_error()
+
+
+def jmoe_cuda_error_string() -> str:
+    """The CUDA error text behind this thread's most recent JMOE_ECUDA."""
+    return load().jmoe_cuda_error_string().decode()
 
 
 def jmoe_status_string(status: int) -> str:

@@ -132,7 +132,14 @@ void stage_mark(int stage, bool after, cudaStream_t s) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-jmoe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? JMOE_OK : JMOE_ECUDA; }
+// The CUDA error behind the calling thread's most recent JMOE_ECUDA.
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+
+jmoe_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return JMOE_OK;
+    t_last_cuda = e;
+    return JMOE_ECUDA;
+}
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -324,6 +331,10 @@ const char* jmoe_status_string(jmoe_status s) {
         case JMOE_EDEVICE: return "JMOE_EDEVICE: invalid expert id seen on the device";
     }
     return "unknown jmoe_status";
+}
+
+const char* jmoe_cuda_error_string(void) {
+    return t_last_cuda == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_cuda);
 }
 
 jmoe_status jmoe_quantize(const void* w_bf16, int64_t rows, int64_t cols, int8_t* q,

@@ -27,6 +27,16 @@ def test_library_exports_every_header_symbol():
         assert hasattr(lib, name), name
 
 
+def test_cuda_error_string_is_per_thread_and_starts_empty():
+    import threading
+
+    got = []
+    t = threading.Thread(target=lambda: got.append(jm.jmoe_cuda_error_string()))
+    t.start()
+    t.join()
+    assert got == ["no CUDA error"]
+
+
 def test_status_strings():
     for code in range(8):
         assert jm.status_string(code).startswith("JMOE_")

@@ -307,6 +307,21 @@ def test_forward_ragged_token_counts(T, d, f, path):
     assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(T), io, go), f"T={T}")
 
 
+@pytest.mark.parametrize("T,d,f", [(8, 1088, 192), (20, 4096, 128), (8, 8192, 128),
+                                   (8, 8256, 128)], ids=lambda v: str(v))
+def test_decode_gate_up_widths(T, d, f):
+    """The decode path over d_model: 17, 64, 128 and 129 k-blocks of 64 (the
+    K pieces of the split-K GEMV and the 4-D gate/up box walk them), with
+    20 tokens in 8-token passes, the last one ragged."""
+    wl = Workload(f"gu_T{T}_d{d}_f{f}", 16, T, d, f, E=4, bias=None)
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g, out = run_layer(dev, jm.JMOE_PATH_DECODE)
+    assert jm.jmoe_last_error() == jm.JMOE_OK
+    _, io, go = ora.route()
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(T), io, go), wl.name)
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_forced_routing_one_expert_and_zero_input(path):
     wl = Workload("forced", 8, 200, 256, 512)

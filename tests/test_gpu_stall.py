@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from layers import DeviceLayer, OracleLayer, assert_close, bf16_to_f64
-from synth.workloads import TINY
+from synth.workloads import TINY, Workload
 
 torch = pytest.importorskip("torch")
 
@@ -22,13 +22,17 @@ import int8_weight_moe_b200 as jm  # noqa: E402
 SHORT_WAIT = 2_000_000  # SM cycles, about 1 ms
 
 
+WIDE = Workload("wide_stall", 18, 8, 8256, 128, E=4)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("target,path", [(jm.JMOE_STALL_TENSOR_GEMM, jm.JMOE_PATH_PREFILL),
-                                         (jm.JMOE_STALL_DECODE_GEMV, jm.JMOE_PATH_DECODE)],
-                         ids=["tensor_gemm", "decode_gemv"])
-def test_wait_runs_out_then_next_call_is_correct(target, path):
-    dev, ora = DeviceLayer(TINY), OracleLayer(TINY)
-    ids, g = jm.jmoe_route(dev.x, dev.w_router, TINY.top_k, dev.bias)
+@pytest.mark.parametrize("target,path,wl", [(jm.JMOE_STALL_TENSOR_GEMM, jm.JMOE_PATH_PREFILL, TINY),
+                                            (jm.JMOE_STALL_DECODE_GEMV, jm.JMOE_PATH_DECODE, TINY),
+                                            (jm.JMOE_STALL_DECODE_GEMV, jm.JMOE_PATH_DECODE, WIDE)],
+                         ids=["tensor_gemm", "decode_gemv", "decode_gemv_d8256"])
+def test_wait_runs_out_then_next_call_is_correct(target, path, wl):
+    dev, ora = DeviceLayer(wl), OracleLayer(wl)
+    ids, g = jm.jmoe_route(dev.x, dev.w_router, wl.top_k, dev.bias)
     torch.cuda.synchronize()
     assert jm.jmoe_last_error() == jm.JMOE_OK
     jm.jmoe_test_stall(target, SHORT_WAIT)
@@ -44,7 +48,7 @@ def test_wait_runs_out_then_next_call_is_correct(target, path):
     assert jm.jmoe_last_error() == jm.JMOE_OK
     _, io, go = ora.route()
     assert np.array_equal(ids.cpu().numpy(), io)
-    assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(TINY.T), io, go), "after stall")
+    assert_close(bf16_to_f64(out), ora.forward_tokens(np.arange(wl.T), io, go), "after stall")
 
 
 @pytest.mark.gpu

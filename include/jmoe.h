@@ -54,7 +54,9 @@ typedef enum {
     JMOE_EWORKSPACE = 4,   /* workspace smaller than the size query returned */
     JMOE_ECUDA = 5,        /* a CUDA runtime call or launch failed */
     JMOE_ETIMEOUT = 6,     /* (device word) a bounded wait inside a kernel ran out */
-    JMOE_EDEVICE = 7       /* (device word) a kernel saw an invalid expert id */
+    JMOE_EDEVICE = 7,      /* (device word) a kernel saw an invalid expert id */
+    JMOE_EBOUNDS = 8       /* (device word) a device bounds check failed; only the
+                              JMOE_CHECKS=1 build (libjmoe_checks.so) has them */
 } jmoe_status;
 
 /* Which expert-GEMM kernels jmoe_forward / jmoe_mlp_forward use. */
@@ -316,6 +318,14 @@ jmoe_status jmoe_test_stall(int32_t target, int64_t wait_cycles);
  * other calls it synchronises the device.  Returns JMOE_OK when no kernel
  * has flagged anything since the last call. */
 jmoe_status jmoe_last_error(void);
+
+/* Test hook of the bounds-check build (libjmoe_checks.so, compiled with
+ * JMOE_CHECKS=1): launches on `stream` a kernel whose single bounds check
+ * fails without touching memory, so that the next jmoe_last_error returns
+ * JMOE_EBOUNDS.  The normal build has no checks and returns JMOE_EUNSUPPORTED
+ * without launching anything.  The pages define no such operation: it tests
+ * the library's own fault reporting. */
+jmoe_status jmoe_test_check(void* stream);
 
 /* A static, human-readable name for a status. */
 const char* jmoe_status_string(jmoe_status status);

@@ -17,10 +17,14 @@ from typing import Optional, Tuple
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libjmoe.so")
+# The bounds-check build (same ABI, device checks compiled in); tests load it
+# by setting LIB_PATH to this path before the first call.
+CHECKS_LIB_PATH = os.path.join(HERE, "libjmoe_checks.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "jmoe.h")
 
 JMOE_OK, JMOE_EINVAL, JMOE_EALIGN, JMOE_EUNSUPPORTED = 0, 1, 2, 3
 JMOE_EWORKSPACE, JMOE_ECUDA, JMOE_ETIMEOUT, JMOE_EDEVICE = 4, 5, 6, 7
+JMOE_EBOUNDS = 8
 JMOE_PATH_AUTO, JMOE_PATH_DECODE, JMOE_PATH_PREFILL = 0, 1, 2
 
 # Every C entry point the header declares.
@@ -29,7 +33,7 @@ EXPORTED = ("jmoe_quantize", "jmoe_route", "jmoe_route_ex", "jmoe_rmsnorm", "jmo
             "jmoe_forward", "jmoe_forward_noalloc", "jmoe_mlp_workspace_size", "jmoe_mlp_forward",
             "jmoe_ep_dispatch", "jmoe_ep_combine",
             "jmoe_profile_events", "jmoe_launch_count", "jmoe_test_stall", "jmoe_last_error",
-            "jmoe_status_string", "jmoe_cuda_error_string")
+            "jmoe_test_check", "jmoe_status_string", "jmoe_cuda_error_string")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # JMOE_NOALLOC_SCRATCH_BYTES
 JMOE_ROUTE_SOFTMAX_GATES = 1
 JMOE_STALL_TENSOR_GEMM, JMOE_STALL_DECODE_GEMV = 1, 2
@@ -66,7 +70,7 @@ def load() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libjmoe.so is not built ({LIB_PATH}); run "
+        raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
                           "`python -m int8_weight_moe_b200.build` or __graft_entry__.build()")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -89,6 +93,7 @@ def load() -> ctypes.CDLL:
     lib.jmoe_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.jmoe_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
     lib.jmoe_test_stall.argtypes = [i32, i64]
+    lib.jmoe_test_check.argtypes = [vp]
     lib.jmoe_last_error.argtypes = []
     for name in EXPORTED[:-2]:
         getattr(lib, name).restype = st
@@ -396,6 +401,16 @@ def jmoe_test_stall(target: int, wait_cycles: int = 0) -> None:
 def jmoe_last_error() -> int:
     """Read and clear the device error word (synchronises the device)."""
     return load().jmoe_last_error()
+
+
+def jmoe_test_check(stream=None) -> int:
+    """Bounds-check build only: make one device check fail (no memory access),
+    so that the next jmoe_last_error() is JMOE_EBOUNDS.  Returns the status
+    (JMOE_EUNSUPPORTED from the normal build)."""
+    import torch
+
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return load().jmoe_test_check(s)
 
 
 def jmoe_cuda_error_string() -> str:

@@ -329,8 +329,14 @@ const char* jmoe_status_string(jmoe_status s) {
         case JMOE_ECUDA: return "JMOE_ECUDA: CUDA call or launch failed";
         case JMOE_ETIMEOUT: return "JMOE_ETIMEOUT: a bounded device wait ran out";
         case JMOE_EDEVICE: return "JMOE_EDEVICE: invalid expert id seen on the device";
+        case JMOE_EBOUNDS: return "JMOE_EBOUNDS: a device bounds check failed";
     }
     return "unknown jmoe_status";
+}
+
+jmoe_status jmoe_test_check(void* stream) {
+    if (!jmoe::checks_built()) return JMOE_EUNSUPPORTED;
+    return from_cuda(jmoe::launch_check_probe((cudaStream_t)stream));
 }
 
 const char* jmoe_cuda_error_string(void) {
@@ -584,6 +590,9 @@ jmoe_status jmoe_last_error(void) {
     unsigned v = 0;
     if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return JMOE_ECUDA;
     if (v != 0 && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return JMOE_ECUDA;
+    v |= jmoe::checks_take_decode() | jmoe::checks_take_prefill() | jmoe::checks_take_permute() |
+         jmoe::checks_take_ep();
+    if (v & jmoe::kErrBounds) return JMOE_EBOUNDS;
     if (v & jmoe::kErrBadExpert) return JMOE_EDEVICE;
     if (v & jmoe::kErrTimeout) return JMOE_ETIMEOUT;
     return JMOE_OK;

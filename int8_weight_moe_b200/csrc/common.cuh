@@ -16,6 +16,38 @@ __device__ __forceinline__ void flag_error(unsigned* err, unsigned bit) {
     if (err) atomicOr(err, bit);
 }
 
+// Device bounds checks, compiled only into the JMOE_CHECKS=1 build
+// (libjmoe_checks.so): JMOE_CHECK(cond) is true when cond holds; when it does
+// not, it raises kErrBounds in this translation unit's check word and is
+// false, and the caller skips the access.  A check never traps.  In the
+// normal build it is the constant true and costs nothing.  Every source file
+// with checks defines its reader of the word (JMOE_DEFINE_CHECKS_READER);
+// jmoe_last_error reads and clears them all.
+#ifndef JMOE_CHECKS
+#define JMOE_CHECKS 0
+#endif
+#if JMOE_CHECKS
+namespace {
+__device__ unsigned s_check_word;  // one per translation unit
+}  // namespace
+#define JMOE_CHECK(cond) \
+    ((cond) ? true : (atomicOr(&::jmoe::s_check_word, ::jmoe::kErrBounds), false))
+#define JMOE_DEFINE_CHECKS_READER(name)                                                      \
+    unsigned name() {                                                                        \
+        unsigned v = 0;                                                                      \
+        if (cudaMemcpyFromSymbol(&v, s_check_word, sizeof(v)) != cudaSuccess) return kErrBounds; \
+        if (v) {                                                                             \
+            const unsigned z = 0;                                                            \
+            cudaMemcpyToSymbol(s_check_word, &z, sizeof(z));                                 \
+        }                                                                                    \
+        return v;                                                                            \
+    }
+#else
+#define JMOE_CHECK(cond) true
+#define JMOE_DEFINE_CHECKS_READER(name) \
+    unsigned name() { return 0; }
+#endif
+
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
     return __uint_as_float(((uint32_t)b) << 16);
 }
@@ -140,7 +172,8 @@ struct GemvParams {
     const int32_t* perm;       // [A]
     const uint16_t* b_src;     // x [T][d] (gate/up) or H [A][f] (down)
     float* P;                  // partial sums [S][A][cols]
-    int64_t A;
+    int64_t A;                 // assignment slots (rows of P and H)
+    int64_t T;                 // tokens (rows of the gate/up activation operand)
     unsigned* err;
     long long wait_cycles;     // bound of every mbarrier wait (SM cycles)
     int fault;                 // test hook: warp 0 of block 0 never issues its first copy

@@ -233,6 +233,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         const bool skip = p.fault && wid == 0 && issued == 0;
         if (skip) skipped = issued;
         if (lane == 0 && !skip) {
+            (void)JMOE_CHECK(pk + pj * kNB * 64 < K && pexp < E &&
+                             prow + (MODE == kGateUp ? 16 : 32) <= (MODE == kGateUp ? p.f : (int64_t)E * p.d));
             uint8_t* dst = ring + slot * kSlotBytes;
             sm100::mbar_arrive_expect_tx(&full[warp][slot], kSlotBytes);
             if (MODE == kGateUp)  // [expert][gate|up][row][k]: 16 rows of both halves
@@ -281,9 +283,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             // A column without a token reads the pass's first row instead: the
             // MMA keeps columns apart and that output column is never stored.
             const int slot = n * 8 + g8 < r.cnt_pass ? n * 8 + g8 : 0;
-            const int64_t row = MODE == kGateUp ? (int64_t)(p.perm[r.base + slot] / p.top_k)
-                                                : (int64_t)(r.base + slot);
-            r.b[n] = p.b_src + row * K + 16 * c + kz;
+            const int gi = r.base + slot;  // grouped index of the column's assignment
+            int64_t row = 0;
+            if (JMOE_CHECK(gi >= 0 && gi < p.A)) {
+                row = MODE == kGateUp ? (int64_t)(p.perm[gi] / p.top_k) : (int64_t)gi;
+                if (!JMOE_CHECK(row >= 0 && row < (MODE == kGateUp ? p.T : p.A))) row = 0;
+            }
+            const int64_t k0 = JMOE_CHECK(kz + (int64_t)kb_item * 64 <= K) ? kz : 0;
+            r.b[n] = p.b_src + row * K + 16 * c + k0;
         }
         return r;
     };
@@ -375,7 +382,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                             MODE == kGateUp
                                 ? (int64_t)m * p.f + cur.u.group * 16 + g8 + (i >> 1) * 8
                                 : (int64_t)cur.u.group * 32 + m * 16 + g8 + (i >> 1) * 8;
-                        if (slot < cur.cnt_pass)
+                        if (slot < cur.cnt_pass &&
+                            JMOE_CHECK(cur.base + slot < p.A && col < cols && cur.u.z < S))
                             P[(int64_t)(cur.base + slot) * cols + col] = acc[n][m][0][i] + acc[n][m][1][i];
                         acc[n][m][0][i] = acc[n][m][1][i] = 0.0f;
                     }
@@ -493,7 +501,8 @@ __global__ void __launch_bounds__(256)
             int e = 0;
             while (e + 1 < E && offsets[e + 1] <= slot) ++e;
             s_e = e;
-            s_sx = ldexpf(1.0f, xexp[perm[slot] / top_k]);
+            const int a = JMOE_CHECK(slot < A) ? perm[slot] : 0;
+            s_sx = ldexpf(1.0f, xexp[JMOE_CHECK(a >= 0 && a < A) ? a / top_k : 0]);
         }
         __syncthreads();
         if (n < f) {
@@ -509,7 +518,7 @@ __global__ void __launch_bounds__(256)
     pdl_launch_dependents();
     for (; slot < used; slot += gridDim.y) {
         int ex = 0;
-        if (n < f) {
+        if (n < f && JMOE_CHECK(slot < A)) {
             const float sx = s_sx;
             float vg[4] = {0.f, 0.f, 0.f, 0.f}, vu[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
@@ -541,8 +550,8 @@ __global__ void __launch_bounds__(256)
 // the bf16 values are kept exactly (8 significant bits, row maximum brought
 // into [2^14, 2^15)).
 __global__ void __launch_bounds__(256)
-    k_h16(const uint16_t* __restrict__ Hb, int64_t f, const int32_t* __restrict__ offsets, int E,
-          const int32_t* __restrict__ hmax, uint16_t* __restrict__ H16) {
+    k_h16(const uint16_t* __restrict__ Hb, int64_t f, int64_t A, const int32_t* __restrict__ offsets,
+          int E, const int32_t* __restrict__ hmax, uint16_t* __restrict__ H16) {
     pdl_wait();
     // only after the wait: the down GEMV relies on it (it reads the grouping
     // tables before its own wait)
@@ -551,6 +560,7 @@ __global__ void __launch_bounds__(256)
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
          v += (int64_t)gridDim.x * blockDim.x) {
         const int slot = (int)((2 * v) / f);
+        if (!JMOE_CHECK(slot < A)) break;
         const float scale = ldexpf(1.0f, -row_shift(hmax[slot]));
         const uint32_t u = reinterpret_cast<const uint32_t*>(Hb)[v];
         const __half2 h = __floats2half2_rn(__uint_as_float(u << 16) * scale,
@@ -584,7 +594,7 @@ __global__ void __launch_bounds__(256)
             const int64_t a = t * top_k + threadIdx.x;
             const int e = ids[a];
             const int slot = inv[a];
-            const bool ok = e >= 0 && e < E && slot >= 0;
+            const bool ok = e >= 0 && e < E && slot >= 0 && JMOE_CHECK(slot < A);
             s_slot[threadIdx.x] = ok ? slot : -1;
             s_e[threadIdx.x] = ok ? e : 0;
             s_gw[threadIdx.x] = gates[a];
@@ -714,6 +724,7 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
     p.d = a.d;
     p.f = a.f;
     p.A = a.A;
+    p.T = a.T;
     p.offsets = a.offsets;
     p.perm = a.perm;
     p.err = a.err;
@@ -743,7 +754,7 @@ cudaError_t launch_decode_nch(const DecodeArgs& a, cudaStream_t stream) {
                          static_cast<uint16_t*>(a.Hb), a.hmax);
         if (err == cudaSuccess)
             err = launch_pdl(k_h16, dim3(grid_for(a.A * a.f / 2, a.num_sms, 8)), dim3(256), 0,
-                             stream, static_cast<const uint16_t*>(a.Hb), a.f, a.offsets, a.E,
+                             stream, static_cast<const uint16_t*>(a.Hb), a.f, a.A, a.offsets, a.E,
                              a.hmax, static_cast<uint16_t*>(a.H));
     }
     if (a.mark) a.mark(5, true, stream);
@@ -797,6 +808,21 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
                      static_cast<const int32_t*>(a.hmax), a.sd, static_cast<uint16_t*>(a.out));
     if (a.mark) a.mark(4, true, stream);
     return err;
+}
+
+JMOE_DEFINE_CHECKS_READER(checks_take_decode)
+
+namespace {
+// The bounds-check build's self-test: one check that fails (n > 0), no access.
+__global__ void k_check_probe(int n) { (void)JMOE_CHECK(n <= 0); }
+}  // namespace
+
+bool checks_built() { return JMOE_CHECKS != 0; }
+
+cudaError_t launch_check_probe(cudaStream_t stream) {
+    k_check_probe<<<1, 1, 0, stream>>>(1);
+    note_launch();
+    return cudaGetLastError();
 }
 
 }  // namespace jmoe

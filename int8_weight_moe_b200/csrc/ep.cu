@@ -26,7 +26,7 @@ namespace {
 // One warp per send row, 16-byte moves; lane 0 writes the row's expert index
 // within its owner rank.
 __global__ void __launch_bounds__(256)
-    k_ep_pack(const uint16_t* __restrict__ x, int64_t d, int top_k,
+    k_ep_pack(const uint16_t* __restrict__ x, int64_t T, int64_t d, int top_k,
               const int32_t* __restrict__ ids, const int32_t* __restrict__ perm,
               const int32_t* __restrict__ offsets, int E, int E_local,
               uint16_t* __restrict__ x_send, int32_t* __restrict__ local_ids) {
@@ -37,7 +37,9 @@ __global__ void __launch_bounds__(256)
     const int64_t nvec = d / 8;
     for (int64_t i = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); i < rows;
          i += (int64_t)gridDim.x * 8) {
+        if (!JMOE_CHECK(i < T * top_k)) break;
         const int32_t a = perm[i];
+        if (!JMOE_CHECK(a >= 0 && a < T * top_k)) continue;
         const int64_t t = a / top_k;
         const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
         uint4* dst = reinterpret_cast<uint4*>(x_send + i * d);
@@ -65,7 +67,7 @@ __global__ void __launch_bounds__(256)
         for (int j = 0; j < top_k; ++j) {
             const int64_t a = t * top_k + j;
             const int32_t slot = inv[a];
-            if (slot < 0) continue;
+            if (slot < 0 || !JMOE_CHECK(slot < T * top_k)) continue;
             const float g = gates[a];
             const uint2 v = *reinterpret_cast<const uint2*>(y_back + (int64_t)slot * d + m);
             o[0] += g * bf16_bits_to_f32((uint16_t)(v.x & 0xffffu));
@@ -94,7 +96,7 @@ cudaError_t launch_ep_dispatch(const void* x, int64_t T, int64_t d, const int32_
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     return launch_pdl(k_ep_pack, dim3((unsigned)blocks), dim3(256), 0, stream,
-                      static_cast<const uint16_t*>(x), d, top_k, ids,
+                      static_cast<const uint16_t*>(x), T, d, top_k, ids,
                       static_cast<const int32_t*>(perm), static_cast<const int32_t*>(offsets), E,
                       E_local, static_cast<uint16_t*>(x_send), local_ids);
 }
@@ -107,5 +109,7 @@ cudaError_t launch_ep_combine(const void* y_back, const int32_t* inv, const floa
                       dim3(256), 0, stream, static_cast<const uint16_t*>(y_back), inv, gates, T, d,
                       top_k, static_cast<uint16_t*>(out));
 }
+
+JMOE_DEFINE_CHECKS_READER(checks_take_ep)
 
 }  // namespace jmoe

@@ -31,7 +31,21 @@ bool encode_4d_u8(CUtensorMap* map, const void* base, const uint64_t (&dims)[4],
 enum : unsigned {
     kErrTimeout = 1u,    // a bounded wait ran out
     kErrBadExpert = 2u,  // an expert id outside [0, E)
+    kErrBounds = 4u,     // a device bounds check failed (JMOE_CHECKS build only)
 };
+
+// Readers of the per-file device check words of the JMOE_CHECKS build (read
+// and clear; 0 in the normal build).  Call with the device current, after a
+// synchronisation.
+unsigned checks_take_decode();
+unsigned checks_take_prefill();
+unsigned checks_take_permute();
+unsigned checks_take_ep();
+// Whether this is the JMOE_CHECKS build, and a kernel whose one check fails
+// while touching no memory (the jmoe_test_check hook; a no-op in the normal
+// build, which has no checks).
+bool checks_built();
+cudaError_t launch_check_probe(cudaStream_t stream);
 
 // Largest bound a caller may give the kernels' mbarrier waits (SM cycles,
 // about 4 s at 2 GHz).
@@ -62,7 +76,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_
                            int32_t* padded_offsets, int32_t* perm, int32_t* inv, unsigned* err,
                            cudaStream_t stream);
 
-cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
+cudaError_t launch_gather_rows(const void* x_bf16, int64_t T, int64_t d, int top_k, int E,
                                const int32_t* offsets, const int32_t* padded_offsets,
                                const int32_t* perm, int64_t max_rows, void* x_perm, int num_sms,
                                cudaStream_t stream);

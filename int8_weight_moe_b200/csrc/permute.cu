@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(kPermuteThreads)
 __global__ void __launch_bounds__(256)
     k_gather_rows(const uint16_t* __restrict__ x, int64_t d, int top_k, int E,
                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ padded_offsets,
-                  const int32_t* __restrict__ perm, int64_t max_rows, uint16_t* __restrict__ x_perm) {
+                  const int32_t* __restrict__ perm, int64_t T, int64_t max_rows,
+                  uint16_t* __restrict__ x_perm) {
     __shared__ int s_off[kMaxE + 1], s_poff[kMaxE + 1];
     if (threadIdx.x <= E) {
         s_off[threadIdx.x] = offsets[threadIdx.x];
@@ -46,7 +47,10 @@ __global__ void __launch_bounds__(256)
         const int64_t r = row - s_poff[e];
         uint4* dst = reinterpret_cast<uint4*>(x_perm + row * d);
         if (r < s_off[e + 1] - s_off[e]) {
-            const int64_t t = perm[s_off[e] + r] / top_k;
+            const int64_t g = s_off[e] + r;
+            if (!JMOE_CHECK(g < (int64_t)T * top_k)) continue;
+            const int64_t t = perm[g] / top_k;
+            if (!JMOE_CHECK(t >= 0 && t < T)) continue;
             const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
             for (int64_t i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
         } else {
@@ -80,7 +84,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t A, int E, int pad, int32_
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
+cudaError_t launch_gather_rows(const void* x_bf16, int64_t T, int64_t d, int top_k, int E,
                                const int32_t* offsets, const int32_t* padded_offsets,
                                const int32_t* perm, int64_t max_rows, void* x_perm, int num_sms,
                                cudaStream_t stream) {
@@ -89,10 +93,12 @@ cudaError_t launch_gather_rows(const void* x_bf16, int64_t d, int top_k, int E,
     const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
     k_gather_rows<<<(unsigned)blocks, 256, 0, stream>>>((const uint16_t*)x_bf16, d, top_k, E,
-                                                        offsets, padded_offsets, perm, max_rows,
+                                                        offsets, padded_offsets, perm, T, max_rows,
                                                         (uint16_t*)x_perm);
     note_launch();
     return cudaGetLastError();
 }
+
+JMOE_DEFINE_CHECKS_READER(checks_take_permute)
 
 }  // namespace jmoe

@@ -90,8 +90,10 @@ __device__ __forceinline__ void warp_permute(const int32_t* __restrict__ ids, in
         const unsigned lower = peers & ((1u << lane) - 1u);
         if (e >= 0) {
             const int pos = s_cursor[e] + __popc(lower);
-            perm[pos] = (int32_t)a;
-            if (inv) inv[a] = pos;
+            if (JMOE_CHECK(pos >= 0 && pos < A)) {
+                perm[pos] = (int32_t)a;
+                if (inv) inv[a] = pos;
+            }
         } else if (a < A && inv) {
             inv[a] = -1;
         }
@@ -167,8 +169,10 @@ __device__ __forceinline__ void block_permute(const int32_t* __restrict__ ids, i
         __syncthreads();
         if (e >= 0) {
             const int pos = s_cursor[e] + s_warp_base[warp][e] + rank;
-            perm[pos] = (int32_t)a;
-            if (inv) inv[a] = pos;
+            if (JMOE_CHECK(pos >= 0 && pos < A)) {
+                perm[pos] = (int32_t)a;
+                if (inv) inv[a] = pos;
+            }
         } else if (a < A && inv) {
             inv[a] = -1;
         }

@@ -141,6 +141,8 @@ struct GemmParams {
     unsigned* err;
     long long wait_cycles;  // bound of every mbarrier wait (SM cycles)
     int fault_tile;         // < 0: none; else the weight producers stop before this tile
+    int rows_padded;        // rows of H (bounds checks)
+    int A;                  // assignments: rows of Y, entries of perm and gates (bounds checks)
 };
 
 struct Shared {
@@ -470,16 +472,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
                             }
                             uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+                            if (JMOE_CHECK(row >= 0 && row < p.rows_padded))
 #pragma unroll
-                            for (int qq = 0; qq < 4; ++qq)
-                                dst[qq] = make_uint4(packed[4 * qq], packed[4 * qq + 1], packed[4 * qq + 2],
-                                                     packed[4 * qq + 3]);
+                                for (int qq = 0; qq < 4; ++qq)
+                                    dst[qq] = make_uint4(packed[4 * qq], packed[4 * qq + 1],
+                                                         packed[4 * qq + 2], packed[4 * qq + 3]);
                         }
                     } else {
                         const int m0 = t.n * BN;
                         const int r = row - S.poff[t.e];
-                        const bool valid = r < S.off[t.e + 1] - S.off[t.e];
-                        const int a = valid ? p.perm[S.off[t.e] + r] : 0;
+                        const int gi = S.off[t.e] + r;  // grouped index of the row
+                        bool valid = r < S.off[t.e + 1] - S.off[t.e];
+                        valid = valid && JMOE_CHECK(gi >= 0 && gi < p.A);
+                        const int a = valid ? p.perm[gi] : 0;
+                        valid = valid && JMOE_CHECK(a >= 0 && a < p.A);
                         const float gate = valid ? p.gates[a] : 0.0f;
                         const float* sd = p.scale + (size_t)t.e * p.w_rows;
 #pragma unroll 1
@@ -575,7 +581,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     cudaError_t err;
     // 1. gather the routed activation rows, grouped by expert, padded per expert
     if (a.mark) a.mark(1, false, stream);
-    err = launch_gather_rows(a.x, a.d, a.top_k, a.E, a.offsets, a.padded_offsets, a.perm,
+    err = launch_gather_rows(a.x, a.T, a.d, a.top_k, a.E, a.offsets, a.padded_offsets, a.perm,
                              a.rows_padded, a.xperm, a.num_sms, stream);
     if (a.mark) a.mark(1, true, stream);
     if (err != cudaSuccess) return err;
@@ -609,6 +615,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     g1.err = a.err;
     g1.wait_cycles = a.wait_cycles > 0 ? a.wait_cycles : kWaitCycles;
     g1.fault_tile = a.fault_tile;
+    g1.rows_padded = (int)a.rows_padded;
+    g1.A = (int)a.A;
     if (a.mark) a.mark(2, false, stream);
     err = launch_gemm<kGateUp>(mA1, mB1, g1, a.num_sms, (int)tile_bound(a, g1.n_tiles), stream);
     if (a.mark) a.mark(2, true, stream);
@@ -637,5 +645,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
+
+JMOE_DEFINE_CHECKS_READER(checks_take_prefill)
 
 }  // namespace jmoe

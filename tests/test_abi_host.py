@@ -138,6 +138,23 @@ def test_launch_counter_counts_nothing_for_rejected_calls():
     assert jm.jmoe_launch_count() == n0
 
 
+def test_check_hook_is_unsupported_in_the_normal_build():
+    # the normal build has no device checks: the hook refuses before any CUDA call
+    assert jm.load().jmoe_test_check(None) == jm.JMOE_EUNSUPPORTED
+    assert jm.status_string(jm.JMOE_EBOUNDS).startswith("JMOE_EBOUNDS")
+
+
+def test_checks_build_exports_the_same_symbols():
+    import ctypes
+    import os
+
+    if not os.path.exists(jm.CHECKS_LIB_PATH):
+        pytest.skip("libjmoe_checks.so not built")
+    lib = ctypes.CDLL(jm.CHECKS_LIB_PATH)
+    for name in jm.EXPORTED:
+        assert hasattr(lib, name), name
+
+
 def test_stall_hook_validation():
     lib = jm.load()
     assert lib.jmoe_test_stall(3, 2_000_000) == jm.JMOE_EINVAL

@@ -33,8 +33,10 @@
 //   warp 1      TMEM allocator (both CTAs); issuer 0 (even CTA only)
 //   warp 2      TMA producer of the CTA's INT8 weight rows [128 x 64 k]
 //   warps 3-10  converters INT8 -> BF16 (shared -> shared, swizzled), in two
-//               groups of 4 that take alternate k-steps
-//   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM
+//               groups of 4 that take alternate k-steps; group h also drains
+//               the second half of accumulator h while the ring is full
+//   warps 11-14 epilogue: TMEM -> registers -> scale / SwiGLU / gate -> HBM,
+//               the first half of every accumulator
 //   warp 15     issuer 1 (even CTA only)
 //
 // Gate/up tiles: the even CTA converts 128 gate channels, the odd CTA the
@@ -57,10 +59,15 @@
 //                           BF16 weights after seeing their CTA's A land
 //   empty_b[s]  (each CTA)  both issuers' MMAs reading BF16 stage s are done
 //   acc_full[h] (each CTA)  accumulator h is final (issuer h's commit multicast)
-//   acc_empty[h] (even CTA) the epilogue warps of both CTAs read it
-// The two accumulators of 256 fp32 columns take all 512 TMEM columns; the
-// epilogue reads accumulator 0 first, so issuer 0 starts its next tile while
-// the epilogue still reads accumulator 1.  Tiles are visited expert by
+//   acc_empty[h] (even CTA) the epilogue warps and converter group h of both
+//                           CTAs read it
+// The two accumulators of 256 fp32 columns take all 512 TMEM columns.  A
+// drain (about 5 us for a whole accumulator with four warps, the SwiGLU's
+// exponentials and divisions the largest part) is split: the epilogue warps
+// take the first half of accumulator 0 and then of 1, converter group h the
+// second half of accumulator h; the converters are idle then anyway, since
+// the ring stays full until the issuers restart, and the issuers restart
+// only after the drain.  Tiles are visited expert by
 // expert in groups of 16 m-tiles (see decode_tile).  No TMA load is
 // multicast; every copy reads global memory into its own CTA.
 #include <cuda.h>
@@ -227,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&S.acc_full[i], 1);  // issuer i's commit
-            mbar_init(&S.acc_empty[i], 2 * kEpiWarps);
+            mbar_init(&S.acc_empty[i], 2 * (kEpiWarps + kConvGroupWarps));  // both CTAs' drainers
         }
         mbar_init(&S.drain, kIssuers);
         S.abort = 0;
@@ -266,6 +273,99 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto wait = [&](uint64_t* bar, uint32_t parity) {
         return mbar_wait_pair(bar, parity, abort, peer_abort, limit);
     };
+
+    // Drains chunks [c_lo, c_hi) (32 columns each; gate/up: 32 channels, whose
+    // gate and up columns sit 128 apart) of accumulator h of tile t into H or
+    // Y, from this warp's TMEM lane quadrant: wait for the accumulator, read,
+    // scale (SwiGLU / gate), store, and arrive on acc_empty[h] of the even CTA.
+    // The epilogue warps drain the first half of every accumulator, converter
+    // group h the second half of accumulator h.
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(&S.acc_empty[0]), 0);
+    auto drain = [&](const Tile& t, int h, int& uses_h, int c_lo, int c_hi) {
+        const int quad = warp & 3;
+        if (!__all_sync(0xffffffffu, wait(&S.acc_full[h], uses_h & 1))) return false;
+        ++uses_h;
+        tc_fence_after();
+        const int q = 2 * h + (int)rank;
+        if (q < t.quarters) {
+            const uint32_t taddr = tmem + h * BN + ((uint32_t)(quad * 32) << 16);
+            const int row = t.row0 + q * BH + quad * 32 + lane;
+            if (MODE == kGateUp) {
+                const int n0 = t.n * BNC;
+                const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
+                const float* su = sg + p.up_offset;
+#pragma unroll 1
+                for (int c = c_lo; c < c_hi; ++c) {
+                    const int ch = n0 + c * 32;
+                    if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
+                    // gate channel n0 + r: column r (the even CTA's B row r);
+                    // its up channel: column 128 + r (the odd CTA's row r)
+                    uint32_t gv[32], uv[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, gv);
+                    tmem_ld_32x32b_x32(taddr + BNC + c * 32, uv);
+                    tmem_ld_wait();
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
+                        const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
+                        const float g0 = g4.x * __uint_as_float(gv[j]);
+                        const float g1 = g4.y * __uint_as_float(gv[j + 1]);
+                        const float g2 = g4.z * __uint_as_float(gv[j + 2]);
+                        const float g3 = g4.w * __uint_as_float(gv[j + 3]);
+                        const float u0 = u4.x * __uint_as_float(uv[j]);
+                        const float u1 = u4.y * __uint_as_float(uv[j + 1]);
+                        const float u2 = u4.z * __uint_as_float(uv[j + 2]);
+                        const float u3 = u4.w * __uint_as_float(uv[j + 3]);
+                        packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                        packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
+                    if (JMOE_CHECK(row >= 0 && row < p.rows_padded))
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq)
+                            dst[qq] = make_uint4(packed[4 * qq], packed[4 * qq + 1],
+                                                 packed[4 * qq + 2], packed[4 * qq + 3]);
+                }
+            } else {
+                const int m0 = t.n * BN;
+                const int r = row - S.poff[t.e];
+                const int gi = S.off[t.e] + r;  // grouped index of the row
+                bool valid = r < S.off[t.e + 1] - S.off[t.e];
+                valid = valid && JMOE_CHECK(gi >= 0 && gi < p.A);
+                const int a = valid ? p.perm[gi] : 0;
+                valid = valid && JMOE_CHECK(a >= 0 && a < p.A);
+                const float gate = valid ? p.gates[a] : 0.0f;
+                const float* sd = p.scale + (size_t)t.e * p.w_rows;
+#pragma unroll 1
+                for (int c = c_lo; c < c_hi; ++c) {
+                    const int m = m0 + c * 32;  // column c: the even CTA's rows, then the odd's
+                    if (m >= p.n_valid) break;  // n_valid is a multiple of 64
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + c * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq) {
+                            const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + qq);
+                            float4 o;
+                            o.x = gate * (s4.x * __uint_as_float(v[4 * qq]));
+                            o.y = gate * (s4.y * __uint_as_float(v[4 * qq + 1]));
+                            o.z = gate * (s4.z * __uint_as_float(v[4 * qq + 2]));
+                            o.w = gate * (s4.w * __uint_as_float(v[4 * qq + 3]));
+                            dst[qq] = o;
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader + h * (uint32_t)sizeof(uint64_t));
+        return true;
+    };
+    constexpr int kAccChunks = (MODE == kGateUp ? BNC : BN) / 32;  // chunks of an accumulator
 
     if (warp == kWarpProdA) {
         if (lane == 0) {
@@ -371,8 +471,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t full_leader = mapa_shared(smem_u32(&S.full[0]), 0);
         uint32_t g = 0;
         bool ok = true;
+        // The group also drains the second half of accumulator G of the
+        // previous tile, at the point where it would otherwise wait for this
+        // tile's MMAs to free a stage -- which needs issuer G to restart, which
+        // needs the drain: k-step kStagesB of the next tile, or the end of the
+        // next tile's k-steps when it has fewer, or after the last tile.
+        int help_uses = 0, pending = -1;
+        auto help = [&](int tile) {
+            const Tile t = decode_tile(S, E, p.n_tiles, tile);
+            if (2 * G >= t.quarters) return true;  // issuer G had no rows in this tile
+            return drain(t, G, help_uses, kAccChunks / 2, kAccChunks);
+        };
         for (int tile = pair; tile < total && ok && !*abort; tile += npairs) {
             for (int kb = 0; kb < KB; ++kb, ++g) {
+                if (pending >= 0 && kb == kStagesB) {
+                    ok = help(pending);
+                    pending = -1;
+                    if (!ok) break;
+                }
                 if ((int)(g & 1) != G) continue;
                 const int s = g % kStagesB;
                 const uint32_t ph = (g / kStagesB) & 1;
@@ -419,101 +535,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     break;
                 }
             }
+            if (ok && pending >= 0) ok = help(pending);
+            pending = tile;
         }
+        if (ok && pending >= 0 && !*abort) help(pending);  // the last tile
     } else {
-        // epilogue warps: TMEM lane quadrant = warp % 4; per tile, accumulator h
-        // holds this CTA's quarter 2h + rank (128 rows x 256 columns)
-        const int quad = warp & 3;
-        const uint32_t acc_empty_leader = mapa_shared(smem_u32(&S.acc_empty[0]), 0);
+        // epilogue warps (TMEM lane quadrant = warp % 4): per tile, the first
+        // half of accumulator h (this CTA's quarter 2h + rank: 128 rows x 256
+        // columns), accumulator 0 first
         int uses[2] = {0, 0};
         bool ok = true;
         for (int tile = pair; tile < total && ok && !*abort; tile += npairs) {
             const Tile t = decode_tile(S, E, p.n_tiles, tile);
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 2 && ok; ++h) {
                 if (2 * h >= t.quarters) break;  // issuer h had no rows in this tile
-                if (!__all_sync(0xffffffffu, wait(&S.acc_full[h], uses[h] & 1))) {
-                    ok = false;
-                    break;
-                }
-                ++uses[h];
-                tc_fence_after();
-                const int q = 2 * h + (int)rank;
-                if (q < t.quarters) {
-                    const uint32_t taddr = tmem + h * BN + ((uint32_t)(quad * 32) << 16);
-                    const int row = t.row0 + q * BH + quad * 32 + lane;
-                    if (MODE == kGateUp) {
-                        const int n0 = t.n * BNC;
-                        const float* sg = p.scale + (size_t)t.e * p.w_rows + n0;
-                        const float* su = sg + p.up_offset;
-#pragma unroll 1
-                        for (int c = 0; c < BNC / 32; ++c) {
-                            const int ch = n0 + c * 32;
-                            if (ch >= p.n_valid) break;  // n_valid is a multiple of 64
-                            // gate channel n0 + r: column r (the even CTA's B row r);
-                            // its up channel: column 128 + r (the odd CTA's row r)
-                            uint32_t gv[32], uv[32];
-                            tmem_ld_32x32b_x32(taddr + c * 32, gv);
-                            tmem_ld_32x32b_x32(taddr + BNC + c * 32, uv);
-                            tmem_ld_wait();
-                            uint32_t packed[16];
-#pragma unroll
-                            for (int j = 0; j < 32; j += 4) {
-                                const float4 g4 = __ldg(reinterpret_cast<const float4*>(sg + c * 32 + j));
-                                const float4 u4 = __ldg(reinterpret_cast<const float4*>(su + c * 32 + j));
-                                const float g0 = g4.x * __uint_as_float(gv[j]);
-                                const float g1 = g4.y * __uint_as_float(gv[j + 1]);
-                                const float g2 = g4.z * __uint_as_float(gv[j + 2]);
-                                const float g3 = g4.w * __uint_as_float(gv[j + 3]);
-                                const float u0 = u4.x * __uint_as_float(uv[j]);
-                                const float u1 = u4.y * __uint_as_float(uv[j + 1]);
-                                const float u2 = u4.z * __uint_as_float(uv[j + 2]);
-                                const float u3 = u4.w * __uint_as_float(uv[j + 3]);
-                                packed[j / 2] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-                                packed[j / 2 + 1] = pack_bf16x2(silu_f32(g2) * u2, silu_f32(g3) * u3);
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(p.H + (size_t)row * p.n_valid + ch);
-                            if (JMOE_CHECK(row >= 0 && row < p.rows_padded))
-#pragma unroll
-                                for (int qq = 0; qq < 4; ++qq)
-                                    dst[qq] = make_uint4(packed[4 * qq], packed[4 * qq + 1],
-                                                         packed[4 * qq + 2], packed[4 * qq + 3]);
-                        }
-                    } else {
-                        const int m0 = t.n * BN;
-                        const int r = row - S.poff[t.e];
-                        const int gi = S.off[t.e] + r;  // grouped index of the row
-                        bool valid = r < S.off[t.e + 1] - S.off[t.e];
-                        valid = valid && JMOE_CHECK(gi >= 0 && gi < p.A);
-                        const int a = valid ? p.perm[gi] : 0;
-                        valid = valid && JMOE_CHECK(a >= 0 && a < p.A);
-                        const float gate = valid ? p.gates[a] : 0.0f;
-                        const float* sd = p.scale + (size_t)t.e * p.w_rows;
-#pragma unroll 1
-                        for (int c = 0; c < BN / 32; ++c) {
-                            const int m = m0 + c * 32;  // column c: the even CTA's rows, then the odd's
-                            if (m >= p.n_valid) break;  // n_valid is a multiple of 64
-                            uint32_t v[32];
-                            tmem_ld_32x32b_x32(taddr + c * 32, v);
-                            tmem_ld_wait();
-                            if (valid) {
-                                float4* dst = reinterpret_cast<float4*>(p.Y + (size_t)a * p.n_valid + m);
-#pragma unroll
-                                for (int qq = 0; qq < 8; ++qq) {
-                                    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sd + m) + qq);
-                                    float4 o;
-                                    o.x = gate * (s4.x * __uint_as_float(v[4 * qq]));
-                                    o.y = gate * (s4.y * __uint_as_float(v[4 * qq + 1]));
-                                    o.z = gate * (s4.z * __uint_as_float(v[4 * qq + 2]));
-                                    o.w = gate * (s4.w * __uint_as_float(v[4 * qq + 3]));
-                                    dst[qq] = o;
-                                }
-                            }
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(acc_empty_leader + h * (uint32_t)sizeof(uint64_t));
+                ok = drain(t, h, uses[h], 0, kAccChunks / 2);
             }
         }
     }

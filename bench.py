@@ -390,9 +390,9 @@ def roofline_entry(layer: Layer, stages: dict, peaks: dict):
     if ms is None or ms <= 0:
         return None
     if layer.prefill_path():
-        # The target is judged against the dense BF16 peak measured on this
-        # pool (a cuBLAS GEMM timed alone, `bf16_tflops`); the power-capped
-        # sustained rate and the data-sheet figure ride along.
+        # The target's dense BF16 peak is the measured rate of a cuBLAS GEMM
+        # timed alone (`bf16_tflops`); the power-capped sustained rate and the
+        # data-sheet figure ride along.
         achieved = work["gate_up_flops"] / (ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         return {"bound": "tensor", "kernel": "gate_up", "achieved": round(achieved, 2),

@@ -19,7 +19,7 @@
  *         g renormalised over the selected set; and the layer list (experts
  *         are MLPs with SwiGLU activation).
  *
- * Readings where the pages leave a step open (all listed in the design doc):
+ * Readings where the pages leave a step open:
  *  - quantisation is symmetric, per output row (output channel), with
  *    scale s = absmax/127 computed as one fp32 division, q = round-half-even
  *    of the fp32 quotient w/s, clamped to [-127, 127]; an all-zero row gets

@@ -57,10 +57,13 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
 
 @pytest.mark.gpu
 def test_noalloc_refuses_problems_beyond_its_scratch():
-    # Large-sized layer, 64 tokens top-2: the decode scratch would be ~37 MiB,
+    # Large-sized layer, 96 tokens top-2: the decode scratch would be ~56 MiB,
     # more than the fixed 32 MiB array; refused on the host, nothing launched.
     desc = jm.MoeDesc(16, 2, 8192, 24576, GOOD, GOOD, GOOD, GOOD, 0)
-    st = jm.load().jmoe_forward_noalloc(ctypes.byref(desc), GOOD, 64, GOOD, GOOD, GOOD, None)
+    too_big = jm.jmoe_forward_workspace_size(
+        jm.MoeDesc(16, 2, 8192, 24576, GOOD, GOOD, GOOD, GOOD, jm.JMOE_PATH_DECODE), 96)
+    assert too_big > jm.NOALLOC_SCRATCH_BYTES
+    st = jm.load().jmoe_forward_noalloc(ctypes.byref(desc), GOOD, 96, GOOD, GOOD, GOOD, None)
     assert st == jm.JMOE_EWORKSPACE
     ok_size = jm.jmoe_forward_workspace_size(
         jm.MoeDesc(16, 2, 8192, 24576, GOOD, GOOD, GOOD, GOOD, jm.JMOE_PATH_DECODE), 32)

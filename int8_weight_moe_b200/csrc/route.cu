@@ -14,9 +14,9 @@
 // is added in fp64 and the result rounded once to fp32.  The products are
 // exact in fp64 (8-bit x 24-bit significands).
 //
-// Work split: for many tokens a CTA of 8 warps handles 16 tokens with the
+// Work split: for many tokens a CTA of 8 warps handles 32 tokens with the
 // router rows and token rows staged in shared memory (k_route_tiles: each
-// lane keeps 8 tokens x 4 experts of fp64 partial sums).
+// lane keeps 8 tokens x 8 experts of fp64 partial sums).
 // For few tokens (decode) one warp per expert: a cluster of 4 CTAs per token
 // (each warp's router row copied to shared memory in one round trip, logits
 // gathered in the first CTA through distributed shared memory), or for rows
@@ -309,117 +309,293 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// Many tokens: a CTA of 8 warps computes the logits of 16 tokens, one group
-// of 16 experts at a time.  The group's router rows and the tokens' rows go
-// through shared memory in k-chunks of 512 (16-byte cp.async copies, the next
-// chunk landing while this one is summed); warp w keeps the fp64 partial sums
-// of tokens 8 (w / 4) .. +7 for experts w % 4, w % 4 + 4, w % 4 + 8, w % 4 + 12
-// of the group.  Lane j accumulates k = j (mod 32) in ascending k across the
-// chunks (the canonical order), so every router weight a lane reads serves 8
-// tokens and every token value 4 experts, and a CTA reads each router row
-// once per 16 tokens.
-constexpr int kTileTok = 16, kTileWarps = 8, kTileChunk = 512;
-constexpr int kTileTokPerWarp = 8, kTileExpPerWarp = 4;
-constexpr int kTileWBytes = kGroupE * kTileChunk * 4;     // 32 KB of router rows
-constexpr int kTileXBytes = kTileTok * kTileChunk * 2;    // 16 KB of token rows
-constexpr size_t kTileSmem = 2 * (size_t)(kTileWBytes + kTileXBytes);
-static_assert(kTileWarps * kTileTokPerWarp * kTileExpPerWarp == kTileTok * kGroupE,
-              "the warps cover the 16 tokens x 16 experts of a group");
+// Many tokens: a CTA of 8 warps computes the logits of 32 tokens, one group
+// of 16 experts at a time, the router rows and token rows streamed through
+// shared memory in k-chunks of 256 (16-byte cp.async copies, four chunks in
+// flight).  Warp w keeps the fp64 partial sums of tokens 8 (w / 2) .. +7 for
+// the experts w % 2, w % 2 + 2, ..., w % 2 + 14 of the group; lane j
+// accumulates k = j (mod 32) in ascending k across the chunks (the canonical
+// order), so every router weight a lane reads serves 8 tokens and every token
+// value 8 experts.
+//
+// No conversion instruction runs in the inner loop (an fp32 -> fp64
+// conversion issues at a small fraction of the fp64 FMA rate).  Each product
+// x * w is formed as (x * 2^-896) * (w * 2^896), which is the same real
+// number, so every fused multiply-add -- and every rounding of the canonical
+// order -- is unchanged:
+// - x * 2^-896 is the bf16 bit pattern moved into the fp64 fields: the 8-bit
+//   exponent field read with the fp64 bias (1023 instead of 127) is exactly
+//   that scaling, for zeros and subnormals too; only an all-ones exponent
+//   (inf, NaN) maps wrongly, so a chunk holding one takes the exact
+//   conversion for it (a CTA-wide flag found while the chunk is staged);
+// - w * 2^896 is exact for every fp32 value (2^127 * 2^896 = 2^1023 still
+//   fits) and is written to shared memory in fp64 once per CTA and chunk,
+//   by integer field arithmetic for normal numbers and by the conversion
+//   instruction otherwise.
+constexpr int kRtTok = 32, kRtK = 256, kRtStages = 4;
+constexpr int kRtTokPerWarp = 8, kRtExpPerWarp = 8;
+constexpr int kRtEStride = kGroupE / kRtExpPerWarp;  // warps per token group; expert stride
+constexpr int kRtWarps = kRtTok / kRtTokPerWarp * kRtEStride;
+constexpr int kRtSums = kRtTokPerWarp * kRtExpPerWarp / 32;  // sums a lane holds after the tree
+constexpr int kRtPrep = kGroupE * kRtK / 4 / (kRtWarps * 32);  // 16-byte pieces per thread and half
+constexpr int kRtWRawBytes = kGroupE * kRtK * 4;          // 16 KB: fp32 router rows
+constexpr int kRtXBytes = kRtTok * kRtK * 2;              // 16 KB: bf16 token rows
+constexpr int kRtStageBytes = kRtWRawBytes + kRtXBytes;
+constexpr int kRtW64Bytes = kGroupE * kRtK * 8;           // 32 KB: scaled fp64 router rows
+constexpr int kRtLogitBytes = kRtTok * kMaxE * 4;         // 8 KB
+constexpr size_t kTileSmem = (size_t)kRtStages * kRtStageBytes + 2 * (size_t)kRtW64Bytes +
+                             2 * (size_t)kRtLogitBytes;
+static_assert(kRtWarps * kRtTokPerWarp * kRtExpPerWarp == kRtTok * kGroupE,
+              "the warps cover the 32 tokens x 16 experts of a group");
+static_assert(kRtK % 64 == 0, "chunks hold whole 64-wide pieces of a row");
+static_assert(kRtTok * kRtK / 8 == kGroupE * kRtK / 4, "token and router rows split alike");
 
-__global__ void __launch_bounds__(kTileWarps * 32, 2)
+// x * 2^-896 from the bf16 bits sign-extended to 32 bits (s << 13 puts the
+// exponent field at bits 20..27, the mantissa at 13..19 and copies of the
+// sign at 28..31; the mask keeps bit 31 of those).
+__device__ __forceinline__ double rt_x_scaled(int s) {
+    return __hiloint2double((int)(((uint32_t)s << 13) & 0x8fffe000u), 0);
+}
+
+// w * 2^896 in fp64 (the exponent field grows by 1792 = 896 + 1023 - 127).
+__device__ __forceinline__ double rt_w_scaled(uint32_t b) {
+    if ((b & 0x7f800000u) - 0x00800000u < 0x7f000000u) {  // normal
+        const uint32_t hi = ((uint32_t)((int32_t)b >> 3) & 0x8fffffffu) + 0x70000000u;
+        return __hiloint2double((int)hi, (int)(b << 29));
+    }
+    return (double)__uint_as_float(b) * 0x1p896;
+}
+
+// One chunk of the warp's kRtTokPerWarp tokens x kRtExpPerWarp experts: n
+// (a multiple of 32) values of each row, X the warp's first token row, Wd its
+// first scaled router row (the warp's experts are kRtEStride rows apart); ne
+// of its experts exist (all of them when kFull).  The operands of the next k
+// are loaded while this one's fused multiply-adds issue.
+template <bool kExact, bool kFull>
+__device__ __forceinline__ void rt_chunk(const int16_t* __restrict__ X, const double* __restrict__ Wd,
+                                         int n, int ne, double (&acc)[kRtTokPerWarp][kRtExpPerWarp]) {
+    const int lane = threadIdx.x & 31;
+    int xs[kRtTokPerWarp];
+    double wv[kRtExpPerWarp];
+#pragma unroll
+    for (int t = 0; t < kRtTokPerWarp; ++t) xs[t] = X[t * kRtK + lane];
+#pragma unroll
+    for (int i = 0; i < kRtExpPerWarp; ++i)
+        wv[i] = kFull || i < ne ? Wd[kRtEStride * i * kRtK + lane] : 0.0;
+#pragma unroll 1
+    for (int k = lane; k < n; k += 32) {
+        double xv[kRtTokPerWarp], wc[kRtExpPerWarp];
+#pragma unroll
+        for (int t = 0; t < kRtTokPerWarp; ++t) {
+            xv[t] = rt_x_scaled(xs[t]);
+            if (kExact && (xs[t] & 0x7f80) == 0x7f80)
+                xv[t] = (double)bf16_bits_to_f32((uint16_t)xs[t]);  // inf or NaN: unscaled is exact
+        }
+#pragma unroll
+        for (int i = 0; i < kRtExpPerWarp; ++i) wc[i] = wv[i];
+        const int kn = k + 32;
+        if (kn < n) {
+#pragma unroll
+            for (int t = 0; t < kRtTokPerWarp; ++t) xs[t] = X[t * kRtK + kn];
+#pragma unroll
+            for (int i = 0; i < kRtExpPerWarp; ++i)
+                if (kFull || i < ne) wv[i] = Wd[kRtEStride * i * kRtK + kn];
+        }
+#pragma unroll
+        for (int i = 0; i < kRtExpPerWarp; ++i)
+            if (kFull || i < ne)
+#pragma unroll
+                for (int t = 0; t < kRtTokPerWarp; ++t) acc[t][i] = fma(xv[t], wc[i], acc[t][i]);
+    }
+}
+
+// The halving tree p_j += p_{j+o} (o = 16 ... 1) of all the warp's sums at
+// once: at each step a lane keeps half of its sums and hands the other half
+// to lane ^ o, which adds them to its own (addition is commutative, so each
+// pair is summed exactly as in the one-sum-at-a-time tree).  Afterwards lane
+// L holds the sums q = kRtSums * L + m, m < kRtSums (q = token * experts per
+// warp + expert slot), in v[m].
+__device__ __forceinline__ void rt_tree(double (&v)[kRtTokPerWarp * kRtExpPerWarp]) {
+    const int lane = threadIdx.x & 31;
+    constexpr int kAll = kRtTokPerWarp * kRtExpPerWarp;
+#pragma unroll
+    for (int o = 16, half = kAll / 2; o >= 1; o >>= 1, half >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int m = 0; m < half; ++m) {
+            const double keep = upper ? v[m + half] : v[m];
+            const double send = upper ? v[m] : v[m + half];
+            v[m] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kRtWarps * 32, 1)
     k_route_tiles(const uint16_t* __restrict__ x, int64_t T, int64_t d, const float* __restrict__ wr,
                   const float* __restrict__ bias, int E, int top_k, int renorm,
                   int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ logits) {
     extern __shared__ __align__(16) uint8_t tile_smem[];
-    __shared__ float s_logit[kTileTok][kMaxE];
-    float* const sw0 = reinterpret_cast<float*>(tile_smem);
-    uint16_t* const sx0 = reinterpret_cast<uint16_t*>(tile_smem + kTileWBytes);
-    const size_t buf_bytes = kTileWBytes + kTileXBytes;
-    auto sw = [&](int b) { return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sw0) + b * buf_bytes); };
-    auto sx = [&](int b) {
-        return reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(sx0) + b * buf_bytes);
+    auto w_raw = [&](int s) { return reinterpret_cast<float*>(tile_smem + s * kRtStageBytes); };
+    auto x_raw = [&](int s) {
+        return reinterpret_cast<int16_t*>(tile_smem + s * kRtStageBytes + kRtWRawBytes);
+    };
+    auto w64 = [&](int b) {
+        return reinterpret_cast<double*>(tile_smem + kRtStages * kRtStageBytes + b * kRtW64Bytes);
+    };
+    auto s_logit = [&](int b) {
+        return reinterpret_cast<float*>(tile_smem + kRtStages * kRtStageBytes + 2 * kRtW64Bytes +
+                                        b * kRtLogitBytes);
     };
     pdl_wait();  // the previous step may still read ids and gates
     pdl_launch_dependents();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int tg = warp / kTileExpPerWarp, eg = warp % kTileExpPerWarp;
-    const int nchunks = (int)((d + kTileChunk - 1) / kTileChunk);
-    for (int64_t t0 = (int64_t)blockIdx.x * kTileTok; t0 < T; t0 += (int64_t)gridDim.x * kTileTok) {
-        for (int e0 = 0; e0 < E; e0 += kGroupE) {
-            // copies of chunk c into buffer b: the group's router rows and the
-            // tokens' rows (tokens past T repeat the last one; never written)
-            auto stage = [&](int c, int b) {
-                const int64_t base = (int64_t)c * kTileChunk;
-                const int n = (int)(d - base < kTileChunk ? d - base : (int64_t)kTileChunk);
-                const int wu = n / 4, xu = n / 8;  // 16-byte units per row
-                float* w_dst = sw(b);
-                uint16_t* x_dst = sx(b);
-                for (int i = threadIdx.x; i < kGroupE * wu; i += blockDim.x) {
-                    const int r = i / wu, u = i - r * wu;
-                    if (e0 + r < E)
-                        cp_async_16(w_dst + r * kTileChunk + 4 * u, wr + (int64_t)(e0 + r) * d + base + 4 * u, 16);
-                }
-                for (int i = threadIdx.x; i < kTileTok * xu; i += blockDim.x) {
-                    const int r = i / xu, u = i - r * xu;
-                    const int64_t tok = t0 + r < T ? t0 + r : T - 1;
-                    cp_async_16(x_dst + r * kTileChunk + 8 * u, x + tok * d + base + 8 * u, 16);
-                }
-                cp_async_commit();
-            };
-            double acc[kTileTokPerWarp][kTileExpPerWarp];
-#pragma unroll
-            for (int t = 0; t < kTileTokPerWarp; ++t)
-#pragma unroll
-                for (int i = 0; i < kTileExpPerWarp; ++i) acc[t][i] = 0.0;
-            stage(0, 0);
-            for (int c = 0; c < nchunks; ++c) {
-                if (c + 1 < nchunks) {
-                    stage(c + 1, (c + 1) & 1);
-                    cp_async_wait<1>();
-                } else {
-                    cp_async_wait<0>();
-                }
-                __syncthreads();
-                const float* W = sw(c & 1);
-                const uint16_t* X = sx(c & 1) + tg * kTileTokPerWarp * kTileChunk;
-                const int n = (int)(d - (int64_t)c * kTileChunk < kTileChunk ? d - (int64_t)c * kTileChunk
-                                                                            : (int64_t)kTileChunk);
-#pragma unroll 2
-                for (int k = lane; k < n; k += 32) {
-                    double xv[kTileTokPerWarp];
-#pragma unroll
-                    for (int t = 0; t < kTileTokPerWarp; ++t)
-                        xv[t] = (double)bf16_bits_to_f32(X[t * kTileChunk + k]);
-#pragma unroll
-                    for (int i = 0; i < kTileExpPerWarp; ++i) {
-                        const int e = eg + kTileExpPerWarp * i;
-                        if (e0 + e < E) {
-                            const double w = (double)W[e * kTileChunk + k];
-#pragma unroll
-                            for (int t = 0; t < kTileTokPerWarp; ++t) acc[t][i] = fma(xv[t], w, acc[t][i]);
-                        }
-                    }
-                }
-                __syncthreads();  // buffer c & 1 is refilled for chunk c + 2
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tg = warp / kRtEStride, eq = warp % kRtEStride;
+    const int nch = (int)((d + kRtK - 1) / kRtK);
+    const int ngroups = (E + kGroupE - 1) / kGroupE;
+    const int64_t ntiles = (T + kRtTok - 1) / kRtTok;
+    const int64_t my_tiles = ntiles > blockIdx.x ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int64_t U = my_tiles * ngroups * nch;  // (tile, group, chunk) units of this CTA
+    // a unit's place, advanced one unit at a time (no divisions)
+    struct Unit {
+        int tile_i, g, c;
+        __device__ void next(int nch_, int ngroups_) {
+            if (++c == nch_) {
+                c = 0;
+                if (++g == ngroups_) { g = 0; ++tile_i; }
             }
-#pragma unroll
-            for (int t = 0; t < kTileTokPerWarp; ++t)
-#pragma unroll
-                for (int i = 0; i < kTileExpPerWarp; ++i) {
-                    double v = acc[t][i];
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-                    const int e = e0 + eg + kTileExpPerWarp * i;
-                    if (lane == 0 && e < E)
-                        s_logit[tg * kTileTokPerWarp + t][e] =
-                            __double2float_rn(v + (bias ? (double)bias[e] : 0.0));
-                }
         }
-        __syncthreads();
-        for (int r = warp; r < kTileTok; r += kTileWarps)
-            if (t0 + r < T) warp_select_topk(s_logit[r], t0 + r, E, top_k, renorm, ids, gates, logits);
-        __syncthreads();
+    };
+    auto t0_of = [&](const Unit& r) { return ((int64_t)blockIdx.x + (int64_t)r.tile_i * gridDim.x) * kRtTok; };
+    auto n_of = [&](const Unit& r) {
+        const int64_t base = (int64_t)r.c * kRtK;
+        return (int)(d - base < kRtK ? d - base : (int64_t)kRtK);
+    };
+    auto rows_of = [&](const Unit& r) { return E - r.g * kGroupE < kGroupE ? E - r.g * kGroupE : kGroupE; };
+    // copies of unit u (at r) into stage u % kRtStages (tokens past T repeat
+    // the last one; their logits are never written); one commit group per
+    // unit, empty past the end, so the group count stays uniform
+    auto stage = [&](int64_t u, const Unit& r) {
+        if (u < U) {
+            const int s = (int)(u % kRtStages);
+            const int64_t base = (int64_t)r.c * kRtK, t0 = t0_of(r);
+            const int n = n_of(r), rows = rows_of(r), e0 = r.g * kGroupE;
+            float* wd = w_raw(s);
+            int16_t* xd = x_raw(s);
+            for (int i = tid; i < kGroupE * (kRtK / 4); i += kRtWarps * 32) {
+                const int row = i / (kRtK / 4), p = i % (kRtK / 4);
+                if (row < rows && 4 * p < n)
+                    cp_async_16(wd + row * kRtK + 4 * p, wr + (int64_t)(e0 + row) * d + base + 4 * p, 16);
+            }
+            for (int i = tid; i < kRtTok * (kRtK / 8); i += kRtWarps * 32) {
+                const int row = i / (kRtK / 8), p = i % (kRtK / 8);
+                const int64_t tok = t0 + row < T ? t0 + row : T - 1;
+                if (8 * p < n) cp_async_16(xd + row * kRtK + 8 * p, x + tok * d + base + 8 * p, 16);
+            }
+        }
+        cp_async_commit();
+    };
+    // piece j (0 .. 2 kRtPrep - 1) of the preparation of unit u (at r): the
+    // first kRtPrep scale the thread's share of the router rows into
+    // w64[u & 1], the others look for an all-ones exponent in its share of the
+    // token rows (returned as nonzero bits)
+    auto prep = [&](int64_t u, const Unit& r, int j) -> uint32_t {
+        const int s = (int)(u % kRtStages);
+        const int n = n_of(r);
+        if (j < kRtPrep) {
+            const int f = tid + j * kRtWarps * 32;  // float4 index in [16][kRtK / 4]
+            const int row = f / (kRtK / 4), k = 4 * (f % (kRtK / 4));
+            if (row < rows_of(r) && k < n) {
+                const uint4 b = *reinterpret_cast<const uint4*>(w_raw(s) + row * kRtK + k);
+                double* dst = w64(u & 1) + row * kRtK + k;
+                *reinterpret_cast<double2*>(dst) = make_double2(rt_w_scaled(b.x), rt_w_scaled(b.y));
+                *reinterpret_cast<double2*>(dst + 2) = make_double2(rt_w_scaled(b.z), rt_w_scaled(b.w));
+            }
+            return 0u;
+        }
+        const int f = tid + (j - kRtPrep) * kRtWarps * 32;  // uint4 index in [32][kRtK / 8]
+        const int row = f / (kRtK / 8), k = 8 * (f % (kRtK / 8));
+        if (k >= n) return 0u;
+        const uint4 b = *reinterpret_cast<const uint4*>(x_raw(s) + row * kRtK + k);
+        uint32_t bad = ((b.x & 0x7f807f80u) + 0x00800080u) | ((b.y & 0x7f807f80u) + 0x00800080u) |
+                       ((b.z & 0x7f807f80u) + 0x00800080u) | ((b.w & 0x7f807f80u) + 0x00800080u);
+        return bad & 0x80008000u;
+    };
+
+    double acc[kRtTokPerWarp][kRtExpPerWarp];
+    Unit st{0, 0, 0};  // the next unit to stage
+    for (int s = 0; s < kRtStages; ++s) {
+        stage(s, st);
+        st.next(nch, ngroups);
     }
+    cp_async_wait<kRtStages - 2>();  // units 0 and 1 have landed
+    __syncthreads();
+    int exact = 0;
+    Unit r{0, 0, 0};
+    if (U > 0) {
+        uint32_t bad = 0;
+        for (int j = 0; j < 2 * kRtPrep; ++j) bad |= prep(0, r, j);
+        exact = __syncthreads_or(bad != 0);
+    }
+    for (int64_t u = 0; u < U; ++u) {
+        // here: w64[u & 1] holds unit u's scaled router rows, `exact` says
+        // whether its token rows hold an inf or NaN, and unit u + 1 has landed
+        if (r.c == 0) {
+#pragma unroll
+            for (int t = 0; t < kRtTokPerWarp; ++t)
+#pragma unroll
+                for (int i = 0; i < kRtExpPerWarp; ++i) acc[t][i] = 0.0;
+        }
+        const int first = r.g * kGroupE + eq;  // the warp's first expert in this group
+        const int avail = first < E ? (E - first + kRtEStride - 1) / kRtEStride : 0;
+        const int ne = avail < kRtExpPerWarp ? avail : kRtExpPerWarp;
+        const int n = n_of(r);
+        const int16_t* X = x_raw((int)(u % kRtStages)) + tg * kRtTokPerWarp * kRtK;
+        const double* Wd = w64(u & 1) + eq * kRtK;
+        if (ne == kRtExpPerWarp) {
+            if (exact) rt_chunk<true, true>(X, Wd, n, ne, acc);
+            else rt_chunk<false, true>(X, Wd, n, ne, acc);
+        } else {
+            if (exact) rt_chunk<true, false>(X, Wd, n, ne, acc);
+            else rt_chunk<false, false>(X, Wd, n, ne, acc);
+        }
+        Unit rn = r;
+        rn.next(nch, ngroups);
+        uint32_t bad = 0;
+        if (u + 1 < U)
+            for (int j = 0; j < 2 * kRtPrep; ++j) bad |= prep(u + 1, rn, j);
+        const bool last_chunk = r.c == nch - 1;
+        if (last_chunk) {
+            double v[kRtTokPerWarp * kRtExpPerWarp];
+#pragma unroll
+            for (int t = 0; t < kRtTokPerWarp; ++t)
+#pragma unroll
+                for (int i = 0; i < kRtExpPerWarp; ++i) v[t * kRtExpPerWarp + i] = acc[t][i];
+            rt_tree(v);
+            float* sl = s_logit(r.tile_i & 1);
+#pragma unroll
+            for (int m = 0; m < kRtSums; ++m) {
+                const int q = kRtSums * lane + m;
+                const int t = q / kRtExpPerWarp, i = q % kRtExpPerWarp;
+                const int e = first + kRtEStride * i;
+                if (e < E)
+                    sl[(tg * kRtTokPerWarp + t) * kMaxE + e] =
+                        __double2float_rn(v[m] + (bias ? (double)bias[e] : 0.0));
+            }
+        }
+        cp_async_wait<1>();  // unit u + 2 has landed
+        exact = __syncthreads_or(bad != 0);
+        stage(u + kRtStages, st);  // into the stage unit u used
+        st.next(nch, ngroups);
+        if (last_chunk && r.g == ngroups - 1) {
+            const float* sl = s_logit(r.tile_i & 1);
+            const int64_t t0 = t0_of(r);
+            for (int row = warp; row < kRtTok; row += kRtWarps)
+                if (t0 + row < T)
+                    warp_select_topk(sl + row * kMaxE, t0 + row, E, top_k, renorm, ids, gates, logits);
+        }
+        r = rn;
+    }
+    cp_async_wait<0>();
 }
 
 }  // namespace
@@ -452,7 +628,7 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
     const bool norm = gamma_bf16 != nullptr;
     // Few tokens: a cluster of 4 CTAs per token, the RMSNorm (if any) fused in
     // front of the logits (or, for very wide rows, a 16-warp CTA streaming the
-    // router rows in chunks); many tokens: 16 tokens per 8-warp CTA with the
+    // router rows in chunks); many tokens: 32 tokens per 8-warp CTA with the
     // rows staged in shared memory (k_route_tiles).  Outside the fused kernel the
     // RMSNorm runs first, into y, and the router reads y.
     const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
@@ -481,13 +657,13 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
             (const uint16_t*)xr, d, w_router, bias, E, top_k, renorm, ids, gates, logits);
         note_launch();
     } else {
-        int64_t blocks = (T + kTileTok - 1) / kTileTok;
-        const int64_t cap = (int64_t)num_sms * 2;  // one wave: two CTAs per SM
+        int64_t blocks = (T + kRtTok - 1) / kRtTok;
+        const int64_t cap = (int64_t)num_sms;  // one CTA per SM (208 KB of shared memory)
         if (blocks > cap) blocks = cap;
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_tiles, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTileSmem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(k_route_tiles, dim3((unsigned)blocks), dim3(kTileWarps * 32), kTileSmem,
+        return launch_pdl(k_route_tiles, dim3((unsigned)blocks), dim3(kRtWarps * 32), kTileSmem,
                           stream, (const uint16_t*)xr, T, d, w_router, bias, E, top_k, renorm, ids,
                           gates, logits);
     }

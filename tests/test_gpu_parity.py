@@ -138,6 +138,48 @@ def test_route_top1_and_ties():
     assert idz.cpu().numpy().tolist() == [[0, 1]] * 4 and bool((gz == 0.5).all())
 
 
+def test_route_many_tokens_special_values():
+    # Many tokens (the tiled kernel) with the values its exact rescaling of the
+    # products has to get right: zero, subnormal, infinite and NaN token values
+    # (one infinity only in the second 256-wide chunk), zero and subnormal router
+    # weights, weights at the top of the fp32 range, and a ragged last chunk.
+    T, d, E = 1300, 576, 16
+    x = synth.normal_bf16_gpu(21, synth.X, 1.0, (T, d))
+    wr = synth.normal_f32_gpu(22, synth.WR, 0.02, (E, d))
+    xi = x.view(torch.int16)
+    x[5] = 0.0
+    xi[6, 1::2] = -32768                                  # -0.0
+    sub = torch.arange(1, 128, dtype=torch.int16, device="cuda")
+    xi[7, :127] = sub                                     # bf16 subnormals
+    xi[7, 127:254] = sub | -32768
+    xi[7, 254:] = 0
+    x[9, 100] = float("inf")
+    x[11, 3] = float("nan")
+    x[13, 10], x[13, 200] = float("-inf"), float("inf")
+    x[15, 300] = float("inf")                             # second chunk only
+    x[1299, 570] = float("-inf")                          # last token, ragged chunk
+    wr[2] = 0.0
+    wr[4, ::3] = 1.0e-40                                  # fp32 subnormals
+    wr[4, 1::3] = -3.0e-45
+    x[:, [5, 7, 17]] *= 0.25                             # keeps the logits below the fp32 limit
+    wr[6, 5], wr[8, 7], wr[9, 17] = 3.0e38, -3.3e38, 2.0 ** 127
+    ids, g, logits = jm.jmoe_route(x, wr, 2, None, want_logits=True)
+    torch.cuda.synchronize()
+    lo, io, go = oracle.route(x.view(torch.int16).cpu().numpy().view(np.uint16),
+                              wr.cpu().numpy(), 2, None)
+    lg = logits.cpu().numpy()
+    nan = np.isnan(lo)
+    assert nan[11].all() and not nan[5].any() and not nan[7].any()
+    # NaN payloads are not part of the method; where the logit is a number it
+    # must match bit for bit
+    assert np.array_equal(np.isnan(lg), nan)
+    assert np.array_equal(lg[~nan].view(np.uint32), lo[~nan].view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    fin = np.isfinite(go).all(axis=1)
+    assert fin.sum() >= T - 5
+    assert np.abs(g.cpu().numpy().astype(np.float64)[fin] - go[fin]).max() <= 1e-6
+
+
 # ----------------------------------------------------------------------------- permutation
 
 

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_finalize(const float* Y, int64_t T, int64_t d, int top_k, int E,
                             const int32_t* ids, void* out, int num_sms, cudaStream_t stream) {
+    if (T <= 0) return cudaSuccess;
     const int64_t cap = (int64_t)num_sms * 8;  // 8 CTAs of 256 threads per SM
     k_finalize<<<(unsigned)(T < cap ? T : cap), 256, 0, stream>>>(Y, T, d, top_k, E, ids,
                                                                  static_cast<uint16_t*>(out));

@@ -69,7 +69,7 @@ class ClockSampler(threading.Thread):
     NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, torch_device: int, period_s: float = 0.02):
+    def __init__(self, torch_device: int, period_s: float = 0.002):
         super().__init__(daemon=True)
         self.period = period_s
         self.samples = []

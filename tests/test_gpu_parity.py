@@ -423,16 +423,27 @@ def test_token_permutation_and_determinism(path):
     assert torch.equal(outp, out[tp])
 
 
-def test_invalid_expert_id_sets_device_error_word():
+@pytest.mark.parametrize("path", [jm.JMOE_PATH_DECODE, jm.JMOE_PATH_PREFILL])
+def test_invalid_expert_id_sets_device_error_word(path):
+    # A slot whose expert id is out of range takes no part in the layer: the
+    # device error word is raised, and the token keeps its other slots (the
+    # same result as a valid slot with gate 0, up to the order of the rows)
     assert jm.jmoe_last_error() in (jm.JMOE_OK, jm.JMOE_EDEVICE)
     dev = DeviceLayer(Workload("bad", 12, 8, 256, 512))
     ids = torch.full((8, 2), 1, dtype=torch.int32, device="cuda")
+    ids[:, 0] = torch.arange(8, dtype=torch.int32, device="cuda") % 4 + 2
     ids[3, 1] = 99
     g = torch.full((8, 2), 0.5, dtype=torch.float32, device="cuda")
-    out = jm.jmoe_forward(dev.desc(jm.JMOE_PATH_DECODE), dev.x, ids, g)
+    out = jm.jmoe_forward(dev.desc(path), dev.x, ids, g)
     assert jm.jmoe_last_error() == jm.JMOE_EDEVICE
     assert jm.jmoe_last_error() == jm.JMOE_OK  # cleared by the read
     assert bool(torch.isfinite(out.float()).all())
+    ids_ok, g_ok = ids.clone(), g.clone()
+    ids_ok[3, 1], g_ok[3, 1] = 1, 0.0
+    ref = jm.jmoe_forward(dev.desc(path), dev.x, ids_ok, g_ok)
+    torch.cuda.synchronize()
+    assert jm.jmoe_last_error() == jm.JMOE_OK
+    assert_close(bf16_to_f64(out), bf16_to_f64(ref), "invalid slot left out")
 
 
 @pytest.mark.parametrize("path,expected", [(jm.JMOE_PATH_DECODE, 6), (jm.JMOE_PATH_PREFILL, 5)])

@@ -180,6 +180,44 @@ def test_route_many_tokens_special_values():
     assert np.abs(g.cpu().numpy().astype(np.float64)[fin] - go[fin]).max() <= 1e-6
 
 
+@pytest.mark.parametrize("T,d", [(8, 576), (4, 12288)], ids=["cluster", "wide_rows"])
+def test_route_few_tokens_special_values(T, d):
+    # The same special values through the few-token routers (one token row
+    # each: zeros and subnormals, +inf, NaN, -inf with +inf, ...), against the
+    # oracle: logits bit for bit where they are numbers, NaN where it is NaN.
+    E = 16
+    x = synth.normal_bf16_gpu(23, synth.X, 1.0, (T, d))
+    wr = synth.normal_f32_gpu(24, synth.WR, 0.02, (E, d))
+    xi = x.view(torch.int16)
+    sub = torch.arange(1, 128, dtype=torch.int16, device="cuda")
+    xi[0, :127] = sub
+    xi[0, 127:254] = sub | -32768
+    xi[0, 254:] = 0
+    x[1, d - 3] = float("inf")
+    x[2, 5] = float("nan")
+    x[3, 7], x[3, d // 2] = float("-inf"), float("inf")
+    if T > 4:
+        x[4] = 0.0
+        xi[5, 1::2] = -32768
+    wr[2] = 0.0
+    wr[4, ::3] = 1.0e-40
+    wr[4, 1::3] = -3.0e-45
+    x[:, [9, 11]] *= 0.25
+    wr[6, 9], wr[9, 11] = 3.0e38, 2.0 ** 127
+    ids, g, logits = jm.jmoe_route(x, wr, 2, None, want_logits=True)
+    torch.cuda.synchronize()
+    lo, io, go = oracle.route(x.view(torch.int16).cpu().numpy().view(np.uint16),
+                              wr.cpu().numpy(), 2, None)
+    lg = logits.cpu().numpy()
+    nan = np.isnan(lo)
+    assert nan[2].all() and not nan[0].any()
+    assert np.array_equal(np.isnan(lg), nan)
+    assert np.array_equal(lg[~nan].view(np.uint32), lo[~nan].view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    fin = np.isfinite(go).all(axis=1)
+    assert fin[0] and np.abs(g.cpu().numpy().astype(np.float64)[fin] - go[fin]).max() <= 1e-6
+
+
 # ----------------------------------------------------------------------------- permutation
 
 

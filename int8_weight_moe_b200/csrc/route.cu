@@ -620,6 +620,26 @@ cudaError_t launch_rmsnorm(const void* x_bf16, int64_t T, int64_t d, const void*
     return cudaGetLastError();
 }
 
+// Whether the tiled kernel beats the per-token clusters for T tokens of width
+// d.  Measured on the B200 (router alone, 16 experts): a wave of clusters (as
+// many four-CTA clusters as fit at once, shared memory deciding how many CTAs
+// share an SM) takes about 5.8 + 0.4 d/1024 us, a round of 32-token tiles (one
+// per SM) about 4 + 0.0151 d us.  d_model 4096: clusters 0.039 ms at 512
+// tokens and 0.069 ms at 1024, tiles 0.070 ms from 1184 to 4736 tokens;
+// d_model 8192: clusters 0.071 ms at 256 tokens, 0.131 at 512, 0.250 at 1024,
+// tiles 0.125 ms.  More experts scale both alike.
+static bool route_tiles_cheaper(int64_t T, int64_t d, size_t cluster_smem, int num_sms) {
+    constexpr int64_t kSmemPerSm = 227 * 1024;
+    int64_t per_sm = kSmemPerSm / (int64_t)(cluster_smem + 1024);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t at_once = (int64_t)num_sms * per_sm;
+    const int64_t waves = (T * kRouteCluster + at_once - 1) / at_once;
+    const int64_t rounds = (T + (int64_t)kRtTok * num_sms - 1) / ((int64_t)kRtTok * num_sms);
+    const double cluster_us = (double)waves * (5.8 + 0.4 * (double)d / 1024.0);
+    const double tiles_us = (double)rounds * (4.0 + 0.0151 * (double)d);
+    return tiles_us < cluster_us;
+}
+
 cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const void* gamma_bf16,
                               float eps, void* y_bf16, const float* w_router, const float* bias,
                               int E, int top_k, int renorm, int32_t* ids, float* gates,
@@ -627,13 +647,16 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
     if (T == 0) return cudaSuccess;
     const bool norm = gamma_bf16 != nullptr;
     // Few tokens: a cluster of 4 CTAs per token, the RMSNorm (if any) fused in
-    // front of the logits (or, for very wide rows, a 16-warp CTA streaming the
-    // router rows in chunks); many tokens: 32 tokens per 8-warp CTA with the
-    // rows staged in shared memory (k_route_tiles).  Outside the fused kernel the
-    // RMSNorm runs first, into y, and the router reads y.
+    // front of the logits, while that is cheaper than the tiles (or, for rows too
+    // wide for the clusters, a 16-warp CTA per token streaming the router rows in
+    // chunks); otherwise 32 tokens per 8-warp CTA with the rows staged in shared
+    // memory (k_route_tiles).  Outside the fused kernel the RMSNorm runs first,
+    // into y, and the router reads y.
     const size_t csmem = (size_t)kExpertsPerCta * d * sizeof(float) + (size_t)d * sizeof(uint16_t);
     const size_t smem = (size_t)kGroupE * kChunkSmem + (size_t)d * sizeof(uint16_t);
-    if (T < (int64_t)num_sms * 8 && csmem <= kClusterMaxSmem && T * kRouteCluster < (1LL << 31)) {
+    const bool few = T < (int64_t)num_sms * 8;
+    const bool cluster_fits = csmem <= kClusterMaxSmem && T * kRouteCluster < (1LL << 31);
+    if (few && cluster_fits && !route_tiles_cheaper(T, d, csmem, num_sms)) {
         const auto kernel = norm ? k_route_cluster<true> : k_route_cluster<false>;
         const cudaError_t e = cudaFuncSetAttribute(
             kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kClusterMaxSmem);
@@ -649,7 +672,7 @@ cudaError_t launch_norm_route(const void* x_bf16, int64_t T, int64_t d, const vo
         if (e != cudaSuccess) return e;
         xr = y_bf16;
     }
-    if (T < (int64_t)num_sms * 8 && smem <= kWideMaxSmem) {
+    if (few && !cluster_fits && smem <= kWideMaxSmem) {
         const cudaError_t e = cudaFuncSetAttribute(
             k_route_wide, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWideMaxSmem);
         if (e != cudaSuccess) return e;

@@ -118,6 +118,29 @@ def test_route_wide_rows_bitexact(T, d, E):
     assert np.abs(g.cpu().numpy().astype(np.float64) - go).max() <= 1e-6
 
 
+@pytest.mark.parametrize("norm", [False, True], ids=["route", "rmsnorm_route"])
+def test_route_mid_tokens_wide_rows_bitexact(norm):
+    # 800 tokens of width 8192: fewer than the tiled kernel's usual threshold,
+    # but the tiles are cheaper than one cluster per token at this width
+    T, d, E = 800, 8192, 16
+    x = synth.normal_bf16_gpu(25, synth.X, 1.0, (T, d))
+    wr = synth.normal_f32_gpu(26, synth.WR, 0.02, (E, d))
+    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+    if norm:
+        gam = (synth.normal_bf16_gpu(27, synth.X, 0.25, (d,)).float() + 1.0).to(torch.bfloat16)
+        xn, ids, g, logits = jm.jmoe_rmsnorm_route(x, gam, 1e-6, wr, 2, want_logits=True)
+        torch.cuda.synchronize()
+        xb = oracle.rmsnorm(xb, gam.view(torch.int16).cpu().numpy().view(np.uint16), 1e-6)
+        assert np.array_equal(xn.view(torch.int16).cpu().numpy().view(np.uint16), xb)
+    else:
+        ids, g, logits = jm.jmoe_route(x, wr, 2, None, want_logits=True)
+        torch.cuda.synchronize()
+    lo, io, go = oracle.route(xb, wr.cpu().numpy(), 2, None)
+    assert np.array_equal(logits.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(ids.cpu().numpy(), io)
+    assert np.abs(g.cpu().numpy().astype(np.float64) - go).max() <= 1e-6
+
+
 def test_route_top1_and_ties():
     d, E = 256, 16
     x = synth.normal_bf16_gpu(3, synth.X, 1.0, (40, d))

@@ -61,8 +61,9 @@ typedef enum {
 
 /* Which expert-GEMM kernels jmoe_forward / jmoe_mlp_forward use. */
 typedef enum {
-    JMOE_PATH_AUTO = 0,    /* decode kernels below max(128, 20 E) assignments (about 20 tokens
-                              per expert), else tensor-core kernels */
+    JMOE_PATH_AUTO = 0,    /* decode kernels below max(128, k E) assignments, k = 26 per
+                              expert at d_model <= 4096, 21 at >= 8192 (linear in between),
+                              else tensor-core kernels */
     JMOE_PATH_DECODE = 1,  /* bandwidth-bound GEMV-like kernels (any size; slow when large) */
     JMOE_PATH_PREFILL = 2  /* tcgen05 / TMEM grouped GEMM kernels */
 } jmoe_path;

@@ -38,15 +38,23 @@ void take_stall(int& target, long long& wait_cycles) {
 }
 
 // The automatic path: the decode (GEMV-like) kernels while there are fewer
-// than max(128, 20 E) token->expert assignments, i.e. about 20 tokens per
-// expert; the tcgen05 grouped GEMM from there on.  The decode kernels re-read
-// an expert's weights (mostly from L2) for every pass of 8 of its tokens; the
-// grouped GEMM streams them once but pads each expert's rows to 128.  Measured
-// on the B200 at d_model 4096, d_ff 14336, 16 experts, top-2: 256 assignments
-// took 1.03 ms on the decode path against 1.29 ms, 384 took 1.38 ms against
-// 1.26 ms.  With one expert (the dense MLP) the bound stays 128.
+// than max(128, k E) token->expert assignments, the tcgen05 grouped GEMM from
+// there on.  The decode kernels re-read an expert's weights (mostly from L2)
+// for every pass of 8 of its tokens; the grouped GEMM streams them once but
+// pads each expert's rows to 128, so its time is flat at small A.  k falls
+// with the width: 26 per expert at d_model 4096 or less, 21 at 8192 or more,
+// linear in between.  Measured on the B200 (16 experts, top-2, the forward
+// alone): d_model 4096, d_ff 14336: decode 1.167 / 1.313 / 1.724 ms at 320 /
+// 384 / 512 assignments against 1.392 / 1.400 / 1.404 ms; d_model 8192, d_ff
+// 24576: decode 4.352 / 4.955 ms at 320 / 384 against 4.635 / 4.537 ms.  With
+// one expert (the dense MLP) the bound stays 128.
 constexpr int64_t kDecodeMinAssignments = 128;
-constexpr int64_t kDecodeTokensPerExpert = 20;
+
+int64_t decode_tokens_per_expert(int64_t d) {
+    if (d <= 4096) return 26;
+    if (d >= 8192) return 21;
+    return 26 - 5 * (d - 4096) / 4096;
+}
 
 int current_device() {
     int dev = 0;
@@ -200,12 +208,11 @@ Workspace plan(int64_t T, int64_t A, int E, int64_t d, int64_t f, bool prefill) 
     return w;
 }
 
-bool use_prefill(int32_t path, int64_t A, int E) {
+bool use_prefill(int32_t path, int64_t A, int E, int64_t d) {
     if (path == JMOE_PATH_DECODE) return false;
     if (path == JMOE_PATH_PREFILL) return true;
-    const int64_t bound = kDecodeTokensPerExpert * E > kDecodeMinAssignments
-                              ? kDecodeTokensPerExpert * E
-                              : kDecodeMinAssignments;
+    const int64_t per_expert = decode_tokens_per_expert(d) * E;
+    const int64_t bound = per_expert > kDecodeMinAssignments ? per_expert : kDecodeMinAssignments;
     return A >= bound && jmoe::prefill_available();
 }
 
@@ -244,7 +251,7 @@ jmoe_status run_experts(const jmoe_moe_desc* desc, const void* x, int64_t T,
                         size_t ws_bytes, bool dense, cudaStream_t stream) {
     const int E = desc->E, k = desc->top_k;
     const int64_t A = T * k, d = desc->d_model, f = desc->d_ff;
-    const bool prefill = use_prefill(desc->path, A, desc->E);
+    const bool prefill = use_prefill(desc->path, A, desc->E, desc->d_model);
     if (prefill && !jmoe::prefill_available()) return JMOE_EUNSUPPORTED;
     const Workspace w = plan(T, A, E, d, f, prefill);
     if (!ws || ws_bytes < w.total) return JMOE_EWORKSPACE;
@@ -429,7 +436,8 @@ jmoe_status jmoe_forward_workspace_size(const jmoe_moe_desc* desc, int64_t T, si
     if (desc->d_model % 64 || desc->d_ff % 64) return JMOE_EUNSUPPORTED;
     if (desc->path < JMOE_PATH_AUTO || desc->path > JMOE_PATH_PREFILL) return JMOE_EINVAL;
     const int64_t A = T * desc->top_k;
-    *bytes = plan(T, A, desc->E, desc->d_model, desc->d_ff, use_prefill(desc->path, A, desc->E)).total;
+    *bytes = plan(T, A, desc->E, desc->d_model, desc->d_ff,
+                  use_prefill(desc->path, A, desc->E, desc->d_model)).total;
     return JMOE_OK;
 }
 

@@ -127,6 +127,12 @@ constexpr int kChunks = kB8Bytes / 16 / kConvThreads;  // 16-byte INT8 chunks pe
 constexpr int kMaxE = 64;
 
 static_assert(kStagesB % 2 == 0 && kStages8 % 2 == 0, "converter groups alternate k-steps");
+// The converters run kStagesB k-steps into the next tile before they help
+// drain the previous one; each of those steps waits for its A copy, which the
+// A producer can issue only while the A ring has a free stage -- and stages of
+// the next tile are freed by MMAs that need the drain.  A shallower A ring
+// waits in a cycle (seen as every bounded wait running out).
+static_assert(kStagesA >= kStagesB, "the A ring must hold the steps converted before the drain");
 static_assert(kChunks * 16 * kConvThreads == kB8Bytes, "converter work split");
 
 enum Mode { kGateUp = 0, kDown = 1 };

@@ -507,6 +507,19 @@ def test_invalid_expert_id_sets_device_error_word(path):
     assert_close(bf16_to_f64(out), bf16_to_f64(ref), "invalid slot left out")
 
 
+def test_automatic_path_follows_the_measured_crossings():
+    # decode kernels below 26 assignments per expert at d_model 4096, 21 at
+    # 8192, linear in between (24 at 6144); 16 experts, top-2.  Only size
+    # queries: nothing is launched.
+    fake = 0x10000
+    for d, f, t_switch in ((4096, 14336, 208), (6144, 16384, 192), (8192, 24576, 168)):
+        desc = jm.MoeDesc(16, 2, d, f, fake, fake, fake, fake, jm.JMOE_PATH_AUTO)
+        assert not jm.uses_prefill_path(desc, t_switch - 1), (d, t_switch - 1)
+        assert jm.uses_prefill_path(desc, t_switch), (d, t_switch)
+    dense = jm.MoeDesc(1, 1, 4096, 14336, fake, fake, fake, fake, jm.JMOE_PATH_AUTO)
+    assert not jm.uses_prefill_path(dense, 127) and jm.uses_prefill_path(dense, 128)
+
+
 @pytest.mark.parametrize("path,expected", [(jm.JMOE_PATH_DECODE, 6), (jm.JMOE_PATH_PREFILL, 5)])
 def test_launch_counter_per_path(path, expected):
     # decode: grouping with fp16 token rows, gate/up GEMV, SwiGLU, fp16 hidden
